@@ -1,0 +1,90 @@
+// Internal launch interface between the C ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4kv {
+
+cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
+                                const int64_t* dst_row, uint8_t* packed, uint8_t* scales,
+                                int64_t cap_rows, int num_sms, cudaStream_t stream);
+
+// ----------------------------------------------------------------------------------------
+// Indexer scoring (Full scan or pool gather), fused with the first-level histogram of the
+// top-K select and, for the hierarchical Full layer, the block max over 8 positions.
+// ----------------------------------------------------------------------------------------
+struct IndexScoreParams {
+  const void* q;            // [B][H_I][128] e4m3 codes or bf16 bits
+  const float* w;           // [B][H_I]
+  int H_I;
+  const void* keys;         // [B][cap][128]
+  bool keys_fp8;
+  const float* key_scale;   // nullable [B][cap]
+  int64_t cap;
+  const int32_t* seq_lens;  // [B]
+  int B;
+  // pool mode (pool != nullptr): tile = 16 pool blocks of 8 rows
+  const int32_t* pool;      // [B][npb]
+  int npb;
+  // outputs
+  float* scores;            // [B][score_stride]; flat: index = position; pool: slot*8 + r
+  int64_t score_stride;
+  uint32_t* hist;           // nullable [B][4096]
+  float* bmax;              // nullable [B][bmax_stride] (flat mode only)
+  int64_t bmax_stride;
+  uint32_t* bmax_hist;      // [B][4096] when bmax != nullptr
+  uint32_t* status;         // workspace status word
+};
+cudaError_t launch_index_score(const IndexScoreParams& p, int num_sms, cudaStream_t stream);
+
+// ----------------------------------------------------------------------------------------
+// Exact top-K select over per-segment fp32 values, given the first-level histogram.
+// ----------------------------------------------------------------------------------------
+struct SelectProblem {
+  const float* values;      // [B][vstride]
+  int64_t vstride;
+  const int32_t* seq_lens;  // [B]
+  int mode;                 // 0: n = seq_len; 1: n = ceil(seq_len / 8) (block ids);
+                            // 2: n = npb*8 pool slots, position = pool[b][i/8]*8 + i%8
+  const int32_t* pool;      // mode 2
+  int npb;
+  int k;
+  uint32_t* hist;           // [B][4096], zeroed by the last CTA of each segment
+  uint32_t* counters;       // [B][4]: n_sure, n_cand, ticket, spare
+  int32_t* sure;            // [B][k]
+  int32_t* cand;            // [B][vstride]
+  int32_t* out_idx;         // [B][k]
+  float* out_score;         // nullable [B][k]
+  int slices;
+};
+cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
+                               cudaStream_t stream);
+int select_slices(int64_t n_values, int B, int num_sms);
+
+// ----------------------------------------------------------------------------------------
+// Sparse attention decode
+// ----------------------------------------------------------------------------------------
+struct AttnParams {
+  const uint16_t* q;        // [B][H][d] bf16
+  int B, H, d;
+  const uint8_t* packed;    // [B][cap][d/2]
+  const uint8_t* scales;    // [B][cap][d/16]
+  int64_t cap;
+  const int32_t* seq_lens;
+  const int32_t* idx;       // [B][top_k]
+  int top_k;
+  float sm_scale;
+  float* out;               // [B][H][d]
+  float* lse;               // nullable [B][H]
+  // split over chunks of the top_k list; partials merged by the last CTA of each (b, hg)
+  int n_chunks;
+  float* part_o;            // [B][n_hg][n_chunks][64][d]
+  float* part_ml;           // [B][n_hg][n_chunks][64][2]
+  uint32_t* tickets;        // [B][n_hg]
+  uint32_t* status;
+};
+cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream);
+int attn_chunks(int B, int H, int top_k, int num_sms);
+
+}  // namespace fp4kv

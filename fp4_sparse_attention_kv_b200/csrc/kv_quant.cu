@@ -1,0 +1,117 @@
+// kv_quant_fp4: quantize-on-write of bf16 KV rows into packed E2M1 codes + E4M3 scales.
+//
+// Method: [PyTorchKR] "DeepSeek-V4.1-Flash, KV 캐시를 토큰당 890바이트로 줄이고 …", section
+// "890바이트를 만든 나머지 절반, FP4 KV 캐시와 지속 캐시 재설계": the main KV is kept as E2M1
+// values with one E4M3 scale per 16 channels (largest magnitude 448 x 6 = 2688).
+//
+// Per 16-channel group: S = E4M3_RNE_sat(amax / 6); code = sign(x) | E2M1_RNE_sat(|x| / S).
+//
+// Exactness argument (the kernel must agree bit for bit with the exact definition):
+//  * amax / 6 is computed by an IEEE fp32 division. The exact quotient of a bf16 amax by 6
+//    is either an E4M3 rounding midpoint itself (then the division is exact) or lies at a
+//    relative distance >= 2^-14.5 from every midpoint, far beyond the 2^-24 error of the
+//    division; the hardware cvt then rounds to nearest-even and saturates at 448.
+//  * |x| / S is formed as |x| * RN(1/S) (two roundings, relative error < 2^-23) and then
+//    snapped to a multiple of 2^-16 by adding and subtracting 128. For r < 8 an exact tie
+//    r = t (t a multiple of 1/4) is recovered exactly, while a non-tie bf16/E4M3 ratio is at
+//    least 2^-10 away from every E2M1 midpoint, so the snap cannot move it across one.
+//    Ratios >= 8 saturate either way.
+//  * cvt.rn.satfinite.e2m1x2.f32 rounds to nearest-even on the code and saturates at 6.
+//  * The sign bit of x is OR-ed in separately, so -0 and negative values rounding to zero
+//    keep the sign (code 0x8).
+// Memory: one warp per row, one 16-channel group per lane: 32 B read, 8 B + 1 B written per
+// lane; a warp reads 1 KiB and writes 256 B + 32 B contiguous.
+#include "fp4kv_common.cuh"
+#include "fp4kv_launch.h"
+
+namespace fp4kv {
+
+namespace {
+
+FP4KV_DEV float snap_ratio(float r) {
+  return __fadd_rn(__fadd_rn(r, 128.0f), -128.0f);
+}
+
+// Quantize one group of 16 bf16 values held as 8 words (2 values per word, low half first).
+// Returns the 8 packed bytes (low nibble = even channel) and the scale code.
+FP4KV_DEV void quant_group(const uint32_t (&w)[8], uint2& packed, uint32_t& scale_code) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    m = max(m, w[i] & 0x7fffu);
+    m = max(m, (w[i] >> 16) & 0x7fffu);
+  }
+  const float amax = bf16_bits_to_f32(m);
+  const uint32_t sc = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+  const float S = f16_lo_to_f32(e4m3x2_to_f16x2(static_cast<uint16_t>(sc)));
+  uint32_t bytes[8];
+  if (S > 0.0f) {
+    const float inv = __frcp_rn(S);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float a0 = bf16_bits_to_f32(w[i] & 0x7fffu);
+      const float a1 = bf16_bits_to_f32((w[i] >> 16) & 0x7fffu);
+      const float r0 = snap_ratio(__fmul_rn(a0, inv));
+      const float r1 = snap_ratio(__fmul_rn(a1, inv));
+      bytes[i] = f32x2_to_e2m1x2_satfinite(r0, r1);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bytes[i] = 0;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    // sign of the even channel (bit 15) -> bit 3; odd channel (bit 31) -> bit 7
+    bytes[i] |= ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);
+  }
+  packed.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+  packed.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+  scale_code = sc;
+}
+
+__global__ void __launch_bounds__(256) k_kv_quant_fp4(const uint16_t* __restrict__ x,
+                                                      int64_t n_rows, int d, int64_t x_stride,
+                                                      const int64_t* __restrict__ dst_row,
+                                                      uint8_t* __restrict__ packed,
+                                                      uint8_t* __restrict__ scales,
+                                                      int64_t cap_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int groups = d / kGroup;
+  for (int64_t r = warp; r < n_rows; r += nwarps) {
+    const int64_t dst = dst_row ? dst_row[r] : r;
+    if (dst < 0 || dst >= cap_rows) continue;
+    const uint16_t* xr = x + r * x_stride;
+    uint8_t* pr = packed + dst * (d / 2);
+    uint8_t* sr = scales + dst * groups;
+    for (int g = lane; g < groups; g += 32) {
+      const uint4 v0 = ld_stream_v4(xr + g * kGroup);
+      const uint4 v1 = ld_stream_v4(xr + g * kGroup + 8);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint2 pk;
+      uint32_t sc;
+      quant_group(w, pk, sc);
+      *reinterpret_cast<uint2*>(pr + g * 8) = pk;
+      sr[g] = static_cast<uint8_t>(sc);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
+                                const int64_t* dst_row, uint8_t* packed, uint8_t* scales,
+                                int64_t cap_rows, int num_sms, cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t rows_per_block = threads / 32;
+  int64_t blocks = (n_rows + rows_per_block - 1) / rows_per_block;
+  const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > max_blocks) blocks = max_blocks;
+  k_kv_quant_fp4<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      x, n_rows, d, x_stride, dst_row, packed, scales, cap_rows);
+  return cudaGetLastError();
+}
+
+}  // namespace fp4kv

@@ -1,0 +1,344 @@
+// Exact top-K select per sequence: K largest fp32 values, ties to the lower position,
+// returned as positions in ascending order padded with -1.
+//
+// Used for the indexer top-K ([PyTorchKR] "DeepSeek-V4.1-Flash, KV 캐시를 토큰당 890바이트로
+// 줄이고 …", section "레이어 사이에서 캐시와 인덱스를 돌려 쓰는 CSA2": each Full or Reindex
+// layer produces its own top-K indices) and for the candidate pool (section "계층적 희소
+// 인덱서로 인덱싱 비용을 컨텍스트 길이에서 분리하기": the blocks with the highest block max).
+//
+// Values are mapped to order-preserving 32-bit keys. The scoring kernel has already built
+// a histogram of the top 12 key bits per sequence. This kernel, launched with several CTAs
+// per sequence:
+//  1. finds the digit b* of the K-th largest key from that histogram (suffix sums);
+//  2. streams its slice of the values: keys with digit > b* are certainly selected
+//     ("sure", fewer than K in total), keys with digit == b* are candidates;
+//  3. takes a ticket; the last CTA of the sequence resolves the candidates exactly with
+//     three more radix passes on the key (8+8+4 bits) and, if the K-th key is tied, radix
+//     passes on the position (lowest positions win), then bitonic-sorts the selected
+//     positions and writes them. It also zeroes the histogram and counters, leaving the
+//     workspace ready for the next call. No CTA ever waits on another.
+#include "fp4kv_common.cuh"
+#include "fp4kv_launch.h"
+
+namespace fp4kv {
+namespace {
+
+constexpr int kSelThreads = 512;
+constexpr int kMaxSel = 4096;
+constexpr int kMaxProblems = 2;
+
+struct SelectArgs {
+  SelectProblem p[kMaxProblems];
+};
+
+FP4KV_DEV int64_t n_values(const SelectProblem& P, int b) {
+  int64_t len = P.seq_lens[b];
+  if (len < 0) len = 0;
+  if (P.mode == 0) return len < P.vstride ? len : P.vstride;
+  if (P.mode == 1) {
+    const int64_t nb = (len + 7) / 8;
+    return nb < P.vstride ? nb : P.vstride;
+  }
+  return int64_t(P.npb) * 8;
+}
+
+FP4KV_DEV int64_t position_of(const SelectProblem& P, int b, int64_t i) {
+  if (P.mode != 2) return i;
+  const int64_t j = P.pool[int64_t(b) * P.npb + i / 8];
+  return j * 8 + (i % 8);
+}
+
+// Block-wide: find the digit d (scanning from the highest digit down) at which the running
+// count of `h[0..nbins)` reaches `r` (r >= 1). Returns d and the count strictly above d.
+// If the total is below r, returns d = -1 and above = total.
+__device__ void find_digit_desc(const uint32_t* h, int nbins, uint32_t r, int* d_out,
+                                uint32_t* above_out, uint32_t* s_scan) {
+  const int tid = threadIdx.x;
+  const int per = (nbins + kSelThreads - 1) / kSelThreads;
+  // thread tid owns the per-digit chunk counted from the top: digits [hi-per, hi)
+  const int hi = nbins - tid * per;
+  uint32_t sum = 0;
+  for (int d = hi - 1; d >= hi - per && d >= 0; --d) sum += h[d];
+  // inclusive scan over threads (thread 0 = highest digits)
+  const int lane = tid & 31, w = tid >> 5;
+  uint32_t x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_scan[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    uint32_t v = lane < kSelThreads / 32 ? s_scan[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < kSelThreads / 32) s_scan[32 + lane] = v;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const uint32_t incl = x + (w > 0 ? s_scan[32 + w - 1] : 0u);
+  const uint32_t excl = incl - sum;
+  const uint32_t total = s_scan[32 + kSelThreads / 32 - 1];
+  if (tid == 0) {
+    s_scan[64] = 0xffffffffu;  // digit
+    s_scan[65] = total;
+  }
+  __syncthreads();
+  if (total >= r && excl < r && incl >= r) {
+    uint32_t acc = excl;
+    for (int d = hi - 1; d >= hi - per && d >= 0; --d) {
+      if (acc + h[d] >= r) {
+        s_scan[64] = static_cast<uint32_t>(d);
+        s_scan[65] = acc;
+        break;
+      }
+      acc += h[d];
+    }
+  }
+  __syncthreads();
+  *d_out = s_scan[64] == 0xffffffffu ? -1 : static_cast<int>(s_scan[64]);
+  *above_out = s_scan[65];
+  __syncthreads();
+}
+
+// Same, scanning from the lowest digit up (used for the smallest positions among ties).
+__device__ void find_digit_asc(const uint32_t* h, int nbins, uint32_t r, int* d_out,
+                               uint32_t* below_out, uint32_t* s_val) {
+  if (threadIdx.x == 0) {
+    uint32_t acc = 0;
+    int dd = nbins - 1;
+    for (int d = 0; d < nbins; ++d) {
+      if (acc + h[d] >= r) { dd = d; break; }
+      acc += h[d];
+    }
+    s_val[0] = static_cast<uint32_t>(dd);
+    s_val[1] = acc;
+  }
+  __syncthreads();
+  *d_out = static_cast<int>(s_val[0]);
+  *below_out = s_val[1];
+  __syncthreads();
+}
+
+__device__ void bitonic_sort_u64(uint64_t* a, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool asc = (i & size) == 0;
+          const uint64_t x = a[i], y = a[j];
+          if ((x > y) == asc) { a[i] = y; a[j] = x; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Warp-aggregated append of `take` lanes' values into list[counter++]; slots at or beyond
+// `capacity` are never written (the counter still counts them).
+FP4KV_DEV void warp_append(bool take, int32_t v, uint32_t* counter, int32_t* list,
+                           uint32_t capacity) {
+  const uint32_t m = __ballot_sync(0xffffffffu, take);
+  if (m == 0) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(m)));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
+  if (take && slot < capacity) list[slot] = v;
+}
+
+__global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs args) {
+  const SelectProblem& P = args.p[blockIdx.z];
+  const int b = blockIdx.y;
+  if (static_cast<int>(blockIdx.x) >= P.slices) return;
+  // the histogram (phase 1 and the radix passes) and the selection buffer (collection and
+  // sort) are never live at the same time: they share one 32 KiB buffer
+  __shared__ uint64_t s_sel[kMaxSel];
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_sel);
+  __shared__ uint32_t s_scan[96];
+  __shared__ uint32_t s_cnt;
+  __shared__ bool s_last;
+  const int tid = threadIdx.x;
+
+  const int64_t n = n_values(P, b);
+  const float* vals = P.values + int64_t(b) * P.vstride;
+  uint32_t* hist = P.hist + int64_t(b) * kHistBins;
+  uint32_t* ctr = P.counters + int64_t(b) * 4;
+  int32_t* sure = P.sure + int64_t(b) * P.k;
+  int32_t* cand = P.cand + int64_t(b) * P.vstride;
+
+  // 1. digit of the K-th largest key
+  for (int i = tid; i < kHistBins; i += kSelThreads) s_hist[i] = __ldcg(hist + i);
+  __syncthreads();
+  int bstar;
+  uint32_t above;
+  find_digit_desc(s_hist, kHistBins, static_cast<uint32_t>(P.k), &bstar, &above, s_scan);
+  // bstar == -1: fewer than K valid values; every valid value is "sure"
+
+  // 2. filter this CTA's slice
+  const int64_t lo = n * blockIdx.x / P.slices;
+  const int64_t hi = n * (blockIdx.x + 1) / P.slices;
+  for (int64_t base = lo; base < hi; base += kSelThreads) {
+    const int64_t i = base + tid;
+    bool is_sure = false, is_cand = false;
+    if (i < hi) {
+      const float v = vals[i];
+      if (v != -INFINITY || P.mode != 2) {
+        const int digit = static_cast<int>(order_key(v) >> (32 - kHistBits));
+        is_sure = digit > bstar;
+        is_cand = digit == bstar;
+      }
+    }
+    warp_append(is_sure, static_cast<int32_t>(i), &ctr[0], sure, static_cast<uint32_t>(P.k));
+    warp_append(is_cand, static_cast<int32_t>(i), &ctr[1], cand, static_cast<uint32_t>(P.vstride));
+  }
+
+  // 3. ticket: the last CTA of this sequence finalises
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t t = atomicAdd(&ctr[2], 1u);
+    s_last = (t == static_cast<uint32_t>(P.slices - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  const uint32_t n_sure = min(__ldcg(&ctr[0]), static_cast<uint32_t>(P.k));
+  const uint32_t n_cand = min(__ldcg(&ctr[1]), static_cast<uint32_t>(P.vstride));
+  uint32_t r = static_cast<uint32_t>(P.k) > n_sure ? static_cast<uint32_t>(P.k) - n_sure : 0u;
+  bool take_all = n_cand <= r;
+  uint32_t ustar = 0;
+  int64_t pos_star = INT64_MAX;
+  if (!take_all && r > 0) {
+    // exact K-th key among the candidates: remaining 20 key bits in passes of 8, 8, 4
+    uint32_t prefix = static_cast<uint32_t>(bstar);
+    int consumed = kHistBits;
+    const int widths[3] = {8, 8, 4};
+    uint32_t cnt_eq = 0;
+    for (int pass = 0; pass < 3; ++pass) {
+      const int wbits = widths[pass];
+      const int shift = 32 - consumed - wbits;
+      const int nb = 1 << wbits;
+      for (int i = tid; i < nb; i += kSelThreads) s_hist[i] = 0;
+      __syncthreads();
+      for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+        const uint32_t key = order_key(vals[__ldcg(cand + c)]);
+        if ((key >> (shift + wbits)) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+      }
+      __syncthreads();
+      int d;
+      uint32_t ab;
+      find_digit_desc(s_hist, nb, r, &d, &ab, s_scan);
+      r -= ab;
+      cnt_eq = s_hist[d];
+      prefix = (prefix << wbits) | static_cast<uint32_t>(d);
+      consumed += wbits;
+      __syncthreads();
+    }
+    ustar = prefix;
+    if (r < cnt_eq) {
+      // lowest r positions among the keys equal to ustar: passes of 8 bits over 32 bits
+      uint64_t pprefix = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kSelThreads) s_hist[i] = 0;
+        __syncthreads();
+        for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+          const int32_t i = __ldcg(cand + c);
+          if (order_key(vals[i]) != ustar) continue;
+          const uint64_t pos = static_cast<uint64_t>(position_of(P, b, i));
+          if ((pos >> (shift + 8)) == pprefix) atomicAdd(&s_hist[(pos >> shift) & 255], 1u);
+        }
+        __syncthreads();
+        int d;
+        uint32_t below;
+        find_digit_asc(s_hist, 256, r, &d, &below, s_scan);
+        r -= below;
+        pprefix = (pprefix << 8) | static_cast<uint64_t>(d);
+      }
+      pos_star = static_cast<int64_t>(pprefix);
+    }
+  }
+
+  // collect the selected (position, value index) pairs
+  if (tid == 0) s_cnt = 0;
+  __syncthreads();
+  for (uint32_t c = tid; c < n_sure; c += kSelThreads) {
+    const int32_t i = __ldcg(sure + c);
+    const uint32_t slot = atomicAdd(&s_cnt, 1u);
+    if (slot < kMaxSel)
+      s_sel[slot] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
+  }
+  if (r > 0 || take_all) {
+    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+      const int32_t i = __ldcg(cand + c);
+      bool take = take_all;
+      const int64_t pos = position_of(P, b, i);
+      if (!take) {
+        const uint32_t key = order_key(vals[i]);
+        take = key > ustar || (key == ustar && pos <= pos_star);
+      }
+      if (take) {
+        const uint32_t slot = atomicAdd(&s_cnt, 1u);
+        if (slot < kMaxSel)
+          s_sel[slot] = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
+      }
+    }
+  }
+  __syncthreads();
+  int m = static_cast<int>(s_cnt);
+  if (m > P.k) m = P.k;
+  int npow = 1;
+  while (npow < m) npow <<= 1;
+  for (int i = m + tid; i < npow; i += kSelThreads) s_sel[i] = ~0ull;
+  __syncthreads();
+  bitonic_sort_u64(s_sel, npow);
+  int32_t* oi = P.out_idx + int64_t(b) * P.k;
+  float* os = P.out_score ? P.out_score + int64_t(b) * P.k : nullptr;
+  for (int j = tid; j < P.k; j += kSelThreads) {
+    if (j < m) {
+      oi[j] = static_cast<int32_t>(s_sel[j] >> 32);
+      if (os) os[j] = vals[static_cast<uint32_t>(s_sel[j] & 0xffffffffu)];
+    } else {
+      oi[j] = -1;
+      if (os) os[j] = -INFINITY;
+    }
+  }
+  // leave the workspace zeroed for the next call
+  for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+  if (tid < 4) ctr[tid] = 0;
+}
+
+}  // namespace
+
+int select_slices(int64_t n_values, int B, int num_sms) {
+  int64_t s = (2 * int64_t(num_sms) + B - 1) / B;
+  const int64_t cap = (n_values + 4095) / 4096;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  if (s > 65535) s = 65535;
+  return static_cast<int>(s);
+}
+
+cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
+                               cudaStream_t stream) {
+  if (n_probs < 1 || n_probs > kMaxProblems || B == 0) return cudaSuccess;
+  SelectArgs args{};
+  int gx = 1;
+  for (int i = 0; i < n_probs; ++i) {
+    args.p[i] = probs[i];
+    if (probs[i].slices > gx) gx = probs[i].slices;
+  }
+  dim3 grid(gx, B, n_probs);
+  k_topk_select<<<grid, kSelThreads, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace fp4kv

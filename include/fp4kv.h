@@ -1,0 +1,193 @@
+/*
+ * libfp4kv -- decode-time sparse attention over a global KV cache stored as FP4.
+ *
+ * C ABI of the library. Every call takes plain pointers and sizes; no call allocates device
+ * memory, synchronises, or aborts. Kernels are enqueued on the caller's CUDA stream
+ * (`stream` is a cudaStream_t; NULL means the legacy default stream). All tensor pointers
+ * are DEVICE pointers owned by the caller unless a comment says otherwise; the library keeps
+ * no pointer after a call returns.
+ *
+ * Method sources (web pages about DeepSeek-V4.1-Flash):
+ *  [PyTorchKR]  discuss.pytorch.kr, "DeepSeek-V4.1-Flash, KV 캐시를 토큰당 890바이트로
+ *               줄이고 플래그십 V4-Pro를 대체하는 552B 규모의 MoE 모델"
+ *               - section "890바이트를 만든 나머지 절반, FP4 KV 캐시와 지속 캐시 재설계":
+ *                 main KV stored as E2M1 values with one E4M3 scale per 16 channels (NVFP4
+ *                 without its second-level global scale), largest magnitude 448 x 6 = 2688,
+ *                 used for storage only and dequantized before attention;
+ *               - section "레이어 사이에서 캐시와 인덱스를 돌려 쓰는 CSA2": the Full / Reindex /
+ *                 Reuse mode table (who computes the main KV, the indexer K and the top-K
+ *                 indices), 32 indexer query heads of dimension 128, attention top-K;
+ *               - section "계층적 희소 인덱서로 인덱싱 비용을 컨텍스트 길이에서 분리하기": the
+ *                 first Full decoder layer scores every visible position, gives each block of
+ *                 8 positions its largest score and keeps the best blocks as a candidate
+ *                 pool; later Reindex layers score only inside the pool.
+ *  [ingu627]    ingu627 blog on DeepSeek V4.1-Flash-1017, section "3. KV 캐시 압축: HBM
+ *               890바이트와 SSD 8분의 1 바운디드 리플레이" (FP4 KV quantization,
+ *               index_topk) and section "MoE 라우팅과 하드웨어 병목의 분리 매칭" (64 query
+ *               heads sharing a single KV head).
+ *
+ * Readings where the pages are silent (fixed by this library):
+ *  - scale S = E4M3(amax / 6) with round-to-nearest-even, saturating at 448; codes
+ *    E2M1(|x| / S) round-to-nearest-even, saturating at 6, with the sign bit of x kept
+ *    (a negative value rounding to zero is stored as 0x8); an all-zero group has S = 0;
+ *  - two codes per byte, even channel in the low nibble; one scale byte per 16 channels;
+ *  - indexer score[n] = ks[n] * sum_h w[h] * max(0, q[h] . k[n]) in fp32 (ks = 1 when no
+ *    key scale is given);
+ *  - top-K by (score descending, position ascending); indices are written in ascending
+ *    position order and padded with -1;
+ *  - attention: o[h] = sum_j softmax_j(sm_scale * q[h] . v_j) v_j with v_j the dequantized
+ *    row (one latent row is both key and value); lse[h] = natural log of the softmax
+ *    denominator plus the max logit.
+ *
+ * Cache layout (batch-major, two planes, rows padded to the capacity `cap`):
+ *    packed [B][cap][d/2]   uint8, E2M1 codes
+ *    scales [B][cap][d/16]  uint8, E4M3 codes
+ *    keys   [B][cap][128]   uint8 E4M3 codes, or uint16 bf16 bits
+ * Position n of sequence b is row b*cap + n. Positions n >= seq_lens[b] are not visible.
+ *
+ * Inputs must be finite. NaN or Inf in any input gives undefined (but memory-safe)
+ * results.
+ */
+#ifndef FP4KV_H_
+#define FP4KV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP4KV_OK = 0,
+  FP4KV_ERR_INVALID_ARG = 1,         /* null pointer, negative size, misaligned pointer  */
+  FP4KV_ERR_UNSUPPORTED = 2,         /* a size outside the supported range                */
+  FP4KV_ERR_CUDA = 3,                /* a launch or runtime call failed (see last_error) */
+  FP4KV_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below fp4kv_workspace_bytes(...)         */
+  FP4KV_ERR_DEVICE_FLAG = 5          /* a kernel reported a timed-out wait (status word)  */
+} fp4kv_status;
+
+typedef enum { FP4KV_KEY_BF16 = 0, FP4KV_KEY_E4M3 = 1 } fp4kv_key_dtype;
+
+typedef enum {
+  FP4KV_OP_KV_QUANT = 0,
+  FP4KV_OP_INDEXER_TOPK = 1,     /* flat (pool == NULL) */
+  FP4KV_OP_REINDEX_TOPK = 2,     /* fp4kv_indexer_topk with a pool */
+  FP4KV_OP_HIER_POOL_SELECT = 3,
+  FP4KV_OP_SPARSE_ATTN = 4,
+  FP4KV_OP_INDEXER_SCORES = 5
+} fp4kv_op;
+
+/* Supported ranges (anything else returns FP4KV_ERR_UNSUPPORTED):
+ *   d % 32 == 0 and 32 <= d <= 1024 (attention: d == 512);   indexer key dim == 128;
+ *   1 <= H_I <= 64;   1 <= top_k <= 4096;   1 <= H <= 128;   1 <= block_size, and
+ *   block_size == 8 for the pool;   1 <= n_pool_blocks <= 4096;   1 <= B <= 65535.       */
+
+/* Text of the last error raised on the calling thread ("" after a successful call). */
+const char* fp4kv_last_error(void);
+/* Library version string (static storage). */
+const char* fp4kv_version(void);
+
+/* Bytes of scratch `ws` that an op needs for the given sizes. `heads` is H for
+ * FP4KV_OP_SPARSE_ATTN and H_I for the indexer ops; unused arguments are ignored.
+ * Returns 0 for ops that need no workspace or for unsupported sizes. */
+size_t fp4kv_workspace_bytes(int32_t op, int32_t B, int64_t cap, int32_t heads, int32_t top_k,
+                             int32_t n_pool_blocks);
+
+/* Zero a workspace before its first use (enqueued on `stream`). Kernels leave the
+ * workspace zeroed again when they finish, so it can be reused by later calls on the same
+ * stream and captured in CUDA graphs; calls that share one workspace must not overlap. */
+fp4kv_status fp4kv_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Device status word of a workspace: bit 0 set if a kernel gave up on a bounded wait.
+ * Enqueues an async copy of the word into *host_status (pinned or pageable host memory)
+ * and synchronises `stream`; then clears the word. For tests and diagnostics. */
+fp4kv_status fp4kv_workspace_status(void* ws, uint32_t* host_status, void* stream);
+
+/* kv_quant_fp4 -- quantize-on-write ([PyTorchKR] FP4 KV section).
+ * x        : bf16 rows [n_rows][x_row_stride] (uint16 bits); d channels used per row.
+ *            16-byte aligned, x_row_stride a multiple of 8.
+ * dst_row  : nullable int64 [n_rows]; input row i is written to cache row dst_row[i]
+ *            (e.g. b*cap + position). NULL writes row i to row i. Entries outside
+ *            [0, cap_rows) are skipped.
+ * packed   : [cap_rows][d/2] uint8, 16-byte aligned.   scales : [cap_rows][d/16] uint8.
+ * Per group of 16 channels: S = E4M3_RNE_sat(amax/6); codes = sign | E2M1_RNE_sat(|x|/S). */
+fp4kv_status fp4kv_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int32_t d, int64_t x_row_stride,
+                                const int64_t* dst_row, uint8_t* packed, uint8_t* scales,
+                                int64_t cap_rows, void* stream);
+
+/* indexer_scores -- Full-mode scoring of every visible entry, no selection
+ * ([PyTorchKR] CSA2 section: the indexer scores all causally visible positions).
+ * q         : [B][H_I][128] E4M3 codes (key_dtype E4M3) or bf16 bits (key_dtype BF16).
+ * w         : fp32 [B][H_I] head weights (any query scale folded in).
+ * keys      : [B][cap][128], same dtype as q. 16-byte aligned.
+ * key_scale : nullable fp32 [B][cap] per-entry key scale ks.
+ * seq_lens  : int32 [B] (device); seq_lens[b] <= cap. Entries n >= seq_lens[b] are not
+ *             scored and out_score[b][n] is left unwritten for them.
+ * out_score : fp32 [B][cap].
+ * ws        : at least fp4kv_workspace_bytes(FP4KV_OP_INDEXER_SCORES, ...) (a status word). */
+fp4kv_status fp4kv_indexer_scores(const void* q, const float* w, int32_t H_I, const void* keys,
+                                  int32_t key_dtype, const float* key_scale, int64_t cap,
+                                  const int32_t* seq_lens, int32_t B, float* out_score,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* indexer_topk -- Full mode (pool == NULL): exact top-K over every visible entry.
+ * Reindex mode (pool != NULL): score only the positions of the pool's blocks
+ * (block j covers positions [j*block_size, (j+1)*block_size) clipped to seq_len; ids < 0
+ * are skipped; ids must be distinct) with this layer's own query, then top-K among them
+ * ([PyTorchKR] CSA2 mode table, Reindex row; hierarchical indexer section).
+ * pool      : nullable int32 [B][n_pool_blocks].
+ * out_idx   : int32 [B][top_k], positions in ascending order, padded with -1.
+ * out_score : nullable fp32 [B][top_k], the score of each chosen position (-inf for pads).
+ * ws        : at least fp4kv_workspace_bytes(FP4KV_OP_INDEXER_TOPK or _REINDEX_TOPK, ...),
+ *             zeroed once by fp4kv_workspace_init. */
+fp4kv_status fp4kv_indexer_topk(const void* q, const float* w, int32_t H_I, const void* keys,
+                                int32_t key_dtype, const float* key_scale, int64_t cap,
+                                const int32_t* seq_lens, int32_t B, const int32_t* pool,
+                                int32_t n_pool_blocks, int32_t block_size, int32_t top_k,
+                                int32_t* out_idx, float* out_score, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* hier_pool_select -- the first Full-mode decoder layer of the hierarchical sparse indexer
+ * ([PyTorchKR] hierarchical indexer section): one scan that yields the flat top-K AND the
+ * candidate pool, i.e. the n_pool_blocks blocks of block_size positions with the largest
+ * block max score (ties: lower block id), as block ids in ascending order padded with -1.
+ * out_pool : int32 [B][n_pool_blocks]. Other arguments as fp4kv_indexer_topk. */
+fp4kv_status fp4kv_hier_pool_select(const void* q, const float* w, int32_t H_I, const void* keys,
+                                    int32_t key_dtype, const float* key_scale, int64_t cap,
+                                    const int32_t* seq_lens, int32_t B, int32_t top_k,
+                                    int32_t block_size, int32_t n_pool_blocks, int32_t* out_idx,
+                                    int32_t* out_pool, float* out_score, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* sparse_attn_decode -- gather the selected rows, dequantize them (E2M1 x E4M3, exact) and
+ * run softmax attention for every query head ([PyTorchKR] FP4 KV section: dequantized
+ * before attention; [ingu627]: 64 query heads over one shared KV head).
+ * Reuse mode is this call with the previous layer's idx ([PyTorchKR] CSA2 mode table).
+ * q        : bf16 bits [B][H][d], 16-byte aligned.   d == 512.
+ * packed, scales : the cache planes (see layout above).
+ * idx      : int32 [B][top_k]; entries < 0 or >= seq_lens[b] are skipped; duplicates count.
+ * out      : fp32 [B][H][d].   lse : nullable fp32 [B][H] (-inf when no entry is valid,
+ *            in which case out is 0).
+ * ws       : at least fp4kv_workspace_bytes(FP4KV_OP_SPARSE_ATTN, B, cap, H, top_k, 0),
+ *            zeroed once by fp4kv_workspace_init. */
+fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, int32_t d,
+                                      const uint8_t* packed, const uint8_t* scales, int64_t cap,
+                                      const int32_t* seq_lens, const int32_t* idx, int32_t top_k,
+                                      float sm_scale, float* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* Benchmark support (no counterpart on the pages). While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on the launch stream (do not enable
+ * during CUDA-graph capture). fp4kv_profile_read waits for the recorded events and returns,
+ * per kernel kind [0 kv_quant, 1 indexer scoring, 2 top-K select, 3 sparse attention], the
+ * number of launches and their summed device time in milliseconds (host arrays of 4), then
+ * clears the records. */
+fp4kv_status fp4kv_profile_enable(int32_t on);
+fp4kv_status fp4kv_profile_read(int32_t* launches, float* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4KV_H_ */

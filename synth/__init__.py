@@ -64,16 +64,18 @@ def hash_rows_cols(key: int, rows: torch.Tensor, ncols: int) -> torch.Tensor:
     return _mix32(rk[:, None] ^ ck[None, :])
 
 
-_NORMAL_TABLE_CPU = None
+_NORMAL_TABLES = {}
 
 
 def normal_table(device) -> torch.Tensor:
     """65,536 bf16 N(0,1) quantiles: ndtri((i + 0.5) / 65536), fp64 then bf16."""
-    global _NORMAL_TABLE_CPU
-    if _NORMAL_TABLE_CPU is None:
-        p = (torch.arange(65536, dtype=torch.float64) + 0.5) / 65536.0
-        _NORMAL_TABLE_CPU = torch.special.ndtri(p).to(torch.bfloat16)
-    return _NORMAL_TABLE_CPU.to(device)
+    key = str(torch.device(device))
+    if key not in _NORMAL_TABLES:
+        if "cpu" not in _NORMAL_TABLES:
+            p = (torch.arange(65536, dtype=torch.float64) + 0.5) / 65536.0
+            _NORMAL_TABLES["cpu"] = torch.special.ndtri(p).to(torch.bfloat16)
+        _NORMAL_TABLES[key] = _NORMAL_TABLES["cpu"].to(device)
+    return _NORMAL_TABLES[key]
 
 
 def normal_bf16(h: torch.Tensor) -> torch.Tensor:
@@ -117,11 +119,12 @@ def kv_rows(seed: int, layer: int, seq: int, rows: torch.Tensor, d: int,
 
 
 def attn_query(seed: int, layer: int, B: int, H: int, d: int, device="cpu") -> torch.Tensor:
-    """bf16 [B, H, d] attention queries, N(0,1) / sqrt(d)."""
-    rows = torch.arange(B * H, dtype=torch.int64, device=device)
+    """bf16 [B, H, d] attention queries, N(0,1) / sqrt(d). Drawn on the host (small) and
+    copied, so every device gets the same bits."""
+    rows = torch.arange(B * H, dtype=torch.int64)
     h = hash_rows_cols(_key(seed, S_Q, layer), rows, d)
     x = normal_bf16(h).to(torch.float32) * (1.0 / math.sqrt(d))
-    return x.to(torch.bfloat16).reshape(B, H, d)
+    return x.to(torch.bfloat16).reshape(B, H, d).to(device)
 
 
 def indexer_keys(seed: int, seq: int, rows: torch.Tensor, dk: int = 128,
@@ -141,16 +144,16 @@ def indexer_query(seed: int, layer: int, B: int, H_I: int, dk: int = 128, fp8: b
 
     Returns (q [B, H_I, dk] as uint8 E4M3 codes when fp8 else bf16, w [B, H_I] fp32).
     With fp8 the query is quantized per (b, h) with scale amax / 448 and the scale is
-    multiplied into w (exact: a positive scale commutes with max(0, .))."""
-    rows = torch.arange(B * H_I, dtype=torch.int64, device=device)
+    multiplied into w (exact: a positive scale commutes with max(0, .)). Drawn on the host
+    (small) and copied, so every device gets the same bits."""
+    rows = torch.arange(B * H_I, dtype=torch.int64)
     h = hash_rows_cols(_key(seed, S_QI, layer), rows, dk)
     q = (normal_bf16(h).to(torch.float32) * (1.0 / math.sqrt(dk))).reshape(B, H_I, dk)
-    hw = hash_rows_cols(_key(seed, S_W, layer), torch.arange(B, dtype=torch.int64,
-                                                             device=device), H_I)
+    hw = hash_rows_cols(_key(seed, S_W, layer), torch.arange(B, dtype=torch.int64), H_I)
     w = ((0.5 + uniform01(hw)) / H_I).to(torch.float32)
     if not fp8:
-        return q.to(torch.bfloat16), w
+        return q.to(torch.bfloat16).to(device), w.to(device)
     amax = q.abs().amax(dim=2).clamp_min(1e-30)
     scale = amax / 448.0
     q8 = (q / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
-    return q8, (w * scale).to(torch.float32)
+    return q8.to(device), (w * scale).to(torch.float32).to(device)

@@ -1,0 +1,325 @@
+"""GPU parity: every call of the C ABI against the CPU oracle on the same seeded inputs.
+
+Sizes span several tiles with ragged tails; the full-size configurations have their own
+file. All calls go through the C ABI (``fp4_sparse_attention_kv_b200.binding``).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import fp4kv_oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def fk(cuda_lib):
+    import fp4_sparse_attention_kv_b200 as fk
+    return fk
+
+
+def _bf16_from_f64(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------------------
+# kv_quant_fp4
+# ----------------------------------------------------------------------------------------
+
+def _quant_gpu(fk, x_bf16: torch.Tensor):
+    n, d = x_bf16.shape
+    xd = x_bf16.to(DEV)
+    packed = torch.empty((n, d // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((n, d // 16), dtype=torch.uint8, device=DEV)
+    fk.kv_quant_fp4(xd, packed, scales)
+    return packed.cpu().numpy(), scales.cpu().numpy()
+
+
+def _exhaustive_groups():
+    """Groups [A, x1..x15]: for every E4M3 scale code s, A is the largest bf16 value whose
+    scale is s, and x runs over every finite bf16 value (both signs) with |x| <= A; plus one
+    group per non-negative finite bf16 amax."""
+    bits = np.arange(0, 0x7F80, dtype=np.uint16)
+    v = O.bf16_bits_to_f64(bits)
+    s_of = O.e4m3_round_sat(v / 6.0)
+    groups = []
+    for s in range(0, 127):
+        cand = v[s_of == s]
+        if cand.size == 0:
+            continue
+        A = cand.max()
+        xs = v[v <= A]
+        xs = np.concatenate([xs, -xs])
+        pad = (-xs.size) % 15
+        xs = np.concatenate([xs, np.zeros(pad)]).reshape(-1, 15)
+        groups.append(np.concatenate([np.full((xs.shape[0], 1), A), xs], axis=1))
+    # every amax value once (scale coverage), sign of the max alternating
+    am = np.zeros((v.size, 16))
+    am[:, 0] = np.where(np.arange(v.size) % 2 == 0, v, -v)
+    am[:, 5] = v / 3.0  # arbitrary second element below the max (bf16-rounded below)
+    groups.append(am)
+    g = np.concatenate(groups, axis=0)
+    pad = (-g.shape[0]) % 32
+    g = np.concatenate([g, np.zeros((pad, 16))], axis=0)
+    return g.reshape(-1, 512)
+
+
+def test_quant_exhaustive_bf16_values_by_scale(fk):
+    x = _exhaustive_groups()
+    xb = _bf16_from_f64(x)
+    xv = P.to_f64(xb)  # exact bf16 values given to both sides
+    gp, gs = _quant_gpu(fk, xb)
+    op, os_ = O.kv_quant_fp4(xv)
+    assert np.array_equal(gs, os_), f"scale bytes differ in {np.sum(gs != os_)} groups"
+    assert np.array_equal(gp, op), f"packed bytes differ in {np.sum(gp != op)} places"
+
+
+def test_quant_golden_example(fk):
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "quant_example.json")))
+    x = np.array(g["rows"], dtype=np.float64)
+    x[0, 7] = -0.0
+    x[1, 3] = -0.0
+    x = np.concatenate([x, np.zeros((2, 32))], axis=1)  # d = 64 (library needs d % 32 == 0)
+    gp, gs = _quant_gpu(fk, _bf16_from_f64(x))
+    assert [bytes(r[:16]).hex().upper() for r in gp] == g["packed_hex"]
+    assert gs[:, :2].tolist() == g["scales"]
+
+
+@pytest.mark.parametrize("d", [512, 64, 1024])
+def test_quant_synthetic_rows_with_saturation(fk, d):
+    rows = torch.arange(3000, dtype=torch.int64)
+    xb = synth.kv_rows(1, 3, 0, rows, d, heavy_frac=0.01)
+    gp, gs = _quant_gpu(fk, xb)
+    op, os_ = O.kv_quant_fp4(P.to_f64(xb))
+    assert np.array_equal(gs, os_) and np.array_equal(gp, op)
+    assert (gs == 0x7E).any()  # some rows saturate the scale at 448
+
+
+def test_quant_scatter_rows_and_stride(fk):
+    d = 512
+    src = synth.kv_rows(2, 0, 0, torch.arange(64), 1024)[:, :d]  # row stride 1024 > d
+    xd = synth.kv_rows(2, 0, 0, torch.arange(64), 1024).to(DEV)[:, :d]
+    cap = 200
+    packed = torch.full((cap, d // 2), 0xAB, dtype=torch.uint8, device=DEV)
+    scales = torch.full((cap, d // 16), 0xCD, dtype=torch.uint8, device=DEV)
+    dst = torch.tensor([3 * i + 1 for i in range(60)] + [-1, cap, 10 ** 9, 0], dtype=torch.int64)
+    fk.kv_quant_fp4(xd, packed, scales, dst_row=dst.to(DEV))
+    op, os_ = O.kv_quant_fp4(P.to_f64(src))
+    pk, sc = packed.cpu().numpy(), scales.cpu().numpy()
+    for i, r in enumerate(dst.tolist()):
+        if 0 <= r < cap:
+            assert np.array_equal(pk[r], op[i]) and np.array_equal(sc[r], os_[i])
+    untouched = sorted(set(range(cap)) - {r for r in dst.tolist() if 0 <= r < cap})
+    assert np.all(pk[untouched] == 0xAB) and np.all(sc[untouched] == 0xCD)
+
+
+# ----------------------------------------------------------------------------------------
+# indexer scores / top-K / pool / reindex
+# ----------------------------------------------------------------------------------------
+
+def _indexer_inputs(seed, B, cap, H_I, fp8):
+    q, w = synth.indexer_query(seed, 0, B, H_I, fp8=fp8, device=DEV)
+    keys = P.keys_dev(seed, B, cap, fp8, DEV)
+    return q, w, keys
+
+
+def test_generator_is_identical_on_host_and_device():
+    rows = torch.arange(0, 5000, 7, dtype=torch.int64)
+    for fp8 in (True, False):
+        a = synth.indexer_keys(3, 1, rows, 128, fp8)
+        b = synth.indexer_keys(3, 1, rows.to(DEV), 128, fp8).cpu()
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    a = synth.kv_rows(4, 2, 1, rows, 512, heavy_frac=0.01)
+    b = synth.kv_rows(4, 2, 1, rows.to(DEV), 512, heavy_frac=0.01).cpu()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    qa, wa = synth.indexer_query(5, 1, 3, 32)
+    qb, wb = synth.indexer_query(5, 1, 3, 32, device=DEV)
+    assert torch.equal(qa, qb.cpu()) and torch.equal(wa, wb.cpu())
+    assert torch.equal(synth.attn_query(6, 0, 2, 16, 512).view(torch.int16),
+                       synth.attn_query(6, 0, 2, 16, 512, device=DEV).cpu().view(torch.int16))
+
+
+@pytest.mark.parametrize("fp8,H_I", [(True, 32), (False, 32), (True, 1), (True, 20), (True, 64)])
+def test_indexer_scores_match_oracle(fk, fp8, H_I):
+    B, cap = 2, 1000
+    q, w, keys = _indexer_inputs(7, B, cap, H_I, fp8)
+    lens = torch.tensor([1000, 613], dtype=torch.int32, device=DEV)
+    ks = torch.rand((B, cap), generator=torch.Generator().manual_seed(1)).to(DEV) + 0.5
+    for key_scale in (None, ks):
+        got = fk.indexer_scores(q, w, keys, lens, key_scale=key_scale).cpu().numpy()
+        for b in range(B):
+            L = int(lens[b])
+            ref = P.oracle_scores_seq(q[b], w[b], keys[b], L, None if key_scale is None else ks[b])
+            err = np.abs(got[b, :L].astype(np.float64) - ref) / np.maximum(np.abs(ref), 1e-3)
+            assert err.max() <= 2e-6, err.max()
+            assert np.all(np.isneginf(got[b, L:]))
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=0, B=1, cap=4096, lens=[4096], H_I=32, fp8=False, k=256),     # the tiny config
+    dict(seed=1, B=3, cap=5000, lens=[5000, 4093, 77], H_I=32, fp8=True, k=300),
+    dict(seed=2, B=2, cap=70000, lens=[70000, 65536], H_I=32, fp8=True, k=2048),
+    dict(seed=3, B=2, cap=3000, lens=[3000, 2999], H_I=8, fp8=True, k=1),
+    dict(seed=4, B=1, cap=9000, lens=[9000], H_I=64, fp8=True, k=4096),
+])
+def test_indexer_topk_matches_oracle(fk, case):
+    q, w, keys = _indexer_inputs(case["seed"], case["B"], case["cap"], case["H_I"], case["fp8"])
+    lens = torch.tensor(case["lens"], dtype=torch.int32, device=DEV)
+    k = case["k"]
+    score = torch.empty((case["B"], k), dtype=torch.float32, device=DEV)
+    idx = fk.indexer_topk(q, w, keys, lens, k, out_score=score).cpu().numpy()
+    score = score.cpu().numpy()
+    for b in range(case["B"]):
+        L = case["lens"][b]
+        ref = P.oracle_scores_seq(q[b], w[b], keys[b], L)
+        P.check_topk(idx[b], ref, np.arange(L), k, f"b={b}")
+        m = min(k, L)
+        assert np.all(np.isneginf(score[b, m:]))
+        err = np.abs(score[b, :m].astype(np.float64) - ref[idx[b, :m]]) / np.maximum(ref[idx[b, :m]], 1e-3)
+        assert err.max() <= 2e-6
+
+
+def test_indexer_topk_ties_go_to_the_lowest_positions(fk):
+    B, cap, k = 2, 3000, 100
+    q, w, _ = _indexer_inputs(9, B, cap, 32, True)
+    row = synth.indexer_keys(9, 0, torch.arange(1, dtype=torch.int64), 128, True)
+    keys = row.repeat(cap, 1).reshape(1, cap, 128).repeat(B, 1, 1).to(DEV).contiguous()
+    keys[1, 2000:2050] = 0  # lower scores in the middle of sequence 1
+    lens = torch.tensor([3000, 2500], dtype=torch.int32, device=DEV)
+    idx = fk.indexer_topk(q, w, keys, lens, k).cpu().numpy()
+    assert idx[0].tolist() == list(range(k))
+    assert idx[1].tolist() == list(range(k))
+    # all scores equal -> every position is a candidate; K larger than one radix bucket
+    idx2 = fk.indexer_topk(q, w, keys, lens, 4096).cpu().numpy()
+    assert idx2[0].tolist() == list(range(3000)) + [-1] * 1096
+
+
+def test_hier_pool_select_matches_oracle(fk):
+    B, cap, k, npb = 2, 20000, 256, 64
+    q, w, keys = _indexer_inputs(11, B, cap, 32, True)
+    lens = torch.tensor([20000, 12345], dtype=torch.int32, device=DEV)
+    idx, pool = fk.hier_pool_select(q, w, keys, lens, k, npb)
+    idx, pool = idx.cpu().numpy(), pool.cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        ref = P.oracle_scores_seq(q[b], w[b], keys[b], L)
+        P.check_topk(idx[b], ref, np.arange(L), k, f"idx b={b}")
+        bm = O.block_max(ref, L, 8)
+        P.check_topk(pool[b], bm, np.arange(bm.size), npb, f"pool b={b}")
+
+
+def test_reindex_matches_oracle_and_full_pool_is_flat(fk):
+    B, cap, k, npb = 2, 20000, 256, 64
+    q, w, keys = _indexer_inputs(12, B, cap, 32, True)
+    q2, w2 = synth.indexer_query(12, 1, B, 32, device=DEV)  # this layer's own query
+    lens = torch.tensor([20000, 9999], dtype=torch.int32, device=DEV)
+    pools = []
+    for b in range(B):
+        L = int(lens[b])
+        ref = P.oracle_scores_seq(q[b], w[b], keys[b], L)
+        pl = O.pool_select(ref, L, 8, npb)
+        pl[5] = -1  # a hole in the pool
+        pools.append(pl)
+    pool = torch.tensor(np.stack(pools), dtype=torch.int32, device=DEV)
+    idx = fk.indexer_topk(q2, w2, keys, lens, k, pool=pool).cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        pos = O.pool_positions(pools[b], L, 8)
+        ref = P.oracle_scores_seq(q2[b], w2[b], keys[b], L)[pos] if pos.size else np.zeros(0)
+        P.check_topk(idx[b], ref, pos, k, f"reindex b={b}")
+    # pool = every block of a short sequence: Reindex equals the flat top-K
+    L = 1000
+    lens_s = torch.tensor([L, L], dtype=torch.int32, device=DEV)
+    allb = torch.arange(125, dtype=torch.int32, device=DEV).repeat(B, 1).contiguous()
+    re = fk.indexer_topk(q2, w2, keys, lens_s, 200, pool=allb).cpu().numpy()
+    fl = fk.indexer_topk(q2, w2, keys, lens_s, 200).cpu().numpy()
+    assert np.array_equal(re, fl)
+
+
+# ----------------------------------------------------------------------------------------
+# sparse attention
+# ----------------------------------------------------------------------------------------
+
+def _attn_case(fk, seed, B, cap, H, lens, idx_np, layer=0, sm_scale=1.0):
+    d = 512
+    x = P.kv_rows_dev(seed, layer, B, cap, d, DEV)
+    packed = torch.empty((B, cap, d // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((B, cap, d // 16), dtype=torch.uint8, device=DEV)
+    fk.kv_quant_fp4(x.view(B * cap, d), packed.view(B * cap, d // 2), scales.view(B * cap, d // 16))
+    del x
+    q = synth.attn_query(seed, layer, B, H, d, device=DEV)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    idx = torch.tensor(idx_np, dtype=torch.int32, device=DEV)
+    out, lse = fk.sparse_attn_decode(q, packed, scales, lens_t, idx, sm_scale)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    qh = P.to_f64(q.cpu())
+    for b in range(B):
+        sel = np.asarray(idx_np[b])
+        valid = sel[(sel >= 0) & (sel < lens[b])]
+        if valid.size:
+            rows = P.kv_rows_host(seed, layer, b, valid, d)
+            pk, sc = O.kv_quant_fp4(rows)  # the oracle's own quantization
+            ro, rl = O.sparse_attn_decode_rows(qh[b], O.kv_dequant_fp4(pk, sc), sm_scale)
+        else:
+            ro, rl = np.zeros((H, d)), np.full(H, -np.inf)
+        P.check_attn(out[b], lse[b], ro, rl, f"b={b}")
+    return out, lse
+
+
+def test_attention_tiny_config_end_to_end(fk):
+    # quantize -> oracle top-K of the bf16 indexer -> attention, 16 heads, K = 256
+    cap, k = 4096, 256
+    q8, w = synth.indexer_query(0, 0, 1, 32, fp8=False)
+    keys = synth.indexer_keys(0, 0, torch.arange(cap), 128, fp8=False)
+    ref = O.indexer_scores(P.to_f64(q8[0]), w[0].double().numpy(), P.to_f64(keys))
+    idx = O.topk_positions(ref, np.arange(cap), k)[None, :]
+    _attn_case(fk, 0, 1, cap, 16, [cap], idx)
+
+
+@pytest.mark.parametrize("H", [64, 16, 20, 128])
+def test_attention_decode_shapes(fk, H):
+    B, cap, k = 3, 8192, 2048
+    rng = np.random.default_rng(H)
+    idx = np.stack([np.sort(rng.choice(cap, k, replace=False)) for _ in range(B)])
+    _attn_case(fk, 21, B, cap, H, [cap] * B, idx, sm_scale=1.0)
+
+
+def test_attention_edge_cases(fk):
+    B, cap, k = 5, 600, 300
+    rng = np.random.default_rng(5)
+    idx = np.stack([rng.choice(cap, k, replace=False) for _ in range(B)]).astype(np.int64)
+    idx[0, :50] = -1                   # holes
+    idx[1, :20] = idx[1, 20]           # duplicates count
+    idx[2, :] = -1                     # nothing valid: out = 0, lse = -inf
+    idx[3, 10:] = 10 ** 6              # beyond the cache
+    lens = [600, 600, 600, 600, 250]   # sequence 4: entries >= 250 invisible
+    out, lse = _attn_case(fk, 31, B, cap, 64, lens, idx, sm_scale=0.75)
+    assert np.all(out[2] == 0) and np.all(np.isneginf(lse[2]))
+
+
+def test_attention_single_entry_returns_the_row(fk):
+    B, cap, k = 2, 100, 1
+    idx = np.array([[7], [99]])
+    out, _ = _attn_case(fk, 41, B, cap, 16, [100, 100], idx)
+    rows = P.kv_rows_host(41, 0, 0, [7], 512)
+    pk, sc = O.kv_quant_fp4(rows)
+    vh = O.kv_dequant_fp4(pk, sc)[0]
+    assert np.allclose(out[0], np.broadcast_to(vh, out[0].shape), rtol=1e-6, atol=1e-6)
+
+
+def test_workspace_is_left_clean_and_status_zero(fk):
+    B, cap, k = 2, 5000, 128
+    q, w, keys = _indexer_inputs(13, B, cap, 32, True)
+    lens = torch.tensor([5000, 4000], dtype=torch.int32, device=DEV)
+    ws = fk.alloc_workspace(fk.workspace_bytes(fk.OP_INDEXER_TOPK, B, cap, 32, k), DEV)
+    a = fk.indexer_topk(q, w, keys, lens, k, ws=ws).clone()
+    b = fk.indexer_topk(q, w, keys, lens, k, ws=ws)
+    assert torch.equal(a, b)
+    assert fk.workspace_status(ws) == 0

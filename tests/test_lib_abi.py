@@ -1,0 +1,95 @@
+"""CPU-only checks of the C-ABI boundary: the shared library builds and loads, exports every
+symbol ``include/fp4kv.h`` declares, and rejects bad arguments on the host before any
+kernel is launched (no GPU needed: validation happens before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_sparse_attention_kv_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "fp4kv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4kv_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary_calls():
+    syms = _declared_symbols()
+    for name in ("fp4kv_kv_quant_fp4", "fp4kv_indexer_topk", "fp4kv_hier_pool_select",
+                 "fp4kv_sparse_attn_decode", "fp4kv_workspace_bytes", "fp4kv_last_error"):
+        assert name in syms
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = binding.lib()
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+    assert set(n for n, _, _ in binding.SIGNATURES) == set(_declared_symbols())
+    assert "sm_100a" in binding.version()
+
+
+def _call(name, *args):
+    L = binding.lib()
+    st = getattr(L, name)(*args)
+    return st, L.fp4kv_last_error().decode()
+
+
+def test_host_validation_rejects_bad_arguments_without_a_gpu():
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: validation fails first
+    # null pointers
+    st, msg = _call("fp4kv_kv_quant_fp4", None, 4, 512, 512, None, None, None, 4, None)
+    assert st == 1 and "null" in msg
+    # unsupported d
+    st, msg = _call("fp4kv_kv_quant_fp4", fake, 4, 48, 48, None, fake, fake, 4, None)
+    assert st == 2 and "d=48" in msg
+    # zero rows is a no-op success
+    st, msg = _call("fp4kv_kv_quant_fp4", None, 0, 512, 512, None, None, None, 0, None)
+    assert st == 0 and msg == ""
+    # indexer: H_I out of range, top_k out of range, misaligned keys, bad block size
+    st, msg = _call("fp4kv_indexer_topk", fake, fake, 65, fake, 1, None, 100, fake, 1, None, 0,
+                    8, 16, fake, None, fake, 1 << 20, None)
+    assert st == 2 and "H_I" in msg
+    st, msg = _call("fp4kv_indexer_topk", fake, fake, 32, fake, 1, None, 100, fake, 1, None, 0,
+                    8, 5000, fake, None, fake, 1 << 20, None)
+    assert st == 2 and "top_k" in msg
+    st, msg = _call("fp4kv_indexer_topk", fake, fake, 32, P(0x10001), 1, None, 100, fake, 1,
+                    None, 0, 8, 16, fake, None, fake, 1 << 20, None)
+    assert st == 1 and "aligned" in msg
+    st, msg = _call("fp4kv_hier_pool_select", fake, fake, 32, fake, 1, None, 100, fake, 1, 16, 4,
+                    8, fake, fake, None, fake, 1 << 20, None)
+    assert st == 2 and "block_size" in msg
+    # workspace too small
+    need = binding.workspace_bytes(binding.OP_INDEXER_TOPK, 1, 100, 32, 16)
+    st, msg = _call("fp4kv_indexer_topk", fake, fake, 32, fake, 1, None, 100, fake, 1, None, 0,
+                    8, 16, fake, None, fake, need - 1, None)
+    assert st == 4 and "ws_bytes" in msg
+    # attention: d must be 512, H <= 128
+    st, msg = _call("fp4kv_sparse_attn_decode", fake, 1, 16, 256, fake, fake, 10, fake, fake, 4,
+                    ctypes.c_float(1.0), fake, None, fake, 1 << 20, None)
+    assert st == 2 and "d=256" in msg
+    st, msg = _call("fp4kv_sparse_attn_decode", fake, 1, 129, 512, fake, fake, 10, fake, fake, 4,
+                    ctypes.c_float(1.0), fake, None, fake, 1 << 20, None)
+    assert st == 2 and "H=129" in msg
+
+
+def test_workspace_sizes_cover_the_configurations():
+    wb = binding.workspace_bytes
+    # scores + candidate list dominate: at least 8 bytes per scored entry
+    assert wb(binding.OP_INDEXER_TOPK, 4, 1 << 20, 32, 2048) >= 4 * (1 << 20) * 8
+    assert wb(binding.OP_HIER_POOL_SELECT, 8, 1 << 20, 32, 2048, 1024) > wb(
+        binding.OP_INDEXER_TOPK, 8, 1 << 20, 32, 2048)
+    assert wb(binding.OP_REINDEX_TOPK, 8, 1 << 20, 32, 2048, 1024) < (1 << 20)
+    assert wb(binding.OP_SPARSE_ATTN, 32, 65536, 64, 2048) > 0
+    assert wb(binding.OP_KV_QUANT, 1, 1) == 0
+
+
+def test_binding_raises_typed_errors():
+    with pytest.raises(binding.Fp4kvError) as ei:
+        binding._check(2)
+    assert ei.value.status == 2
