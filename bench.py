@@ -16,6 +16,7 @@ step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import hashlib
 import json
 import math
@@ -120,12 +121,14 @@ class ClockSampler:
             nv.nvmlInit()
             self._nv = nv
             bus = None
-            try:
-                bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            try:  # torch reports the PCI location as integers
+                pr = torch.cuda.get_device_properties(device_index)
+                dom, b, dv = int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id)
+                bus = f"{dom:08X}:{b:02X}:{dv:02X}.0".encode()
             except Exception:
                 bus = None
-            if bus:
-                self._h = nv.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+            if isinstance(bus, bytes):
+                self._h = nv.nvmlDeviceGetHandleByPciBusId(bus)
             else:
                 vis = os.environ.get("CUDA_VISIBLE_DEVICES")
                 idx = int(vis.split(",")[device_index]) if vis and vis.split(",")[0].isdigit() else device_index
@@ -505,7 +508,12 @@ def run_reference(args, cfg_name, cfg):
     return 0
 
 
+def phase(msg):
+    print(f"[bench] {time.strftime('%H:%M:%S')} {msg}", file=sys.stderr, flush=True)
+
+
 def main(argv=None):
+    faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -531,6 +539,7 @@ def main(argv=None):
 
     import fp4_sparse_attention_kv_b200 as fk
     fk.lib()
+    phase(f"building workload {cfg_name}")
     if cfg_name == "quant":
         wl = QuantWorkload(cfg, fk, device, rank)
     elif cfg_name == "hier":
@@ -540,11 +549,14 @@ def main(argv=None):
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
 
+    phase("clock sampler")
     sampler = ClockSampler(local)
     barrier(world, device)
+    phase("timed steps")
     total_ms, prof = timed_steps(wl, args.steps, args.warmup, flush, sampler, fk)
     barrier(world, device)
     step_ms = max_over_ranks(total_ms / args.steps, world, device)
+    phase("end-to-end steps")
     e2e_ms, h2d, d2h = e2e_steps(wl, args.steps, args.warmup)
     e2e_step_ms = max_over_ranks(e2e_ms / args.steps, world, device)
 
@@ -599,6 +611,7 @@ def main(argv=None):
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
+            phase("cpu baseline (oracle)")
             result["cpu_baseline"] = cpu_baseline(cfg_name, cfg)
         print(json.dumps(result), flush=True)
     return 0

@@ -139,13 +139,13 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
   L.sure = off;
   for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(int32_t) * B * L.k[i]);
   L.cand = off;
-  for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(int32_t) * B * L.vstride[i]);
+  for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(uint64_t) * B * L.vstride[i]);
   L.total = off;
   return L;
 }
 
 struct AttnLayout {
-  size_t tickets = 0, part_ml = 0, part_o = 0, total = 0;
+  size_t part_ml = 0, part_o = 0, total = 0;
   int n_chunks = 1, n_hg = 1;
 };
 
@@ -154,8 +154,6 @@ AttnLayout attn_layout(int64_t B, int64_t H, int64_t top_k, int sms) {
   L.n_hg = static_cast<int>((H + 63) / 64);
   L.n_chunks = fp4kv::attn_chunks(static_cast<int>(B), static_cast<int>(H), static_cast<int>(top_k), sms);
   size_t off = kAlign;
-  L.tickets = off;
-  off += up(sizeof(uint32_t) * B * L.n_hg);
   if (L.n_chunks > 1) {
     L.part_ml = off;
     off += up(sizeof(float) * B * L.n_hg * L.n_chunks * 64 * 2);
@@ -177,6 +175,8 @@ fp4kv_status check_indexer_args(const void* q, const float* w, int32_t H_I, cons
   if (H_I < 1 || H_I > 64) return fail(FP4KV_ERR_UNSUPPORTED, "H_I=%d outside [1, 64]", H_I);
   if (cap < 1 || cap > (int64_t(1) << 31) - 8)
     return fail(FP4KV_ERR_UNSUPPORTED, "cap=%lld outside [1, 2^31 - 8]", (long long)cap);
+  if (int64_t(B) * cap > (int64_t(1) << 31) - 256)
+    return fail(FP4KV_ERR_UNSUPPORTED, "B*cap=%lld must stay below 2^31 rows", (long long)(int64_t(B) * cap));
   if (key_dtype != FP4KV_KEY_BF16 && key_dtype != FP4KV_KEY_E4M3)
     return fail(FP4KV_ERR_UNSUPPORTED, "key_dtype=%d", key_dtype);
   if (!aligned(q, 16) || !aligned(keys, 16) || !aligned(w, 4))
@@ -344,7 +344,7 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
     P.sure = reinterpret_cast<int32_t*>(base + sure_off);
     P.cand = reinterpret_cast<int32_t*>(base + cand_off);
     sure_off += up(sizeof(int32_t) * B * L.k[i]);
-    cand_off += up(sizeof(int32_t) * B * L.vstride[i]);
+    cand_off += up(sizeof(uint64_t) * B * L.vstride[i]);
     P.out_idx = (i == 0) ? out_idx : out_pool;
     P.out_score = (i == 0) ? out_score : nullptr;
     const int64_t nvals = (kind == 1) ? int64_t(n_pool_blocks) * 8 : (i == 0 ? cap : (cap + 7) / 8);
@@ -431,7 +431,6 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
   p.out = out;
   p.lse = lse;
   p.n_chunks = L.n_chunks;
-  p.tickets = reinterpret_cast<uint32_t*>(base + L.tickets);
   p.part_ml = L.n_chunks > 1 ? reinterpret_cast<float*>(base + L.part_ml) : nullptr;
   p.part_o = L.n_chunks > 1 ? reinterpret_cast<float*>(base + L.part_o) : nullptr;
   p.status = reinterpret_cast<uint32_t*>(base);

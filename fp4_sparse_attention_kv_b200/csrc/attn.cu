@@ -21,8 +21,8 @@
 // Per sub-tile of 64 entries: the warps gather packed rows + scales with coalesced 16-byte
 // loads and write fp16 rows into an XOR-swizzled shared buffer (conflict-free for stores and
 // for ldmatrix); S = Q V^T (m16n8k16 MMAs), per-head running max / sum, P to shared memory,
-// O += P V. Each chunk writes its unnormalised O with (max, sum); the last CTA of a
-// (sequence, head group) merges the chunks. No CTA waits on another.
+// O += P V. Each chunk writes its unnormalised O with (max, sum); a small second kernel
+// (k_attn_combine, one warp per head) merges the chunks. No CTA waits on another.
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
 
@@ -62,7 +62,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(const AttnParam
   float* sC = reinterpret_cast<float*>(sPl + kSmemP);  // [64] log2-domain logit scale
   float* sRed = sC + 64;                                // [8 warps][16 rows]
   int32_t* sIdx = reinterpret_cast<int32_t*>(sRed + 128);  // [64] position or -1
-  __shared__ bool s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -333,7 +332,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(const AttnParam
     return;
   }
 
-  // ---- split: write this chunk's partial, the last CTA of (b, hg) merges ----
+  // ---- split: write this chunk's unnormalised partial; k_attn_combine merges them ----
   const int64_t part = (int64_t(b) * n_hg + hg) * n_chunks + chunk;
   float* po = p.part_o + part * kHeadsPerCta * kD;
   float* pml = p.part_ml + part * kHeadsPerCta * 2;
@@ -349,56 +348,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(const AttnParam
     pml[2 * h8] = m_g8;
     pml[2 * h8 + 1] = L8;
   }
-  __syncthreads();
-  uint32_t* ticket = p.tickets + int64_t(b) * n_hg + hg;
-  if (tid == 0) {
-    __threadfence();
-    s_last = atomicAdd(ticket, 1u) == uint32_t(n_chunks - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+}
 
-  const float* po0 = p.part_o + (int64_t(b) * n_hg + hg) * n_chunks * kHeadsPerCta * kD;
+// Merge of the chunk partials (log-sum-exp combine): grid (8 head blocks, head groups, B),
+// one warp per head, each lane 16 of the 512 dims.
+__global__ void __launch_bounds__(256) k_attn_combine(const AttnParams p, int n_hg) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hg = blockIdx.y, b = blockIdx.z;
+  const int hh = blockIdx.x * 8 + warp;
+  const int nh = min(kHeadsPerCta, p.H - hg * kHeadsPerCta);
+  if (hh >= nh) return;
+  const int n_chunks = p.n_chunks;
   const float* pml0 = p.part_ml + (int64_t(b) * n_hg + hg) * n_chunks * kHeadsPerCta * 2;
-  // thread -> (head, quarter of the dims)
-  const int hh = tid >> 2, q4 = tid & 3;
-  if (hh < nh) {
-    float M = -INFINITY;
-    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, __ldcg(pml0 + (int64_t(c) * kHeadsPerCta + hh) * 2));
-    float Lt = 0.0f;
-    for (int c = 0; c < n_chunks; ++c) {
-      const float mc = __ldcg(pml0 + (int64_t(c) * kHeadsPerCta + hh) * 2);
-      const float lc = __ldcg(pml0 + (int64_t(c) * kHeadsPerCta + hh) * 2 + 1);
-      if (lc > 0.0f) Lt += lc * exp2f(mc - M);
+  const float* po0 = p.part_o + (int64_t(b) * n_hg + hg) * n_chunks * kHeadsPerCta * kD;
+  float M = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pml0[(int64_t(c) * kHeadsPerCta + hh) * 2]);
+  float Lt = 0.0f;
+  float4 acc[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < n_chunks; ++c) {
+    const float mc = pml0[(int64_t(c) * kHeadsPerCta + hh) * 2];
+    const float lc = pml0[(int64_t(c) * kHeadsPerCta + hh) * 2 + 1];
+    if (!(lc > 0.0f)) continue;
+    const float wgt = exp2f(mc - M);
+    Lt += lc * wgt;
+    const float4* src = reinterpret_cast<const float4*>(po0 + (int64_t(c) * kHeadsPerCta + hh) * kD) + 4 * lane;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 v = src[u];
+      acc[u].x += wgt * v.x; acc[u].y += wgt * v.y; acc[u].z += wgt * v.z; acc[u].w += wgt * v.w;
     }
-    const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
-    float* orow = p.out + (int64_t(b) * p.H + hbase + hh) * kD;
-    for (int d0 = q4 * 4; d0 < kD; d0 += 64) {
-      float4 acc4[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c = 0; c < n_chunks; ++c) {
-        const float mc = __ldcg(pml0 + (int64_t(c) * kHeadsPerCta + hh) * 2);
-        const float lc = __ldcg(pml0 + (int64_t(c) * kHeadsPerCta + hh) * 2 + 1);
-        if (!(lc > 0.0f)) continue;
-        const float wgt = exp2f(mc - M);
-        const float* src = po0 + (int64_t(c) * kHeadsPerCta + hh) * kD + d0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + 16 * u));
-          acc4[u].x += wgt * v.x; acc4[u].y += wgt * v.y; acc4[u].z += wgt * v.z; acc4[u].w += wgt * v.w;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        *reinterpret_cast<float4*>(orow + d0 + 16 * u) =
-            make_float4(acc4[u].x * inv, acc4[u].y * inv, acc4[u].z * inv, acc4[u].w * inv);
-    }
-    if (p.lse != nullptr && q4 == 0)
-      p.lse[int64_t(b) * p.H + hbase + hh] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
   }
-  if (tid == 0) *ticket = 0u;  // leave the workspace ready for the next call
+  const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
+  float4* dst = reinterpret_cast<float4*>(p.out + (int64_t(b) * p.H + hg * kHeadsPerCta + hh) * kD) + 4 * lane;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    dst[u] = make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
+  if (p.lse != nullptr && lane == 0)
+    p.lse[int64_t(b) * p.H + hg * kHeadsPerCta + hh] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
 }
 
 template <int MT>
@@ -409,6 +397,9 @@ cudaError_t launch_mt(const AttnParams& p, int n_hg, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_chunks, n_hg, p.B);
   kern<<<grid, kAttnThreads, kSmemAttn, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_chunks == 1) return e;
+  k_attn_combine<<<dim3(kHeadsPerCta / 8, n_hg, p.B), 256, 0, stream>>>(p, n_hg);
   return cudaGetLastError();
 }
 

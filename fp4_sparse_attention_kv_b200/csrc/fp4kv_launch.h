@@ -53,7 +53,7 @@ struct SelectProblem {
   uint32_t* hist;           // [B][4096], zeroed by the last CTA of each segment
   uint32_t* counters;       // [B][4]: n_sure, n_cand, ticket, spare
   int32_t* sure;            // [B][k]
-  int32_t* cand;            // [B][vstride]
+  int32_t* cand;            // [B][vstride] 8-byte candidates ((order key << 32) | index)
   int32_t* out_idx;         // [B][k]
   float* out_score;         // nullable [B][k]
   int slices;
@@ -77,11 +77,10 @@ struct AttnParams {
   float sm_scale;
   float* out;               // [B][H][d]
   float* lse;               // nullable [B][H]
-  // split over chunks of the top_k list; partials merged by the last CTA of each (b, hg)
+  // split over chunks of the top_k list; partials merged by a combine kernel
   int n_chunks;
   float* part_o;            // [B][n_hg][n_chunks][64][d]
   float* part_ml;           // [B][n_hg][n_chunks][64][2]
-  uint32_t* tickets;        // [B][n_hg]
   uint32_t* status;
 };
 cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream);

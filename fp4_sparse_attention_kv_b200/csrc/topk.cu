@@ -141,8 +141,8 @@ __device__ void bitonic_sort_u64(uint64_t* a, int n) {
 
 // Warp-aggregated append of `take` lanes' values into list[counter++]; slots at or beyond
 // `capacity` are never written (the counter still counts them).
-FP4KV_DEV void warp_append(bool take, int32_t v, uint32_t* counter, int32_t* list,
-                           uint32_t capacity) {
+template <typename T>
+FP4KV_DEV void warp_append(bool take, T v, uint32_t* counter, T* list, uint32_t capacity) {
   const uint32_t m = __ballot_sync(0xffffffffu, take);
   if (m == 0) return;
   const int lane = threadIdx.x & 31;
@@ -154,14 +154,104 @@ FP4KV_DEV void warp_append(bool take, int32_t v, uint32_t* counter, int32_t* lis
   if (take && slot < capacity) list[slot] = v;
 }
 
+// candidate = (order key << 32) | value index
+FP4KV_DEV uint32_t cand_key(uint64_t c) { return static_cast<uint32_t>(c >> 32); }
+FP4KV_DEV int32_t cand_idx(uint64_t c) { return static_cast<int32_t>(c & 0xffffffffu); }
+
+template <bool kShared>
+FP4KV_DEV uint64_t load_cand(const uint64_t* c, uint32_t i) {
+  if constexpr (kShared) return c[i];
+  return __ldcg(reinterpret_cast<const unsigned long long*>(c) + i);
+}
+
+// Exact resolution of the candidates (all sharing the top 12 key bits `bstar`): finds the
+// r-th largest key ustar among them and, when that key is tied, the largest position
+// pos_star that is still taken (lowest positions win). Candidates live in shared memory
+// (kShared) or, when too many, in global memory.
+template <bool kShared>
+__device__ void resolve_candidates(const SelectProblem& P, int b, const uint64_t* cand,
+                                   uint32_t n_cand, uint32_t r, int bstar, uint32_t* s_hist,
+                                   uint32_t* s_scan, uint32_t* ustar_out, int64_t* pos_star_out) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = static_cast<uint32_t>(bstar);
+  int consumed = kHistBits;
+  const int widths[3] = {8, 8, 4};
+  uint32_t cnt_eq = 0;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int wbits = widths[pass];
+    const int shift = 32 - consumed - wbits;
+    const int nb = 1 << wbits;
+    for (int i = tid; i < nb; i += kSelThreads) s_hist[i] = 0;
+    __syncthreads();
+    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+      const uint32_t key = cand_key(load_cand<kShared>(cand, c));
+      if ((key >> (shift + wbits)) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    int d;
+    uint32_t ab;
+    find_digit_desc(s_hist, nb, r, &d, &ab, s_scan);
+    r -= ab;
+    cnt_eq = s_hist[d];
+    prefix = (prefix << wbits) | static_cast<uint32_t>(d);
+    consumed += wbits;
+    __syncthreads();
+  }
+  *ustar_out = prefix;
+  *pos_star_out = INT64_MAX;
+  if (r < cnt_eq) {
+    // lowest r positions among the keys equal to ustar: passes of 8 bits over 32 bits
+    uint64_t pprefix = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) s_hist[i] = 0;
+      __syncthreads();
+      for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+        const uint64_t cv = load_cand<kShared>(cand, c);
+        if (cand_key(cv) != prefix) continue;
+        const uint64_t pos = static_cast<uint64_t>(position_of(P, b, cand_idx(cv)));
+        if ((pos >> (shift + 8)) == pprefix) atomicAdd(&s_hist[(pos >> shift) & 255], 1u);
+      }
+      __syncthreads();
+      int d;
+      uint32_t below;
+      find_digit_asc(s_hist, 256, r, &d, &below, s_scan);
+      r -= below;
+      pprefix = (pprefix << 8) | static_cast<uint64_t>(d);
+    }
+    *pos_star_out = static_cast<int64_t>(pprefix);
+  }
+}
+
+template <bool kShared>
+__device__ void collect_candidates(const SelectProblem& P, int b, const uint64_t* cand,
+                                   uint32_t n_cand, bool take_all, uint32_t ustar,
+                                   int64_t pos_star, uint64_t* s_sel, uint32_t* s_cnt) {
+  for (uint32_t c = threadIdx.x; c < n_cand; c += kSelThreads) {
+    const uint64_t cv = load_cand<kShared>(cand, c);
+    const int32_t i = cand_idx(cv);
+    const int64_t pos = position_of(P, b, i);
+    const uint32_t key = cand_key(cv);
+    const bool take = take_all || key > ustar || (key == ustar && pos <= pos_star);
+    if (take) {
+      const uint32_t slot = atomicAdd(s_cnt, 1u);
+      if (slot < kMaxSel) s_sel[slot] = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
+    }
+  }
+}
+
+constexpr int kCandSmem = 6144;  // candidates staged in shared memory when they fit
+constexpr size_t kSelSmem = size_t(kMaxSel) * 8 + size_t(kCandSmem) * 8;
+
 __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs args) {
   const SelectProblem& P = args.p[blockIdx.z];
   const int b = blockIdx.y;
   if (static_cast<int>(blockIdx.x) >= P.slices) return;
-  // the histogram (phase 1 and the radix passes) and the selection buffer (collection and
-  // sort) are never live at the same time: they share one 32 KiB buffer
-  __shared__ uint64_t s_sel[kMaxSel];
+  // s_sel: the selected (position, index) pairs; its first 16 KiB also serve as the
+  // histogram of phase 1 and of the radix passes (never live at the same time).
+  extern __shared__ __align__(16) uint8_t sel_smem[];
+  uint64_t* s_sel = reinterpret_cast<uint64_t*>(sel_smem);
   uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_sel);
+  uint64_t* s_cand = s_sel + kMaxSel;
   __shared__ uint32_t s_scan[96];
   __shared__ uint32_t s_cnt;
   __shared__ bool s_last;
@@ -172,7 +262,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   uint32_t* hist = P.hist + int64_t(b) * kHistBins;
   uint32_t* ctr = P.counters + int64_t(b) * 4;
   int32_t* sure = P.sure + int64_t(b) * P.k;
-  int32_t* cand = P.cand + int64_t(b) * P.vstride;
+  uint64_t* cand = reinterpret_cast<uint64_t*>(P.cand) + int64_t(b) * P.vstride;
 
   // 1. digit of the K-th largest key
   for (int i = tid; i < kHistBins; i += kSelThreads) s_hist[i] = __ldcg(hist + i);
@@ -185,19 +275,31 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   // 2. filter this CTA's slice
   const int64_t lo = n * blockIdx.x / P.slices;
   const int64_t hi = n * (blockIdx.x + 1) / P.slices;
-  for (int64_t base = lo; base < hi; base += kSelThreads) {
-    const int64_t i = base + tid;
-    bool is_sure = false, is_cand = false;
-    if (i < hi) {
-      const float v = vals[i];
-      if (v != -INFINITY || P.mode != 2) {
-        const int digit = static_cast<int>(order_key(v) >> (32 - kHistBits));
+  // all loads of a batch are issued before any append (whose atomics would otherwise keep
+  // the next load from being hoisted, costing one memory round trip per 512 values)
+  constexpr int kBatch = 8;
+  for (int64_t base = lo; base < hi; base += int64_t(kSelThreads) * kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t i = base + int64_t(u) * kSelThreads + tid;
+      v[u] = i < hi ? __ldg(vals + i) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t i = base + int64_t(u) * kSelThreads + tid;
+      bool is_sure = false, is_cand = false;
+      uint32_t key = 0;
+      if (i < hi && (v[u] != -INFINITY || P.mode != 2)) {
+        key = order_key(v[u]);
+        const int digit = static_cast<int>(key >> (32 - kHistBits));
         is_sure = digit > bstar;
         is_cand = digit == bstar;
       }
+      warp_append<int32_t>(is_sure, static_cast<int32_t>(i), &ctr[0], sure, static_cast<uint32_t>(P.k));
+      warp_append<uint64_t>(is_cand, (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(i),
+                            &ctr[1], cand, static_cast<uint32_t>(P.vstride));
     }
-    warp_append(is_sure, static_cast<int32_t>(i), &ctr[0], sure, static_cast<uint32_t>(P.k));
-    warp_append(is_cand, static_cast<int32_t>(i), &ctr[1], cand, static_cast<uint32_t>(P.vstride));
   }
 
   // 3. ticket: the last CTA of this sequence finalises
@@ -213,58 +315,21 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
 
   const uint32_t n_sure = min(__ldcg(&ctr[0]), static_cast<uint32_t>(P.k));
   const uint32_t n_cand = min(__ldcg(&ctr[1]), static_cast<uint32_t>(P.vstride));
-  uint32_t r = static_cast<uint32_t>(P.k) > n_sure ? static_cast<uint32_t>(P.k) - n_sure : 0u;
-  bool take_all = n_cand <= r;
+  const uint32_t r = static_cast<uint32_t>(P.k) > n_sure ? static_cast<uint32_t>(P.k) - n_sure : 0u;
+  const bool take_all = n_cand <= r;
+  const bool in_smem = n_cand <= static_cast<uint32_t>(kCandSmem);
+  if (in_smem) {
+    for (uint32_t c = tid; c < n_cand; c += kSelThreads)
+      s_cand[c] = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + c);
+    __syncthreads();
+  }
   uint32_t ustar = 0;
   int64_t pos_star = INT64_MAX;
   if (!take_all && r > 0) {
-    // exact K-th key among the candidates: remaining 20 key bits in passes of 8, 8, 4
-    uint32_t prefix = static_cast<uint32_t>(bstar);
-    int consumed = kHistBits;
-    const int widths[3] = {8, 8, 4};
-    uint32_t cnt_eq = 0;
-    for (int pass = 0; pass < 3; ++pass) {
-      const int wbits = widths[pass];
-      const int shift = 32 - consumed - wbits;
-      const int nb = 1 << wbits;
-      for (int i = tid; i < nb; i += kSelThreads) s_hist[i] = 0;
-      __syncthreads();
-      for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-        const uint32_t key = order_key(vals[__ldcg(cand + c)]);
-        if ((key >> (shift + wbits)) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
-      }
-      __syncthreads();
-      int d;
-      uint32_t ab;
-      find_digit_desc(s_hist, nb, r, &d, &ab, s_scan);
-      r -= ab;
-      cnt_eq = s_hist[d];
-      prefix = (prefix << wbits) | static_cast<uint32_t>(d);
-      consumed += wbits;
-      __syncthreads();
-    }
-    ustar = prefix;
-    if (r < cnt_eq) {
-      // lowest r positions among the keys equal to ustar: passes of 8 bits over 32 bits
-      uint64_t pprefix = 0;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += kSelThreads) s_hist[i] = 0;
-        __syncthreads();
-        for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-          const int32_t i = __ldcg(cand + c);
-          if (order_key(vals[i]) != ustar) continue;
-          const uint64_t pos = static_cast<uint64_t>(position_of(P, b, i));
-          if ((pos >> (shift + 8)) == pprefix) atomicAdd(&s_hist[(pos >> shift) & 255], 1u);
-        }
-        __syncthreads();
-        int d;
-        uint32_t below;
-        find_digit_asc(s_hist, 256, r, &d, &below, s_scan);
-        r -= below;
-        pprefix = (pprefix << 8) | static_cast<uint64_t>(d);
-      }
-      pos_star = static_cast<int64_t>(pprefix);
-    }
+    if (in_smem)
+      resolve_candidates<true>(P, b, s_cand, n_cand, r, bstar, s_hist, s_scan, &ustar, &pos_star);
+    else
+      resolve_candidates<false>(P, b, cand, n_cand, r, bstar, s_hist, s_scan, &ustar, &pos_star);
   }
 
   // collect the selected (position, value index) pairs
@@ -277,20 +342,10 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
       s_sel[slot] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
   }
   if (r > 0 || take_all) {
-    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-      const int32_t i = __ldcg(cand + c);
-      bool take = take_all;
-      const int64_t pos = position_of(P, b, i);
-      if (!take) {
-        const uint32_t key = order_key(vals[i]);
-        take = key > ustar || (key == ustar && pos <= pos_star);
-      }
-      if (take) {
-        const uint32_t slot = atomicAdd(&s_cnt, 1u);
-        if (slot < kMaxSel)
-          s_sel[slot] = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
-      }
-    }
+    if (in_smem)
+      collect_candidates<true>(P, b, s_cand, n_cand, take_all, ustar, pos_star, s_sel, &s_cnt);
+    else
+      collect_candidates<false>(P, b, cand, n_cand, take_all, ustar, pos_star, s_sel, &s_cnt);
   }
   __syncthreads();
   int m = static_cast<int>(s_cnt);
@@ -337,7 +392,10 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
     if (probs[i].slices > gx) gx = probs[i].slices;
   }
   dim3 grid(gx, B, n_probs);
-  k_topk_select<<<grid, kSelThreads, 0, stream>>>(args);
+  cudaError_t e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSelSmem));
+  if (e != cudaSuccess) return e;
+  k_topk_select<<<grid, kSelThreads, kSelSmem, stream>>>(args);
   return cudaGetLastError();
 }
 
