@@ -41,6 +41,8 @@ SIGNATURES = [
      [_P, _P, _I32, _P, _I32, _P, _I64, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     ("fp4kv_sparse_attn_decode", ctypes.c_int,
      [_P, _I32, _I32, _I32, _P, _P, _I64, _P, _P, _I32, _F32, _P, _P, _P, _SZ, _P]),
+    ("fp4kv_indexer_topk_noalloc", ctypes.c_int,
+     [_P, _P, _I32, _P, _I32, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _P, _P, _P]),
     ("fp4kv_profile_enable", ctypes.c_int, [_I32]),
     ("fp4kv_profile_read", ctypes.c_int, [ctypes.POINTER(_I32), ctypes.POINTER(_F32)]),
 ]
@@ -273,3 +275,26 @@ def profile_read() -> dict:
     ms = (ctypes.c_float * 4)()
     _check(lib().fp4kv_profile_read(n, ms))
     return {KERNEL_KINDS[i]: (int(n[i]), float(ms[i])) for i in range(4)}
+
+
+def indexer_topk_noalloc(q, w, keys, seq_lens, top_k, pool=None, block_size=8, key_scale=None,
+                         out_idx=None, out_score=None):
+    """Same as ``indexer_topk`` but without a workspace: the library uses its own fixed 8 MiB
+    device scratch (for callers that cannot allocate device memory). Calls on one device
+    must not overlap on the GPU. Output tensors, when not given, are allocated here by torch
+    for convenience; pass them to keep the call itself allocation-free."""
+    kd, B, cap, H_I = _check_indexer(q, w, keys, seq_lens, key_scale)
+    npb = 0
+    if pool is not None:
+        _need(pool, torch.int32, "pool", keys.device)
+        npb = pool.shape[1]
+    if out_idx is None:
+        out_idx = torch.empty((B, top_k), dtype=torch.int32, device=keys.device)
+    _need(out_idx, torch.int32, "out_idx", keys.device)
+    if out_score is not None:
+        _need(out_score, torch.float32, "out_score", keys.device)
+    _check(lib().fp4kv_indexer_topk_noalloc(_ptr(q), _ptr(w), H_I, _ptr(keys), kd, _ptr(key_scale),
+                                            cap, _ptr(seq_lens), B, _ptr(pool), npb, block_size,
+                                            top_k, _ptr(out_idx), _ptr(out_score),
+                                            _stream(keys.device)))
+    return out_idx

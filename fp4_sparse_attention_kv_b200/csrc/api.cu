@@ -443,6 +443,80 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
   return ok();
 }
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of fp4kv_indexer_topk.
+//
+// Some callers cannot allocate device memory at all: code embedded in a host runtime that
+// owns every byte of device memory (a serving engine with a fixed, pre-reserved pool, or a
+// plugin interface that hands out no allocator), and latency-critical decode loops where
+// cudaMalloc's implicit device-wide synchronisation is not acceptable. For them the
+// scratch of the indexer top-K lives in this file-scope device array instead of a
+// caller-provided workspace. Every GPU that loads the library holds these bytes until the
+// process exits.
+// ---------------------------------------------------------------------------------------
+constexpr size_t kNoAllocBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_ws[kNoAllocBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[256] = {};
+
+// Device address of g_noalloc_ws on the current device, looked up once per device (with
+// that device current). In host code the array's name is only a host-side stand-in.
+fp4kv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 256) return fail(FP4KV_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+    if (e != cudaSuccess || p == nullptr)
+      return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                       "indexer_topk_noalloc: cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP4KV_OK;
+}
+}  // namespace
+
+fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H_I,
+                                        const void* keys, int32_t key_dtype,
+                                        const float* key_scale, int64_t cap,
+                                        const int32_t* seq_lens, int32_t B, const int32_t* pool,
+                                        int32_t n_pool_blocks, int32_t block_size, int32_t top_k,
+                                        int32_t* out_idx, float* out_score, void* stream) {
+  fp4kv_status st = check_indexer_args(q, w, H_I, keys, key_dtype, cap, seq_lens, B);
+  if (st != FP4KV_OK) return st;
+  if (!out_idx) return fail(FP4KV_ERR_INVALID_ARG, "null out_idx");
+  if (top_k < 1 || top_k > 4096) return fail(FP4KV_ERR_UNSUPPORTED, "top_k=%d outside [1, 4096]", top_k);
+  if (pool) {
+    if (block_size != 8) return fail(FP4KV_ERR_UNSUPPORTED, "block_size=%d (only 8)", block_size);
+    if (n_pool_blocks < 1 || n_pool_blocks > 4096)
+      return fail(FP4KV_ERR_UNSUPPORTED, "n_pool_blocks=%d outside [1, 4096]", n_pool_blocks);
+  }
+  const int kind = pool ? 1 : 0;
+  const IndexerLayout L = indexer_layout(kind, B, cap, top_k, pool ? n_pool_blocks : 0);
+  if (L.total > kNoAllocBytes)
+    return fail(FP4KV_ERR_UNSUPPORTED,
+                "indexer_topk_noalloc: these sizes need %zu bytes of scratch, above the built-in "
+                "maximum of %zu (use fp4kv_indexer_topk with a caller workspace)",
+                L.total, kNoAllocBytes);
+  void* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != FP4KV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word and the histogram + counters must start at zero
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.sure - L.hist, s);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: clearing scratch");
+  return run_indexer(kind, q, w, H_I, keys, key_dtype, key_scale, cap, seq_lens, B, pool,
+                     pool ? n_pool_blocks : 0, top_k, out_idx, nullptr, out_score, ws, L.total, s);
+}
+
 fp4kv_status fp4kv_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> g(prof::mu);
   prof::enabled = on != 0;

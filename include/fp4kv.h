@@ -177,6 +177,28 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
                                       float sm_scale, float* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* indexer_topk_noalloc -- fp4kv_indexer_topk without a caller workspace. (The pages have
+ * no counterpart: this is an integration aid.) For callers that cannot allocate device
+ * memory: code inside a host runtime that owns all device memory (a serving engine with a
+ * fixed pre-reserved pool, a plugin interface without an allocator), or latency-critical
+ * decode loops that cannot afford cudaMalloc's implicit device-wide synchronisation.
+ * Arguments and results are those of fp4kv_indexer_topk minus ws / ws_bytes. The scratch is
+ * a file-scope device array of 8 MiB that every GPU loading the library keeps until the
+ * process exits; sizes whose workspace (fp4kv_workspace_bytes of the same op) exceeds 8 MiB
+ * return FP4KV_ERR_UNSUPPORTED with an explanatory message. The call allocates nothing: it
+ * clears the scratch's counters with cudaMemsetAsync on `stream` and launches the same
+ * kernels as fp4kv_indexer_topk. The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current) and caches it; make that first
+ * call before any stream capture. All calls on a device share the one array, so calls whose
+ * kernels overlap on the GPU (different streams, or different host threads) race and give
+ * wrong results: serialise them. */
+fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H_I,
+                                        const void* keys, int32_t key_dtype,
+                                        const float* key_scale, int64_t cap,
+                                        const int32_t* seq_lens, int32_t B, const int32_t* pool,
+                                        int32_t n_pool_blocks, int32_t block_size, int32_t top_k,
+                                        int32_t* out_idx, float* out_score, void* stream);
+
 /* Benchmark support (no counterpart on the pages). While enabled, every kernel the library
  * launches is bracketed by two CUDA events recorded on the launch stream (do not enable
  * during CUDA-graph capture). fp4kv_profile_read waits for the recorded events and returns,
