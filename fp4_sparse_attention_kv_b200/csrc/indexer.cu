@@ -10,17 +10,19 @@
 //    layers score only inside the candidate pool.
 // The head-combining rule (weighted sum of ReLU dot products) is this library's reading.
 //
-// Kernel (one persistent CTA per SM, warp-specialised, 6 warps):
+// Kernel (persistent, two CTAs per SM for E4M3 keys, warp-specialised, 6 warps):
 //  * warp 0 (one lane): TMA producer. Streams 128-row key tiles (16 KiB of E4M3 or 32 KiB of
-//    bf16, 128-byte swizzled) plus the tile's query block into a shared-memory ring. Full
-//    mode: one box per tile; Reindex mode: one 8-row box (1 KiB) per pool block.
+//    bf16, 128-byte swizzled) into a shared-memory ring as deep as shared memory allows, and
+//    each sequence's query block into one of two query slots. Full mode: one box per tile;
+//    Reindex mode: one 8-row box (1 KiB) per pool block.
 //  * warp 1: allocates TMEM; one lane issues tcgen05.mma (M = 128 entries, N = padded head
 //    count, K = 128 dims; kind::f8f6f4 on E4M3 directly, kind::f16 on bf16) into a ring of
 //    fp32 accumulators in TMEM, and commits to the ring's mbarriers.
-//  * warps 2-5: epilogue. Each thread owns one row (TMEM lane): loads its N head dot
-//    products, combines heads, writes the fp32 score, and adds the score's top 12 key bits to
-//    a shared-memory histogram flushed per sequence (first pass of the exact top-K). With a
-//    block-max output it reduces each block of 8 rows across 8 lanes and histograms those.
+//  * warps 2-5: the epilogue warpgroup. Each thread owns one row
+//    (TMEM lane): loads its N head dot products, combines heads, writes the fp32 score, and
+//    adds the score's top 12 key bits to its warpgroup's shared-memory histogram, flushed per
+//    sequence (first pass of the exact top-K). With a block-max output it reduces each block
+//    of 8 rows across 8 lanes and histograms those.
 // Every wait is bounded in time; on timeout the kernel sets a status bit and winds down.
 #include <cstdio>
 
@@ -33,25 +35,38 @@ namespace {
 
 constexpr int kTileRows = 128;
 constexpr int kPoolBlock = 8;
-constexpr int kThreads = 192;  // producer, mma, 4 epilogue warps
+constexpr int kEpiGroups = 1;   // epilogue warpgroups (alternating tiles when > 1)
 constexpr int kEpiThreads = 128;
-constexpr int kAccCols = 256;  // TMEM columns allocated (ring of accumulators)
+constexpr int kThreads = 64 + kEpiGroups * kEpiThreads;  // producer, mma, epilogue groups
+constexpr int kAccCols = 256;  // TMEM columns allocated per CTA (ring of accumulators)
+constexpr size_t kSmemPerSm = 227 * 1024;
 
+// Two CTAs per SM for E4M3 keys: each CTA's single MMA-issuing thread serialises its
+// wait -> issue -> commit chain per tile, and two independent chains per SM keep the
+// stream near the HBM rate where one deep ring could not. The bf16 (small) case keeps one
+// CTA per SM so that its 32 KiB stages fit.
 template <bool FP8, int N>
 struct ScanCfg {
+  static constexpr int kCtasPerSm = FP8 ? 2 : 1;
+  static constexpr size_t kSmemBudget = kSmemPerSm / kCtasPerSm - 1024;
   static constexpr int kRowBytes = FP8 ? 128 : 256;
   static constexpr int kKeyBytes = kTileRows * kRowBytes;  // one stage of keys
-  static constexpr int kQBytes = N * kRowBytes;            // the stage's query block
-  static constexpr int kStageBytes = kKeyBytes + kQBytes;
-  static constexpr int kStages = FP8 ? 6 : 3;
+  static constexpr int kQBytes = N * kRowBytes;            // one query block (per sequence)
+  static constexpr int kStageBytes = kKeyBytes;
+  static constexpr size_t kHistBytes = size_t(2 * kEpiGroups) * kHistBins * sizeof(uint32_t);
+  static constexpr size_t kFixed = 1024 + 2 * size_t(kQBytes) + kHistBytes + 1024;
+  static constexpr int kStagesFit = static_cast<int>((kSmemBudget - kFixed) / kStageBytes);
+  static constexpr int kStages = kStagesFit > 16 ? 16 : kStagesFit;
   static constexpr int kAccSlots = kAccCols / N;
-  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes +
-                                  (2 * kStages + 2 * kAccSlots) * sizeof(uint64_t) +
-                                  2 * kHistBins * sizeof(uint32_t) + 64;
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + 2 * size_t(kQBytes) +
+                                  (2 * kStages + 2 * kAccSlots + 4) * sizeof(uint64_t) + kHistBytes + 64;
+  static_assert(kStages >= 2, "shared memory budget");
+  static_assert(kSmem <= kSmemBudget, "shared memory budget");
   static constexpr uint32_t kIdesc = umma_idesc(FP8 ? 0u : 1u, 128, N);
 };
 
-FP4KV_DEV void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads)); }
+// named barrier of one epilogue warpgroup (ids 1 and 2)
+FP4KV_DEV void epi_sync(int group) { asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(kEpiThreads)); }
 
 struct Tiles {
   int64_t begin, end, per_seq;
@@ -85,7 +100,7 @@ FP4KV_DEV int64_t seq_len_of(const IndexScoreParams& p, int b) {
 }
 
 template <bool FP8, int N>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, ScanCfg<FP8, N>::kCtasPerSm)
     k_index_score_tc(const IndexScoreParams p, const __grid_constant__ CUtensorMap tm_keys,
                      const __grid_constant__ CUtensorMap tm_q, int64_t tiles_per_seq,
                      int64_t total_tiles) {
@@ -93,13 +108,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + size_t(Cfg::kStages) * Cfg::kStageBytes);
+  uint8_t* qbuf = ring + size_t(Cfg::kStages) * Cfg::kStageBytes;  // 2 query slots
+  uint64_t* full = reinterpret_cast<uint64_t*>(qbuf + 2 * size_t(Cfg::kQBytes));
   uint64_t* empty = full + Cfg::kStages;
   uint64_t* tfull = empty + Cfg::kStages;
   uint64_t* tempty = tfull + Cfg::kAccSlots;
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(tempty + Cfg::kAccSlots);
-  uint32_t* s_bhist = s_hist + kHistBins;
-  uint32_t* s_tmem = s_bhist + kHistBins;
+  uint64_t* qfull = tempty + Cfg::kAccSlots;  // [2]
+  uint64_t* qempty = qfull + 2;               // [2]
+  uint32_t* s_hist_all = reinterpret_cast<uint32_t*>(qempty + 2);  // [group][2][bins]
+  uint32_t* s_tmem = s_hist_all + 2 * kEpiGroups * kHistBins;
   volatile uint32_t* s_abort = s_tmem + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,14 +133,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < Cfg::kAccSlots; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], 4);  // one arrival per warp of the tile's epilogue warpgroup
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&qfull[j], 1);
+      mbar_init(&qempty[j], 1);
     }
     *s_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_keys);
     prefetch_tmap(&tm_q);
   }
-  for (int i = threadIdx.x; i < 2 * kHistBins; i += blockDim.x) s_hist[i] = 0;
+  for (int i = threadIdx.x; i < 2 * kEpiGroups * kHistBins; i += blockDim.x) s_hist_all[i] = 0;
   if (warp == 1) {
     tmem_alloc(s_tmem, kAccCols);
     tmem_relinquish();
@@ -136,12 +157,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------- TMA producer ----------------------------------
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, nq = 0;  // tiles issued, query blocks issued
+      int cur_b = -1, q_b = -1;
+      int64_t len = 0;
       TileIter ti;
       for (ti.init(T); !ti.done(); ti.next()) {
-        const int64_t len = seq_len_of(p, ti.b);
+        if (ti.b != cur_b) {
+          cur_b = ti.b;
+          len = seq_len_of(p, cur_b);
+        }
         const int64_t unit = pool_mode ? ti.tis * (kTileRows / kPoolBlock) : ti.tis * kTileRows;
         if (!pool_mode && unit >= len) continue;
+        if (ti.b != q_b) {
+          // first active tile of a sequence: its query block into the next slot, once the
+          // MMA issuer has released that slot's previous query block
+          const int slot = nq & 1;
+          if (!mbar_wait_timed(&qempty[slot], ((nq >> 1) & 1) ^ 1)) {
+            atomicOr(p.status, kFlagWaitTimeout);
+            *s_abort = 1;
+            break;
+          }
+          uint8_t* qdst = qbuf + size_t(slot) * Cfg::kQBytes;
+          const int32_t qy = ti.b * p.H_I;
+          mbar_arrive_expect_tx(&qfull[slot], Cfg::kQBytes);
+          if constexpr (FP8) {
+            tma_load_2d(qdst, &tm_q, 0, qy, &qfull[slot]);
+          } else {
+            tma_load_2d(qdst, &tm_q, 0, qy, &qfull[slot]);
+            tma_load_2d(qdst + Cfg::kQBytes / 2, &tm_q, 64, qy, &qfull[slot]);
+          }
+          q_b = ti.b;
+          ++nq;
+        }
         const int stage = it % Cfg::kStages;
         const uint32_t ph = (it / Cfg::kStages) & 1;
         ++it;
@@ -152,10 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* dst = ring + size_t(stage) * Cfg::kStageBytes;
         const int32_t row_base = static_cast<int32_t>(int64_t(ti.b) * p.cap);
-        uint32_t bytes = Cfg::kQBytes;
         if (!pool_mode) {
-          bytes += Cfg::kKeyBytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
+          mbar_arrive_expect_tx(&full[stage], Cfg::kKeyBytes);
           const int32_t y = row_base + static_cast<int32_t>(unit);
           if constexpr (FP8) {
             tma_load_2d(dst, &tm_keys, 0, y, &full[stage]);
@@ -166,44 +211,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int32_t* pl = p.pool + int64_t(ti.b) * p.npb;
           int32_t blk[kTileRows / kPoolBlock];
-          for (int s = 0; s < kTileRows / kPoolBlock; ++s) {
-            const int64_t slot = unit + s;
+          uint32_t bytes = 0;
+          for (int s2 = 0; s2 < kTileRows / kPoolBlock; ++s2) {
+            const int64_t slot = unit + s2;
             int32_t j = slot < p.npb ? pl[slot] : -1;
             if (j < 0 || int64_t(j) * kPoolBlock >= p.cap) j = -1;
-            blk[s] = j;
+            blk[s2] = j;
             if (j >= 0) bytes += kPoolBlock * Cfg::kRowBytes;
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          for (int s = 0; s < kTileRows / kPoolBlock; ++s) {
-            if (blk[s] < 0) continue;
-            const int32_t y = row_base + blk[s] * kPoolBlock;
+          for (int s2 = 0; s2 < kTileRows / kPoolBlock; ++s2) {
+            if (blk[s2] < 0) continue;
+            const int32_t y = row_base + blk[s2] * kPoolBlock;
             if constexpr (FP8) {
-              tma_load_2d(dst + s * 1024, &tm_keys, 0, y, &full[stage]);
+              tma_load_2d(dst + s2 * 1024, &tm_keys, 0, y, &full[stage]);
             } else {
-              tma_load_2d(dst + s * 1024, &tm_keys, 0, y, &full[stage]);
-              tma_load_2d(dst + Cfg::kKeyBytes / 2 + s * 1024, &tm_keys, 64, y, &full[stage]);
+              tma_load_2d(dst + s2 * 1024, &tm_keys, 0, y, &full[stage]);
+              tma_load_2d(dst + Cfg::kKeyBytes / 2 + s2 * 1024, &tm_keys, 64, y, &full[stage]);
             }
           }
-        }
-        // the sequence's query block (rows beyond the last sequence are zero-filled)
-        uint8_t* qdst = dst + Cfg::kKeyBytes;
-        const int32_t qy = ti.b * p.H_I;
-        if constexpr (FP8) {
-          tma_load_2d(qdst, &tm_q, 0, qy, &full[stage]);
-        } else {
-          tma_load_2d(qdst, &tm_q, 0, qy, &full[stage]);
-          tma_load_2d(qdst + Cfg::kQBytes / 2, &tm_q, 64, qy, &full[stage]);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer ------------------------------------
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, nseg = 0;
+      int cur_b = -1, qslot = 0;
+      int64_t len = 0;
+      bool have_q = false;
       TileIter ti;
       for (ti.init(T); !ti.done(); ti.next()) {
-        if (!pool_mode && ti.tis * kTileRows >= seq_len_of(p, ti.b)) continue;
+        if (ti.b != cur_b) {
+          cur_b = ti.b;
+          len = seq_len_of(p, cur_b);
+          if (have_q) umma_commit(&qempty[qslot]);  // previous sequence's query block free
+          have_q = false;
+        }
+        if (!pool_mode && ti.tis * kTileRows >= len) continue;
         if (*s_abort) break;
+        if (!have_q) {
+          qslot = nseg & 1;
+          if (!mbar_wait_timed(&qfull[qslot], (nseg >> 1) & 1)) {
+            atomicOr(p.status, kFlagWaitTimeout);
+            *s_abort = 1;
+            break;
+          }
+          ++nseg;
+          have_q = true;
+        }
         const int stage = it % Cfg::kStages;
         const uint32_t ph = (it / Cfg::kStages) & 1;
         const int acc = it % Cfg::kAccSlots;
@@ -216,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t a0 = smem_u32(ring + size_t(stage) * Cfg::kStageBytes);
-        const uint32_t b0 = a0 + Cfg::kKeyBytes;
+        const uint32_t b0 = smem_u32(qbuf + size_t(qslot) * Cfg::kQBytes);
         const uint32_t d = tmem_base + uint32_t(acc * N);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {  // 4 x 32 bytes of K per 128-byte swizzle row
@@ -235,19 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&empty[stage]);
         umma_commit(&tfull[acc]);
       }
+      if (have_q) umma_commit(&qempty[qslot]);
     }
   } else {
-    // ------------------------------- epilogue (warps 2..5) -------------------------
+    // ------------------------------- epilogue (2 warpgroups) -----------------------
+    const int group = (warp - 2) >> 2;          // warpgroup: tiles it % kEpiGroups == group
+    const int gtid = threadIdx.x - 64 - group * kEpiThreads;
     const int quarter = warp & 3;               // TMEM lanes [32*quarter, +32)
     const int row = 32 * quarter + lane;        // tile row owned by this thread
     const uint32_t lane_addr = uint32_t(32 * quarter) << 16;
+    uint32_t* s_hist = s_hist_all + 2 * group * kHistBins;
+    uint32_t* s_bhist = s_hist + kHistBins;
     float wv[N];
     int cur_b = -1;
     uint32_t it = 0;
     TileIter ti;
     auto flush = [&](int b) {
-      epi_sync();
-      for (int i = threadIdx.x - 64; i < kHistBins; i += kEpiThreads) {
+      epi_sync(group);
+      for (int i = gtid; i < kHistBins; i += kEpiThreads) {
         const uint32_t c = s_hist[i];
         if (c) atomicAdd(p.hist + int64_t(b) * kHistBins + i, c);
         s_hist[i] = 0;
@@ -257,15 +318,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           s_bhist[i] = 0;
         }
       }
-      epi_sync();
+      epi_sync(group);
     };
+    int len_b = -1;
+    int64_t len = 0;
     for (ti.init(T); !ti.done(); ti.next()) {
-      const int64_t len = seq_len_of(p, ti.b);
+      if (ti.b != len_b) {
+        len_b = ti.b;
+        len = seq_len_of(p, len_b);
+      }
       if (!pool_mode && ti.tis * kTileRows >= len) continue;
+      const uint32_t my = it++;
+      if ((my % kEpiGroups) != static_cast<uint32_t>(group)) continue;
       if (*s_abort) break;
-      const int acc = it % Cfg::kAccSlots;
-      const uint32_t aph = (it / Cfg::kAccSlots) & 1;
-      ++it;
+      const int acc = my % Cfg::kAccSlots;
+      const uint32_t aph = (my / Cfg::kAccSlots) & 1;
       if (ti.b != cur_b) {
         if (cur_b >= 0 && p.hist != nullptr) flush(cur_b);
         cur_b = ti.b;
@@ -278,18 +345,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float s = 0.0f;
+      uint32_t r[N];
 #pragma unroll
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem_base + lane_addr + uint32_t(acc * N + c0), r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) s += wv[c0 + j] * fmaxf(__uint_as_float(r[j]), 0.0f);
-      }
+      for (int c0 = 0; c0 < N; c0 += 16)
+        tmem_ld16(tmem_base + lane_addr + uint32_t(acc * N + c0),
+                  *reinterpret_cast<uint32_t(*)[16]>(&r[c0]));
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      // four independent FMA chains, combined in a fixed order
+      float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int h = 0; h < N; ++h) part[h & 3] += wv[h] * fmaxf(__uint_as_float(r[h]), 0.0f);
+      float s = (part[0] + part[1]) + (part[2] + part[3]);
 
       const int64_t seq_base = int64_t(ti.b) * p.cap;
       float* srow = p.scores + int64_t(ti.b) * p.score_stride;
@@ -386,7 +455,7 @@ cudaError_t launch_n(const IndexScoreParams& p, int num_sms, cudaStream_t stream
   if (!make_map(&tk, p.keys, !FP8, kKeyDim, uint64_t(p.B) * uint64_t(p.cap), pool_mode ? kPoolBlock : kTileRows) ||
       !make_map(&tq, p.q, !FP8, kKeyDim, uint64_t(p.B) * uint64_t(p.H_I), N))
     return cudaErrorInvalidValue;
-  int grid = num_sms;
+  int grid = num_sms * Cfg::kCtasPerSm;
   if (total < grid) grid = static_cast<int>(total);
   auto kern = k_index_score_tc<FP8, N>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

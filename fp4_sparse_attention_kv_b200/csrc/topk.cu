@@ -123,20 +123,59 @@ __device__ void find_digit_asc(const uint32_t* h, int nbins, uint32_t r, int* d_
   __syncthreads();
 }
 
-__device__ void bitonic_sort_u64(uint64_t* a, int n) {
-  for (int size = 2; size <= n; size <<= 1) {
+// Block-wide ascending bitonic sort of N = kSelThreads * E keys held in shared memory.
+// Each thread keeps E consecutive keys in registers: strides below E are exchanged inside
+// the thread, strides up to 16 E through warp shuffles, and only the widest strides through
+// shared memory (one barrier pair each). Every stage is unrolled at compile time.
+template <typename T, int E>
+__device__ void block_sort(T* s) {
+  constexpr int N = kSelThreads * E;
+  const int tid = threadIdx.x;
+  T v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = s[tid * E + e];
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool asc = (i & size) == 0;
-          const uint64_t x = a[i], y = a[j];
-          if ((x > y) == asc) { a[i] = y; a[j] = x; }
+      if (stride >= 32 * E) {
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) s[tid * E + e] = v[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const T p = s[i ^ stride];
+          const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
+          v[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
         }
+      } else if (stride >= E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const T p = __shfl_xor_sync(0xffffffffu, v[e], stride / E);
+          const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
+          v[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
+        }
+      } else {
+        T nv[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const T p = v[e ^ stride];
+          const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
+          nv[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = nv[e];
       }
-      __syncthreads();
     }
   }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e) s[tid * E + e] = v[e];
+  __syncthreads();
 }
 
 // Warp-aggregated append of `take` lanes' values into list[counter++]; slots at or beyond
@@ -350,20 +389,39 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   __syncthreads();
   int m = static_cast<int>(s_cnt);
   if (m > P.k) m = P.k;
-  int npow = 1;
-  while (npow < m) npow <<= 1;
-  for (int i = m + tid; i < npow; i += kSelThreads) s_sel[i] = ~0ull;
-  __syncthreads();
-  bitonic_sort_u64(s_sel, npow);
+  const int nsort = m <= kSelThreads * 4 ? kSelThreads * 4 : kSelThreads * 8;
   int32_t* oi = P.out_idx + int64_t(b) * P.k;
   float* os = P.out_score ? P.out_score + int64_t(b) * P.k : nullptr;
-  for (int j = tid; j < P.k; j += kSelThreads) {
-    if (j < m) {
-      oi[j] = static_cast<int32_t>(s_sel[j] >> 32);
-      if (os) os[j] = vals[static_cast<uint32_t>(s_sel[j] & 0xffffffffu)];
-    } else {
-      oi[j] = -1;
-      if (os) os[j] = -INFINITY;
+  if (P.mode != 2) {
+    // position == value index: sort 32-bit positions (padding sorts last)
+    uint32_t* s_pos = reinterpret_cast<uint32_t*>(s_cand);
+    for (int i = tid; i < nsort; i += kSelThreads)
+      s_pos[i] = i < m ? static_cast<uint32_t>(s_sel[i] >> 32) : 0xffffffffu;
+    __syncthreads();
+    if (nsort == kSelThreads * 4) block_sort<uint32_t, 4>(s_pos);
+    else block_sort<uint32_t, 8>(s_pos);
+    for (int j = tid; j < P.k; j += kSelThreads) {
+      if (j < m) {
+        oi[j] = static_cast<int32_t>(s_pos[j]);
+        if (os) os[j] = vals[s_pos[j]];
+      } else {
+        oi[j] = -1;
+        if (os) os[j] = -INFINITY;
+      }
+    }
+  } else {
+    for (int i = m + tid; i < nsort; i += kSelThreads) s_sel[i] = ~0ull;
+    __syncthreads();
+    if (nsort == kSelThreads * 4) block_sort<uint64_t, 4>(s_sel);
+    else block_sort<uint64_t, 8>(s_sel);
+    for (int j = tid; j < P.k; j += kSelThreads) {
+      if (j < m) {
+        oi[j] = static_cast<int32_t>(s_sel[j] >> 32);
+        if (os) os[j] = vals[static_cast<uint32_t>(s_sel[j] & 0xffffffffu)];
+      } else {
+        oi[j] = -1;
+        if (os) os[j] = -INFINITY;
+      }
     }
   }
   // leave the workspace zeroed for the next call
