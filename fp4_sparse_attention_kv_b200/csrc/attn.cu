@@ -13,394 +13,613 @@
 //  * q (bf16) is multiplied per head by a power of two 2^k so that max|q| lies in
 //    [2^14, 2^15), then rounded to fp16: exact for every element within 2^29 of the head's
 //    max; 2^-k is folded back into the logit scale.
-//  * S = q . v_hat on tensor cores (fp16 x fp16 -> fp32); online softmax in fp32 with exp2.
-//  * P is split as P_hi + P_lo, both fp16, after scaling by 2^8 (P_lo stays out of the fp16
-//    subnormal range); P.V is two MMAs, so P carries ~22 bits into the product.
+//  * S = q . v_hat on tensor cores (fp16 x fp16 -> fp32); softmax in fp32 with exp2 against a
+//    per-head reference m. The reference moves only when a logit exceeds it by more than 2^9
+//    (so p < 2^9); it is then set 2^3 above the new maximum, and O and the row sums are
+//    rescaled once for every head that moved.
+//  * P is split as P_hi + P_lo, both fp16, after scaling by 2^6 (fp16 stays in range and P_lo
+//    out of the subnormal range); P.V is two MMAs, so P carries ~22 bits into the product.
 //
-// Work split: CTA = (chunk of the index list, group of <= 64 heads, sequence); 8 warps.
-// Per sub-tile of 64 entries: the warps gather packed rows + scales with coalesced 16-byte
-// loads and write fp16 rows into an XOR-swizzled shared buffer (conflict-free for stores and
-// for ldmatrix); S = Q V^T (m16n8k16 MMAs), per-head running max / sum, P to shared memory,
-// O += P V. Each chunk writes its unnormalised O with (max, sum); a small second kernel
-// (k_attn_combine, one warp per head) merges the chunks. No CTA waits on another.
+// Kernel (one CTA per (chunk of the index list, group of 64 heads, sequence); 13 warps):
+//  * the tile is 128 selected entries. S^T = V_hat Q^T (M = 128 entries, N = 64 heads,
+//    K = 512) and O^T += V_hat^T P^T (M = 128 dims x 4, N = 64 heads, K = 128 entries) run on
+//    tcgen05 with fp32 accumulators in TMEM (O^T: 256 columns; S^T: two 64-column slots).
+//  * warps 8-11 gather: each thread loads one selected row (256 B codes + 32 B scales) with
+//    16-byte loads, dequantizes it 64 dims at a time into a 128-byte-swizzled fp16 chunk
+//    buffer (8 chunks = the tile's 128 KiB V_hat) that serves as the K-major A operand of
+//    S^T and as the MN-major A operand of O^T;
+//  * warp 12: TMEM allocation and the single MMA-issuing thread;
+//  * warps 0-7 convert Q, then own the 128 TMEM lanes in pairs (warp w: lane quarter w % 4,
+//    heads 32 (w / 4) .. + 32): per tile each thread reads its entry's 32 logits, keeps 32
+//    per-head running row sums in registers, and writes its half of the entry's row of P^T
+//    (MN-major B operand). Cross-lane reductions happen only when a reference moves and
+//    once at the end, when O^T is staged in shared memory and leaves in one bulk store.
+//  Per-chunk barriers let the next tile's dequantization overlap the current tile's P.V.
+//  Chunks of the index list go to different CTAs; k_attn_combine merges their partials.
+// Every mbarrier wait is bounded in time. Decisions that lead to a named barrier are made
+// uniform across the softmax warps by a barrier vote, so a timed-out wait cannot strand a
+// warp; on timeout the kernel sets a status bit and winds down.
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
+#include "fp4kv_sm100.cuh"
 
 namespace fp4kv {
 namespace {
 
-constexpr int kD = 512;          // latent width the kernel is built for
-constexpr int kHeadsPerCta = 64;
-constexpr int kSub = 64;         // entries per sub-tile
-constexpr int kAttnThreads = 256;
-constexpr float kPScale = 256.0f;
+constexpr int kD = 512;           // latent width the kernel is built for
+constexpr int kHeadsPerCta = 64;  // N of both MMAs (absent heads are zero rows)
+constexpr int kTile = 128;        // selected entries per tile
+constexpr int kChunks = 8;        // 64-dim chunks of a row
+constexpr float kPScale = 64.0f;  // P is stored as p * 2^6
+constexpr float kMoveLog2 = 9.0f;     // a logit above m + 9 moves the reference ...
+constexpr float kHeadroomLog2 = 3.0f; // ... to 3 above the new maximum
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kSoftWarps = 8;
+constexpr int kGatherWarps = 4;
+constexpr int kMmaWarp = kSoftWarps + kGatherWarps;
+constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 416
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr uint32_t kFlagMisaligned = 2u;
 
-constexpr size_t kSmemQ = size_t(kHeadsPerCta) * kD * 2;
-constexpr size_t kSmemV = size_t(kSub) * kD * 2;
-constexpr size_t kSmemP = size_t(kHeadsPerCta) * kSub * 2;
-constexpr size_t kSmemAttn = kSmemQ + kSmemV + 2 * kSmemP + 64 * 4 + 8 * 16 * 4 + 64 * 4 + 16;
+constexpr uint32_t kQChunkBytes = kHeadsPerCta * 128;  // 64 heads x 64 dims x 2 B
+constexpr uint32_t kVChunkBytes = kTile * 128;         // 128 entries x 64 dims x 2 B
+constexpr uint32_t kPBytes = kTile * 128;              // 128 entries x 64 heads x 2 B
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffV = kOffQ + kChunks * kQChunkBytes;
+constexpr uint32_t kOffPh = kOffV + kChunks * kVChunkBytes;
+constexpr uint32_t kOffPl = kOffPh + kPBytes;
+constexpr uint32_t kOffBar = kOffPl + kPBytes;  // 24 mbarriers
+constexpr uint32_t kOffC = kOffBar + 256;       // [64] log2-domain logit scale per head
+constexpr uint32_t kOffRed = kOffC + 256;       // [4][64] cross-warp exchange
+constexpr uint32_t kOffM = kOffRed + 1024;      // [64] per-head reference (log2 domain)
+constexpr uint32_t kOffA = kOffM + 256;         // [64] rescale factor of the last move
+constexpr uint32_t kOffL = kOffA + 256;         // [64] row sums at the end
+constexpr uint32_t kOffTmem = kOffL + 256;
+constexpr uint32_t kSmemAttn = kOffTmem + 16;
+static_assert(kSmemAttn <= 232448, "shared memory");
+// At the end the V_hat region holds the [64 heads][512 dims] fp32 output tile.
+static_assert(kChunks * kVChunkBytes == kHeadsPerCta * kD * 4, "output staging");
 
-// byte offset of 16-byte chunk `c` of row `r` in a buffer of 1 KiB rows (64 chunks)
-FP4KV_DEV uint32_t off_wide(int r, int c) { return uint32_t(r) * 1024u + (uint32_t(c ^ (r & 7)) << 4); }
-// same for 128-byte rows (8 chunks)
-FP4KV_DEV uint32_t off_narrow(int r, int c) { return uint32_t(r) * 128u + (uint32_t(c ^ (r & 7)) << 4); }
+// TMEM columns: O^T dim-tile c at [64c, 64c + 64); S^T slot u at [256 + 64u, +64)
+constexpr uint32_t kColS = 256;
 
-FP4KV_DEV void ldmatrix_x2(uint32_t& r0, uint32_t& r1, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r0), "=r"(r1) : "r"(addr));
+enum { B_VREADY = 0, B_VFREE = 8, B_SFULL = 16, B_SFREE = 18, B_PREADY = 20, B_PFREE = 21,
+       B_QREADY = 22, B_DONE = 23 };
+
+FP4KV_DEV void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory"); }
+// Barrier among the softmax warps that also ORs a predicate over them.
+FP4KV_DEV bool softmax_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, 1, %2, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(r) : "r"(v ? 1u : 0u), "n"(kSoftThreads) : "memory");
+  return r != 0;
 }
 
-template <int MT>
-__global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(const AttnParams p) {
+// Butterfly transpose-reduction of 32 values per lane across the warp: on return, lane l
+// holds the reduction over all 32 lanes of value l.
+template <bool kMax>
+FP4KV_DEV float butterfly32(const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool hi = lane & 16;
+    const float r = __shfl_xor_sync(0xffffffffu, hi ? v[i] : v[i + 16], 16);
+    const float keep = hi ? v[i + 16] : v[i];
+    a[i] = kMax ? fmaxf(keep, r) : keep + r;
+  }
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 8;
+    const float r = __shfl_xor_sync(0xffffffffu, hi ? a[i] : a[i + 8], 8);
+    const float keep = hi ? a[i + 8] : a[i];
+    b[i] = kMax ? fmaxf(keep, r) : keep + r;
+  }
+  float c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 4;
+    const float r = __shfl_xor_sync(0xffffffffu, hi ? b[i] : b[i + 4], 4);
+    const float keep = hi ? b[i + 4] : b[i];
+    c[i] = kMax ? fmaxf(keep, r) : keep + r;
+  }
+  float d[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 2;
+    const float r = __shfl_xor_sync(0xffffffffu, hi ? c[i] : c[i + 2], 2);
+    const float keep = hi ? c[i + 2] : c[i];
+    d[i] = kMax ? fmaxf(keep, r) : keep + r;
+  }
+  const bool hi = lane & 1;
+  const float r = __shfl_xor_sync(0xffffffffu, hi ? d[0] : d[1], 1);
+  const float keep = hi ? d[1] : d[0];
+  return kMax ? fmaxf(keep, r) : keep + r;
+}
+
+FP4KV_DEV void fail_wait(const AttnParams& p, volatile uint32_t* abort_flag) {
+  atomicOr(p.status, kFlagWaitTimeout);
+  *abort_flag = 1;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sQ = smem;
-  uint8_t* sV = sQ + kSmemQ;
-  uint8_t* sPh = sV + kSmemV;
-  uint8_t* sPl = sPh + kSmemP;
-  float* sC = reinterpret_cast<float*>(sPl + kSmemP);  // [64] log2-domain logit scale
-  float* sRed = sC + 64;                                // [8 warps][16 rows]
-  int32_t* sIdx = reinterpret_cast<int32_t*>(sRed + 128);  // [64] position or -1
+  if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled operand layouts need 1 KiB alignment
+    if (threadIdx.x == 0) atomicOr(p.status, kFlagMisaligned);
+    return;
+  }
+  // The merge kernel that follows waits for this grid to complete; let it be scheduled now.
+  griddep_launch_dependents();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  float* sC = reinterpret_cast<float*>(smem + kOffC);
+  float* sRed = reinterpret_cast<float*>(smem + kOffRed);
+  float* sM = reinterpret_cast<float*>(smem + kOffM);
+  float* sA = reinterpret_cast<float*>(smem + kOffA);
+  float* sL = reinterpret_cast<float*>(smem + kOffL);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
+  volatile uint32_t* s_abort = s_tmem + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, tq = lane & 3;
   const int chunk = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int n_hg = gridDim.y;
+  const int n_hg = gridDim.y, n_chunks = gridDim.x;
   const int hbase = hg * kHeadsPerCta;
   const int nh = min(kHeadsPerCta, p.H - hbase);
   int64_t len = p.seq_lens[b];
   if (len > p.cap) len = p.cap;
-
-  // ---- Q: bf16 -> fp16 with a per-head power-of-two scale, swizzled rows ----
-  for (int hh = warp; hh < kHeadsPerCta; hh += 8) {
-    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
-    float c = 0.0f;
-    if (hh < nh) {
-      const uint16_t* qr = p.q + (int64_t(b) * p.H + hbase + hh) * kD + 16 * lane;
-      const uint4 v0 = *reinterpret_cast<const uint4*>(qr);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(qr + 8);
-      const uint32_t wd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      uint32_t m = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = max(m, max(wd[i] & 0x7fffu, (wd[i] >> 16) & 0x7fffu));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      int k = 0;
-      if (m != 0) {
-        const int e = int((m >> 7) & 0xff) - 127;  // exponent of max|q| (bf16 normal)
-        k = 14 - (e < -126 ? -126 : e);
-        if (k > 127) k = 127;
-        if (k < -126) k = -126;
-      }
-      const float up = __uint_as_float(uint32_t(127 + k) << 23);
-      uint32_t h[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        h[i] = pack_f16x2(bf16_bits_to_f32(wd[i] & 0xffffu) * up, bf16_bits_to_f32(wd[i] >> 16) * up);
-      o0 = make_uint4(h[0], h[1], h[2], h[3]);
-      o1 = make_uint4(h[4], h[5], h[6], h[7]);
-      // 2^-k in two steps so that it never underflows or overflows as a float
-      c = p.sm_scale * kLog2e * __uint_as_float(uint32_t(127 - k / 2) << 23) *
-          __uint_as_float(uint32_t(127 - (k - k / 2)) << 23);
-    }
-    *reinterpret_cast<uint4*>(sQ + off_wide(hh, 2 * lane)) = o0;
-    *reinterpret_cast<uint4*>(sQ + off_wide(hh, 2 * lane + 1)) = o1;
-    if (lane == 0) sC[hh] = c;
-  }
-
-  // ---- per-warp roles ----
-  const int mt = warp % MT;         // m-tile (16 heads) of this warp in both phases
-  const int wi = warp / MT;         // index among the warps sharing the m-tile
-  constexpr int kWarpsPerMt = 8 / MT;
-  constexpr int kNtS = MT;          // S: n-tiles (8 entries) per warp
-  constexpr int kNtO = 8 * MT;      // PV: n-tiles (8 dims) per warp
-  const int dim0 = wi * (kD / kWarpsPerMt);
-
-  float o[kNtO][4];
-#pragma unroll
-  for (int i = 0; i < kNtO; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-  float m_g = -INFINITY, m_g8 = -INFINITY, l_g = 0.0f, l_g8 = 0.0f;
-
-  const int n_chunks = gridDim.x;
   const int e_begin = int(int64_t(p.top_k) * chunk / n_chunks);
   const int e_end = int(int64_t(p.top_k) * (chunk + 1) / n_chunks);
+  const int n_tiles = (e_end - e_begin + kTile - 1) / kTile;
   const int32_t* idx = p.idx + int64_t(b) * p.top_k;
-  const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
-  const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
 
-  for (int st = e_begin; st < e_end; st += kSub) {
-    if (tid < kSub) {
-      const int j = st + tid;
-      int32_t pos = j < e_end ? idx[j] : -1;
-      if (pos < 0 || pos >= len) pos = -1;
-      sIdx[tid] = pos;
+  if (tid == 0) {
+    for (int j = 0; j < kChunks; ++j) {
+      mbar_init(&bars[B_VREADY + j], kGatherWarps);
+      mbar_init(&bars[B_VFREE + j], 1);
     }
-    __syncthreads();  // sIdx ready; previous sub-tile fully consumed
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars[B_SFULL + u], 1);
+      mbar_init(&bars[B_SFREE + u], kSoftWarps);
+    }
+    mbar_init(&bars[B_PREADY], kSoftWarps);
+    mbar_init(&bars[B_PFREE], 1);
+    mbar_init(&bars[B_QREADY], kSoftWarps);
+    mbar_init(&bars[B_DONE], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
 
-    // ---- gather + dequantize: warp -> 8 entries, lane -> (entry, quarter) ----
-    {
-      const int e = 8 * warp + (lane & 7);
-      const int qd = lane >> 3;
-      const int32_t pos = sIdx[e];
+  if (warp >= kSoftWarps && warp < kMmaWarp) {
+    // ------------------------------ gather + dequantize ------------------------------
+    const int e = tid - kSoftThreads;  // tile row of this thread
+    const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
+    const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
+    for (int t = 0; t < n_tiles && !*s_abort; ++t) {
+      const int je = e_begin + t * kTile + e;
+      int32_t pos = je < e_end ? idx[je] : -1;
+      if (pos < 0 || pos >= len) pos = -1;
+      uint4 pk[16];
+      uint4 sc0 = make_uint4(0, 0, 0, 0), sc1 = sc0;
       if (pos >= 0) {
         const uint8_t* prow = packed_b + int64_t(pos) * (kD / 2);
         const uint8_t* srow = scales_b + int64_t(pos) * (kD / kGroup);
-        uint4 pk[4];
-        uint16_t sp[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int pc = qd + 4 * j;
-          pk[j] = ld_nc_v4(prow + 16 * pc);
-          sp[j] = __ldg(reinterpret_cast<const unsigned short*>(srow + 2 * pc));
+        for (int i = 0; i < 16; ++i) pk[i] = ld_nc_v4(prow + 16 * i);
+        sc0 = ld_nc_v4(srow);
+        sc1 = ld_nc_v4(srow + 16);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = make_uint4(0, 0, 0, 0);
+      }
+      const uint32_t scw[8] = {sc0.x, sc0.y, sc0.z, sc0.w, sc1.x, sc1.y, sc1.z, sc1.w};
+      bool ok = true;  // (no break inside this fully unrolled loop: registers stay registers)
+#pragma unroll
+      for (int jc = 0; jc < kChunks; ++jc) {
+        if (ok && !mbar_wait_timed(&bars[B_VFREE + jc], (t & 1) ^ 1)) {
+          fail_wait(p, s_abort);
+          ok = false;
         }
+        if (!ok) continue;
+        uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + e * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int pc = qd + 4 * j;
-          const uint32_t s_lo = e4m3x2_to_f16x2(uint16_t((sp[j] & 0xffu) * 0x101u));
-          const uint32_t s_hi = e4m3x2_to_f16x2(uint16_t((sp[j] >> 8) * 0x101u));
-          const uint32_t wd[4] = {pk[j].x, pk[j].y, pk[j].z, pk[j].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t s2 = i < 2 ? s_lo : s_hi;
-            uint4 v;
-            v.x = hmul2_f16(e2m1x2_to_f16x2(wd[i] & 0xffu), s2);
-            v.y = hmul2_f16(e2m1x2_to_f16x2((wd[i] >> 8) & 0xffu), s2);
-            v.z = hmul2_f16(e2m1x2_to_f16x2((wd[i] >> 16) & 0xffu), s2);
-            v.w = hmul2_f16(e2m1x2_to_f16x2(wd[i] >> 24), s2);
-            *reinterpret_cast<uint4*>(sV + off_wide(e, 4 * pc + i)) = v;
+        for (int g = 0; g < 4; ++g) {  // 16 dims per scale group
+          const uint32_t sb = (scw[jc] >> (8 * g)) & 0xffu;
+          const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint16_t>(sb * 0x101u));
+          const uint4 src = pk[2 * jc + (g >> 1)];
+          const uint32_t w0 = (g & 1) ? src.z : src.x;
+          const uint32_t w1 = (g & 1) ? src.w : src.y;
+          uint4 o0, o1;
+          o0.x = hmul2_f16(e2m1x2_to_f16x2(w0 & 0xffu), s2);
+          o0.y = hmul2_f16(e2m1x2_to_f16x2((w0 >> 8) & 0xffu), s2);
+          o0.z = hmul2_f16(e2m1x2_to_f16x2((w0 >> 16) & 0xffu), s2);
+          o0.w = hmul2_f16(e2m1x2_to_f16x2(w0 >> 24), s2);
+          o1.x = hmul2_f16(e2m1x2_to_f16x2(w1 & 0xffu), s2);
+          o1.y = hmul2_f16(e2m1x2_to_f16x2((w1 >> 8) & 0xffu), s2);
+          o1.z = hmul2_f16(e2m1x2_to_f16x2((w1 >> 16) & 0xffu), s2);
+          o1.w = hmul2_f16(e2m1x2_to_f16x2(w1 >> 24), s2);
+          *reinterpret_cast<uint4*>(vrow + (((2 * g) ^ (e & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(vrow + (((2 * g + 1) ^ (e & 7)) << 4)) = o1;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_VREADY + jc]);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = umma_idesc(0u, 128, kHeadsPerCta, 0u, 0u);
+      constexpr uint32_t kIdescPV = umma_idesc(0u, 128, kHeadsPerCta, 1u, 1u);
+      const uint32_t q0 = smem_u32(smem + kOffQ), v0 = smem_u32(smem + kOffV);
+      const uint32_t ph0 = smem_u32(smem + kOffPh), pl0 = smem_u32(smem + kOffPl);
+      bool ok = mbar_wait_timed(&bars[B_QREADY], 0);
+      if (!ok) fail_wait(p, s_abort);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        if (*s_abort) break;
+        const int u = t & 1;
+        if (!mbar_wait_timed(&bars[B_SFREE + u], ((t >> 1) & 1) ^ 1)) {
+          fail_wait(p, s_abort);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ds = tmem + kColS + 64u * u;
+        for (int jc = 0; jc < kChunks && ok; ++jc) {
+          if (!mbar_wait_timed(&bars[B_VREADY + jc], t & 1)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_f16(ds, sw128_kmajor_desc(v0 + jc * kVChunkBytes + 32 * k),
+                     sw128_kmajor_desc(q0 + jc * kQChunkBytes + 32 * k), kIdescQK, (jc | k) != 0);
         }
+        if (!ok) {
+          fail_wait(p, s_abort);
+          break;
+        }
+        umma_commit(&bars[B_SFULL + u]);
+        if (!mbar_wait_timed(&bars[B_PREADY], t & 1)) {
+          fail_wait(p, s_abort);
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t d = tmem + 64u * c;
+#pragma unroll
+          for (int s = 0; s < kTile / 16; ++s) {
+            const uint64_t a = sw128_mnmajor_desc(v0 + 2 * c * kVChunkBytes + 2048 * s, kVChunkBytes);
+            umma_f16(d, a, sw128_mnmajor_desc(ph0 + 2048 * s, kPBytes), kIdescPV, t > 0 || s > 0);
+            umma_f16(d, a, sw128_mnmajor_desc(pl0 + 2048 * s, kPBytes), kIdescPV, true);
+          }
+          umma_commit(&bars[B_VFREE + 2 * c]);
+          umma_commit(&bars[B_VFREE + 2 * c + 1]);
+        }
+        umma_commit(&bars[B_PFREE]);
+      }
+      // every MMA issued above completes before TMEM is released
+      umma_commit(&bars[B_DONE]);
+      if (!mbar_wait_timed(&bars[B_DONE], 0)) fail_wait(p, s_abort);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------- Q conversion, softmax and output (warps 0-7) ----------------------
+    // Q: bf16 -> fp16 with a per-head power-of-two scale; K-major 128B-swizzled chunks. Each
+    // warp converts heads warp, warp + 8, ...; its eight rows are loaded before any is
+    // converted so that the global loads overlap.
+    {
+      uint4 qv[kHeadsPerCta / kSoftWarps][2];
+#pragma unroll
+      for (int r = 0; r < kHeadsPerCta / kSoftWarps; ++r) {
+        const int hh = warp + kSoftWarps * r;
+        qv[r][0] = qv[r][1] = make_uint4(0, 0, 0, 0);
+        if (hh < nh) {
+          const uint16_t* qr = p.q + (int64_t(b) * p.H + hbase + hh) * kD + 16 * lane;
+          qv[r][0] = *reinterpret_cast<const uint4*>(qr);
+          qv[r][1] = *reinterpret_cast<const uint4*>(qr + 8);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kHeadsPerCta / kSoftWarps; ++r) {
+        const int hh = warp + kSoftWarps * r;
+        const uint32_t wd[8] = {qv[r][0].x, qv[r][0].y, qv[r][0].z, qv[r][0].w,
+                                qv[r][1].x, qv[r][1].y, qv[r][1].z, qv[r][1].w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = max(m, max(wd[i] & 0x7fffu, (wd[i] >> 16) & 0x7fffu));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        int k = 0;
+        if (m != 0) {
+          const int ex = int((m >> 7) & 0xff) - 127;  // exponent of max|q|
+          k = 14 - (ex < -126 ? -126 : ex);
+          if (k > 127) k = 127;
+          if (k < -126) k = -126;
+        }
+        const float up = __uint_as_float(uint32_t(127 + k) << 23);
+        uint32_t h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          h[i] = pack_f16x2(bf16_bits_to_f32(wd[i] & 0xffffu) * up, bf16_bits_to_f32(wd[i] >> 16) * up);
+        const float c = hh < nh ? p.sm_scale * kLog2e * __uint_as_float(uint32_t(127 - k / 2) << 23) *
+                                      __uint_as_float(uint32_t(127 - (k - k / 2)) << 23)
+                                : 0.0f;
+        // dims [16 lane, 16 lane + 16): chunk lane / 4, 16-byte units 2 (lane % 4) and +1
+        uint8_t* qrow = smem + kOffQ + (lane >> 2) * kQChunkBytes + hh * 128;
+        const int u0 = 2 * (lane & 3);
+        *reinterpret_cast<uint4*>(qrow + ((u0 ^ (hh & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(qrow + (((u0 + 1) ^ (hh & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+        if (lane == 0) {
+          sC[hh] = c;
+          sM[hh] = -INFINITY;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_QREADY]);
+      softmax_sync();  // sC / sM of every head are visible to all softmax warps
+    }
+
+    const int q4 = warp & 3;          // TMEM lane quarter
+    const int h0 = 32 * (warp >> 2);  // first of this thread's 32 heads
+    const int e = 32 * q4 + lane;     // tile row (entry) / output dim within a dim tile
+    const uint32_t lane_addr = uint32_t(32 * q4) << 16;
+    float lsum[32];  // per-head running row sums over this thread's entries
+#pragma unroll
+    for (int j = 0; j < 32; ++j) lsum[j] = 0.0f;
+    bool fail = false;  // uniform across the softmax warps
+    for (int t = 0; t < n_tiles; ++t) {
+      const int u = t & 1;
+      const int je = e_begin + t * kTile + e;
+      const int32_t pos = je < e_end ? idx[je] : -1;
+      const bool valid = pos >= 0 && pos < len;
+      bool f = !mbar_wait_timed(&bars[B_SFULL + u], (t >> 1) & 1);
+      f = __any_sync(0xffffffffu, f);
+      float z[32];
+      bool over = false;
+      if (!f) {
+        tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + kColS + 64u * u + h0, r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_SFREE + u]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          z[j] = valid ? __uint_as_float(r[j]) * sC[h0 + j] : -INFINITY;
+          over |= z[j] > sM[h0 + j] + kMoveLog2;
+        }
+        // the previous tile's P.V must be complete before P is rewritten or O rescaled
+        // (it precedes this tile's S in the tensor pipe, so this wait is normally free)
+        f = !mbar_wait_timed(&bars[B_PFREE], (t & 1) ^ 1);
+        f = __any_sync(0xffffffffu, f);
       } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4*>(sV + off_wide(e, 4 * (qd + 4 * j) + i)) = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 32; ++j) z[j] = -INFINITY;
       }
-    }
-    __syncthreads();
-
-    // ---- S = Q V^T for (m-tile mt, entries [8*kNtS*wi, +8*kNtS)) ----
-    float acc[kNtS][4];
+      if (softmax_any(over || f)) {
+        if (softmax_any(f)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        // move the reference of every head with a logit above m + 2^9
+        const float tmax = butterfly32<true>(z);  // lane l: head h0 + l over this warp's rows
+        sRed[q4 * 64 + h0 + lane] = tmax;
+        softmax_sync();
+        if (q4 == 0) {
+          const int h = h0 + lane;
+          const float tm = fmaxf(fmaxf(sRed[h], sRed[64 + h]), fmaxf(sRed[128 + h], sRed[192 + h]));
+          const float mo = sM[h];
+          float mn = mo, a = 1.0f;
+          if (tm > mo + kMoveLog2) {
+            mn = tm + kHeadroomLog2;
+            a = mo == -INFINITY ? 0.0f : exp2f(mo - mn);
+          }
+          sM[h] = mn;
+          sA[h] = a;
+        }
+        softmax_sync();
+        bool moved = false;
 #pragma unroll
-    for (int j = 0; j < kNtS; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-    const uint32_t sQ_base = smem_u32(sQ), sV_base = smem_u32(sV);
-    const int arow = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
-#pragma unroll 4
-    for (int ks = 0; ks < kD / 16; ++ks) {
-      uint32_t a[4];
-      ldmatrix_x4(a, sQ_base + off_wide(arow, 2 * ks + (lane >> 4)));
-      if constexpr (kNtS == 1) {
-        uint32_t b0, b1;
-        const int ent = 8 * wi + (lane & 7);
-        ldmatrix_x2(b0, b1, sV_base + off_wide(ent, 2 * ks + ((lane >> 3) & 1)));
-        mma_f16_16816(acc[0], a, b0, b1);
-      } else {
+        for (int j = 0; j < 32; ++j) {
+          const float a = sA[h0 + j];
+          lsum[j] *= a;
+          moved |= a != 1.0f;
+        }
+        if (t > 0 && moved) {  // rescale this thread's O^T elements of the moved heads
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r[16];
+            const int j0 = 16 * (c & 1);
+            const uint32_t addr = tmem + lane_addr + 64u * (c >> 1) + h0 + j0;
+            tmem_ld16(addr, r);
+            tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < kNtS; jj += 2) {
-          uint32_t bb[4];
-          const int ent = 8 * (wi * kNtS + jj + (lane >> 4)) + (lane & 7);
-          ldmatrix_x4(bb, sV_base + off_wide(ent, 2 * ks + ((lane >> 3) & 1)));
-          mma_f16_16816(acc[jj], a, bb[0], bb[1]);
-          mma_f16_16816(acc[jj + 1], a, bb[2], bb[3]);
+            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * sA[h0 + j0 + j]);
+            tmem_st16(addr, r);
+          }
+          tmem_st_wait();
         }
       }
-    }
-
-    // ---- online softmax (log2 domain) ----
-    const float cg = sC[16 * mt + g], cg8 = sC[16 * mt + g + 8];
-    float mx = -INFINITY, mx8 = -INFINITY;
+      // probabilities (< 2^9), row sums, and this thread's half of the entry's row of P^T
+      uint8_t* prow_h = smem + kOffPh + e * 128;
+      uint8_t* prow_l = smem + kOffPl + e * 128;
 #pragma unroll
-    for (int jj = 0; jj < kNtS; ++jj) {
-      const int e0 = 8 * (wi * kNtS + jj) + 2 * tq;
-      const bool v0 = sIdx[e0] >= 0, v1 = sIdx[e0 + 1] >= 0;
-      acc[jj][0] = v0 ? acc[jj][0] * cg : -INFINITY;
-      acc[jj][1] = v1 ? acc[jj][1] * cg : -INFINITY;
-      acc[jj][2] = v0 ? acc[jj][2] * cg8 : -INFINITY;
-      acc[jj][3] = v1 ? acc[jj][3] * cg8 : -INFINITY;
-      mx = fmaxf(mx, fmaxf(acc[jj][0], acc[jj][1]));
-      mx8 = fmaxf(mx8, fmaxf(acc[jj][2], acc[jj][3]));
-    }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    mx8 = fmaxf(mx8, __shfl_xor_sync(0xffffffffu, mx8, 1));
-    mx8 = fmaxf(mx8, __shfl_xor_sync(0xffffffffu, mx8, 2));
-    if (tq == 0) {
-      sRed[warp * 16 + g] = mx;
-      sRed[warp * 16 + g + 8] = mx8;
-    }
-    __syncthreads();
-    float tmax = -INFINITY, tmax8 = -INFINITY;
+      for (int unit = 0; unit < 4; ++unit) {
+        uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int k = 0; k < kWarpsPerMt; ++k) {
-      tmax = fmaxf(tmax, sRed[(k * MT + mt) * 16 + g]);
-      tmax8 = fmaxf(tmax8, sRed[(k * MT + mt) * 16 + g + 8]);
-    }
-    const float mn = fmaxf(m_g, tmax), mn8 = fmaxf(m_g8, tmax8);
-    const float al = mn == -INFINITY ? 1.0f : exp2f(m_g - mn);
-    const float al8 = mn8 == -INFINITY ? 1.0f : exp2f(m_g8 - mn8);
-    m_g = mn;
-    m_g8 = mn8;
-    float ps = 0.0f, ps8 = 0.0f;
-#pragma unroll
-    for (int jj = 0; jj < kNtS; ++jj) {
-      const float p0 = mn == -INFINITY ? 0.0f : exp2f(acc[jj][0] - mn);
-      const float p1 = mn == -INFINITY ? 0.0f : exp2f(acc[jj][1] - mn);
-      const float p2 = mn8 == -INFINITY ? 0.0f : exp2f(acc[jj][2] - mn8);
-      const float p3 = mn8 == -INFINITY ? 0.0f : exp2f(acc[jj][3] - mn8);
-      ps += p0 + p1;
-      ps8 += p2 + p3;
-      const int e0 = 8 * (wi * kNtS + jj) + 2 * tq;
-      const float s0 = p0 * kPScale, s1 = p1 * kPScale, s2 = p2 * kPScale, s3 = p3 * kPScale;
-      const uint32_t h01 = pack_f16x2(s0, s1), h23 = pack_f16x2(s2, s3);
-      const uint32_t l01 = pack_f16x2(s0 - f16_lo_to_f32(h01), s1 - f16_hi_to_f32(h01));
-      const uint32_t l23 = pack_f16x2(s2 - f16_lo_to_f32(h23), s3 - f16_hi_to_f32(h23));
-      const int r0 = 16 * mt + g, r8 = r0 + 8, cc = e0 >> 3, within = (e0 & 7) * 2;
-      *reinterpret_cast<uint32_t*>(sPh + off_narrow(r0, cc) + within) = h01;
-      *reinterpret_cast<uint32_t*>(sPh + off_narrow(r8, cc) + within) = h23;
-      *reinterpret_cast<uint32_t*>(sPl + off_narrow(r0, cc) + within) = l01;
-      *reinterpret_cast<uint32_t*>(sPl + off_narrow(r8, cc) + within) = l23;
-    }
-    l_g = l_g * al + ps;
-    l_g8 = l_g8 * al8 + ps8;
-#pragma unroll
-    for (int i = 0; i < kNtO; ++i) {
-      o[i][0] *= al;
-      o[i][1] *= al;
-      o[i][2] *= al8;
-      o[i][3] *= al8;
-    }
-    __syncthreads();  // P complete
-
-    // ---- O += P V for (m-tile mt, dims [dim0, dim0 + 8*kNtO)) ----
-    const uint32_t sPh_base = smem_u32(sPh), sPl_base = smem_u32(sPl);
-#pragma unroll
-    for (int ks = 0; ks < kSub / 16; ++ks) {
-      uint32_t ah[4], alo[4];
-      ldmatrix_x4(ah, sPh_base + off_narrow(arow, 2 * ks + (lane >> 4)));
-      ldmatrix_x4(alo, sPl_base + off_narrow(arow, 2 * ks + (lane >> 4)));
-      const int ent = 16 * ks + 8 * ((lane >> 3) & 1) + (lane & 7);
-#pragma unroll
-      for (int np = 0; np < kNtO / 2; ++np) {
-        uint32_t bb[4];
-        ldmatrix_x4_trans(bb, sV_base + off_wide(ent, (dim0 >> 3) + 2 * np + (lane >> 4)));
-        mma_f16_16816(o[2 * np], ah, bb[0], bb[1]);
-        mma_f16_16816(o[2 * np], alo, bb[0], bb[1]);
-        mma_f16_16816(o[2 * np + 1], ah, bb[2], bb[3]);
-        mma_f16_16816(o[2 * np + 1], alo, bb[2], bb[3]);
+        for (int k = 0; k < 4; ++k) {
+          const int j = 8 * unit + 2 * k;
+          const float m0 = sM[h0 + j], m1 = sM[h0 + j + 1];
+          const float p0 = m0 == -INFINITY ? 0.0f : exp2f(z[j] - m0);
+          const float p1 = m1 == -INFINITY ? 0.0f : exp2f(z[j + 1] - m1);
+          lsum[j] += p0;
+          lsum[j + 1] += p1;
+          const float a = p0 * kPScale, c2 = p1 * kPScale;
+          hi[k] = pack_f16x2(a, c2);
+          lo[k] = pack_f16x2(a - f16_lo_to_f32(hi[k]), c2 - f16_hi_to_f32(hi[k]));
+        }
+        const uint32_t off = uint32_t((((h0 >> 3) + unit) ^ (e & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow_h + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(prow_l + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_PREADY]);
+    }
+    // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----
+    if (!fail && n_tiles > 0) {
+      bool f = !mbar_wait_timed(&bars[B_PFREE], (n_tiles - 1) & 1);
+      f = __any_sync(0xffffffffu, f);
+      fail = softmax_any(f);
+    }
+    if (fail) {
+      if (tid == 0) fail_wait(p, s_abort);
+    } else {
+      tc_fence_after();
+      const float lw = butterfly32<false>(lsum);  // lane l: head h0 + l over this warp's rows
+      sRed[q4 * 64 + h0 + lane] = lw;
+      softmax_sync();
+      if (q4 == 0) {
+        const int h = h0 + lane;
+        sL[h] = sRed[h] + sRed[64 + h] + sRed[128 + h] + sRed[192 + h];
+      }
+      softmax_sync();
+      const bool split = n_chunks > 1;
+      float f_out[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float L = sL[h0 + j];
+        f_out[j] = L > 0.0f ? (split ? 1.0f : 1.0f / (kPScale * L)) : 0.0f;
+      }
+      float* stage = reinterpret_cast<float*>(smem + kOffV);  // [64 heads][512 dims]
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stage[(h0 + j) * kD + 128 * c + e] = __uint_as_float(r[j]) * f_out[j];
+      }
+      fence_proxy_async_smem();
+      softmax_sync();
+      const int64_t part = (int64_t(b) * n_hg + hg) * n_chunks + chunk;
+      float* dst = split ? p.part_o + part * kHeadsPerCta * kD : p.out + (int64_t(b) * p.H + hbase) * kD;
+      const uint32_t bytes = uint32_t(split ? kHeadsPerCta : nh) * kD * 4u;
+      if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+        if (tid == 0) {
+          bulk_s2g(dst, stage, bytes);
+          bulk_commit();
+        }
+      } else {  // the output is only 8-byte aligned: copy with the softmax threads
+        const float2* s2 = reinterpret_cast<const float2*>(stage);
+        float2* d2 = reinterpret_cast<float2*>(dst);
+        for (uint32_t i = tid; i < bytes / 8; i += kSoftThreads) d2[i] = s2[i];
+      }
+      if (q4 == 0) {
+        const int h = h0 + lane;
+        const float L = sL[h];
+        if (split) {
+          p.part_ml[(part * kHeadsPerCta + h) * 2] = sM[h];
+          p.part_ml[(part * kHeadsPerCta + h) * 2 + 1] = L;
+        } else if (p.lse != nullptr && h < nh) {
+          p.lse[int64_t(b) * p.H + hbase + h] = L > 0.0f ? sM[h] * kLn2 + logf(L) : -INFINITY;
+        }
+      }
+      if (tid == 0) bulk_wait_read_all();  // the staging buffer stays valid until read
     }
   }
 
-  // ---- per-head sums across the warps of an m-tile ----
-  l_g += __shfl_xor_sync(0xffffffffu, l_g, 1);
-  l_g += __shfl_xor_sync(0xffffffffu, l_g, 2);
-  l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, 1);
-  l_g8 += __shfl_xor_sync(0xffffffffu, l_g8, 2);
+  tc_fence_before();
   __syncthreads();
-  if (tq == 0) {
-    sRed[warp * 16 + g] = l_g;
-    sRed[warp * 16 + g + 8] = l_g8;
-  }
-  __syncthreads();
-  float L = 0.0f, L8 = 0.0f;
-#pragma unroll
-  for (int k = 0; k < kWarpsPerMt; ++k) {
-    L += sRed[(k * MT + mt) * 16 + g];
-    L8 += sRed[(k * MT + mt) * 16 + g + 8];
-  }
-  const int h0 = 16 * mt + g, h8 = h0 + 8;
-
-  if (n_chunks == 1) {
-    const float inv = L > 0.0f ? 1.0f / (kPScale * L) : 0.0f;
-    const float inv8 = L8 > 0.0f ? 1.0f / (kPScale * L8) : 0.0f;
-#pragma unroll
-    for (int i = 0; i < kNtO; ++i) {
-      const int dim = dim0 + 8 * i + 2 * tq;
-      if (h0 < nh)
-        *reinterpret_cast<float2*>(p.out + (int64_t(b) * p.H + hbase + h0) * kD + dim) =
-            make_float2(o[i][0] * inv, o[i][1] * inv);
-      if (h8 < nh)
-        *reinterpret_cast<float2*>(p.out + (int64_t(b) * p.H + hbase + h8) * kD + dim) =
-            make_float2(o[i][2] * inv8, o[i][3] * inv8);
-    }
-    if (p.lse != nullptr && wi == 0 && tq == 0) {
-      if (h0 < nh) p.lse[int64_t(b) * p.H + hbase + h0] = L > 0.0f ? m_g * kLn2 + logf(L) : -INFINITY;
-      if (h8 < nh) p.lse[int64_t(b) * p.H + hbase + h8] = L8 > 0.0f ? m_g8 * kLn2 + logf(L8) : -INFINITY;
-    }
-    return;
-  }
-
-  // ---- split: write this chunk's unnormalised partial; k_attn_combine merges them ----
-  const int64_t part = (int64_t(b) * n_hg + hg) * n_chunks + chunk;
-  float* po = p.part_o + part * kHeadsPerCta * kD;
-  float* pml = p.part_ml + part * kHeadsPerCta * 2;
-#pragma unroll
-  for (int i = 0; i < kNtO; ++i) {
-    const int dim = dim0 + 8 * i + 2 * tq;
-    *reinterpret_cast<float2*>(po + h0 * kD + dim) = make_float2(o[i][0], o[i][1]);
-    *reinterpret_cast<float2*>(po + h8 * kD + dim) = make_float2(o[i][2], o[i][3]);
-  }
-  if (wi == 0 && tq == 0) {
-    pml[2 * h0] = m_g;
-    pml[2 * h0 + 1] = L;
-    pml[2 * h8] = m_g8;
-    pml[2 * h8 + 1] = L8;
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
-// Merge of the chunk partials (log-sum-exp combine): grid (8 head blocks, head groups, B),
-// one warp per head, each lane 16 of the 512 dims.
-__global__ void __launch_bounds__(256) k_attn_combine(const AttnParams p, int n_hg) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hg = blockIdx.y, b = blockIdx.z;
-  const int hh = blockIdx.x * 8 + warp;
+// Merge of the chunk partials (log-sum-exp combine). Grid (64 heads, head groups, B), 128
+// threads: the chunk weights 2^(m_c - M) are computed once into shared memory, then every
+// thread accumulates 4 of the 512 dims over the chunks, four chunks' loads in flight at once.
+constexpr int kMaxChunks = 256;
+__global__ void __launch_bounds__(128) k_attn_combine(const AttnParams p, int n_hg) {
+  __shared__ float s_w[kMaxChunks];
+  __shared__ float s_red[2][4];
+  griddep_wait();  // the attention grid's partials are complete and visible
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hh = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
   const int nh = min(kHeadsPerCta, p.H - hg * kHeadsPerCta);
   if (hh >= nh) return;
   const int n_chunks = p.n_chunks;
-  const float* pml0 = p.part_ml + (int64_t(b) * n_hg + hg) * n_chunks * kHeadsPerCta * 2;
-  const float* po0 = p.part_o + (int64_t(b) * n_hg + hg) * n_chunks * kHeadsPerCta * kD;
-  float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pml0[(int64_t(c) * kHeadsPerCta + hh) * 2]);
-  float Lt = 0.0f;
-  float4 acc[4];
+  const int64_t base = (int64_t(b) * n_hg + hg) * n_chunks;
+  float mloc = -INFINITY;
+  for (int c = tid; c < n_chunks; c += 128) {
+    const float mc = p.part_ml[((base + c) * kHeadsPerCta + hh) * 2];
+    const float lc = p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1];
+    s_w[c] = lc > 0.0f ? mc : -INFINITY;
+    if (lc > 0.0f) mloc = fmaxf(mloc, mc);
+  }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < n_chunks; ++c) {
-    const float mc = pml0[(int64_t(c) * kHeadsPerCta + hh) * 2];
-    const float lc = pml0[(int64_t(c) * kHeadsPerCta + hh) * 2 + 1];
-    if (!(lc > 0.0f)) continue;
-    const float wgt = exp2f(mc - M);
-    Lt += lc * wgt;
-    const float4* src = reinterpret_cast<const float4*>(po0 + (int64_t(c) * kHeadsPerCta + hh) * kD) + 4 * lane;
+  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if (lane == 0) s_red[0][warp] = mloc;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
+  float lsum = 0.0f;
+  for (int c = tid; c < n_chunks; c += 128) {
+    const float mc = s_w[c];
+    const float w = mc == -INFINITY ? 0.0f : exp2f(mc - M);
+    s_w[c] = w;
+    lsum += w * p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  if (lane == 0) s_red[1][warp] = lsum;
+  __syncthreads();
+  const float Lt = s_red[1][0] + s_red[1][1] + s_red[1][2] + s_red[1][3];
+  const float4* src = reinterpret_cast<const float4*>(p.part_o + (base * kHeadsPerCta + hh) * kD) + tid;
+  const int64_t cstride = int64_t(kHeadsPerCta) * kD / 4;  // float4s between chunks
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int c = 0;
+  for (; c + 4 <= n_chunks; c += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = src[(c + u) * cstride];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float4 v = src[u];
-      acc[u].x += wgt * v.x; acc[u].y += wgt * v.y; acc[u].z += wgt * v.z; acc[u].w += wgt * v.w;
+      const float w = s_w[c + u];
+      acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
     }
   }
+  for (; c < n_chunks; ++c) {
+    const float4 v = src[c * cstride];
+    const float w = s_w[c];
+    acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+  }
   const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
-  float4* dst = reinterpret_cast<float4*>(p.out + (int64_t(b) * p.H + hg * kHeadsPerCta + hh) * kD) + 4 * lane;
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    dst[u] = make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
-  if (p.lse != nullptr && lane == 0)
+  float4* dst = reinterpret_cast<float4*>(p.out + (int64_t(b) * p.H + hg * kHeadsPerCta + hh) * kD) + tid;
+  *dst = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (p.lse != nullptr && tid == 0)
     p.lse[int64_t(b) * p.H + hg * kHeadsPerCta + hh] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
-}
-
-template <int MT>
-cudaError_t launch_mt(const AttnParams& p, int n_hg, cudaStream_t stream) {
-  auto kern = k_sparse_attn<MT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemAttn));
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.n_chunks, n_hg, p.B);
-  kern<<<grid, kAttnThreads, kSmemAttn, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_chunks == 1) return e;
-  k_attn_combine<<<dim3(kHeadsPerCta / 8, n_hg, p.B), 256, 0, stream>>>(p, n_hg);
-  return cudaGetLastError();
 }
 
 }  // namespace
@@ -408,8 +627,9 @@ cudaError_t launch_mt(const AttnParams& p, int n_hg, cudaStream_t stream) {
 int attn_chunks(int B, int H, int top_k, int num_sms) {
   const int n_hg = (H + kHeadsPerCta - 1) / kHeadsPerCta;
   int c = num_sms / (B * n_hg);
-  const int max_c = top_k / 128;
+  const int max_c = top_k / kTile;
   if (c > max_c) c = max_c;
+  if (c > kMaxChunks) c = kMaxChunks;
   if (c < 1) c = 1;
   return c;
 }
@@ -418,10 +638,28 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t st
   (void)num_sms;
   if (p.B == 0) return cudaSuccess;
   const int n_hg = (p.H + kHeadsPerCta - 1) / kHeadsPerCta;
-  const int heads = p.H < kHeadsPerCta ? p.H : kHeadsPerCta;
-  if (heads <= 16) return launch_mt<1>(p, n_hg, stream);
-  if (heads <= 32) return launch_mt<2>(p, n_hg, stream);
-  return launch_mt<4>(p, n_hg, stream);
+  cudaError_t e = cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemAttn));
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_chunks, n_hg, p.B);
+  k_sparse_attn_tc<<<grid, kAttnThreads, kSmemAttn, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_chunks == 1) return e;
+  // launched as a programmatic dependent of the attention grid: its CTAs are scheduled while
+  // the attention grid runs and wait in griddep_wait(), which hides the launch gap
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kHeadsPerCta, n_hg, p.B);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_attn_combine, p, n_hg);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 }  // namespace fp4kv
