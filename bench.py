@@ -361,27 +361,37 @@ class QuantWorkload:
 def timed_steps(wl, steps, warmup, flush, sampler, fk):
     """Device time of `steps` steps. When `flush` is given, L2 is flushed (a write larger
     than L2) before each step, outside the timed windows; otherwise every step streams more
-    than twice the L2 capacity, so no step starts with the previous step's data cached."""
+    than twice the L2 capacity, so no step starts with the previous step's data cached.
+
+    The steps are timed bare (CUDA events around each step only), then run once more with
+    the library's per-launch events on for the per-kernel breakdown: events recorded
+    between two launches would keep the second from starting early as a programmatic
+    dependent of the first, so they stay out of the headline timing."""
     s = torch.cuda.current_stream()
     for _ in range(warmup):
         wl.step()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(steps)]
-    fk.profile_read()  # drop warm-up records
+
+    def run(n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            if flush is not None:
+                flush.zero_()
+            a.record(s)
+            wl.step()
+            b.record(s)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
     sampler.start()
+    total_ms = run(steps)
+    fk.profile_read()  # drop earlier records
     fk.profile_enable(True)
-    for a, b in evs:
-        if flush is not None:
-            flush.zero_()
-        a.record(s)
-        wl.step()
-        b.record(s)
-    torch.cuda.synchronize()
+    run(steps)
     fk.profile_enable(False)
     sampler.stop()
     prof = fk.profile_read()
-    total_ms = sum(a.elapsed_time(b) for a, b in evs)
     return total_ms, prof
 
 

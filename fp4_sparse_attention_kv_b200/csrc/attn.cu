@@ -83,6 +83,7 @@ static_assert(kChunks * kVChunkBytes == kHeadsPerCta * kD * 4, "output staging")
 
 // TMEM columns: O^T dim-tile c at [64c, 64c + 64); S^T slot u at [256 + 64u, +64)
 constexpr uint32_t kColS = 256;
+static_assert(4096 / kTile <= 32, "the per-thread validity mask holds one bit per tile");
 
 enum { B_VREADY = 0, B_VFREE = 8, B_SFULL = 16, B_SFREE = 18, B_PREADY = 20, B_PFREE = 21,
        B_QREADY = 22, B_DONE = 23 };
@@ -205,10 +206,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     const int e = tid - kSoftThreads;  // tile row of this thread
     const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
     const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
+    griddep_wait();  // the index list comes from the preceding kernel on the stream
+    int32_t pos_next = e_begin + e < e_end ? idx[e_begin + e] : -1;
     for (int t = 0; t < n_tiles && !*s_abort; ++t) {
-      const int je = e_begin + t * kTile + e;
-      int32_t pos = je < e_end ? idx[je] : -1;
+      int32_t pos = pos_next;
       if (pos < 0 || pos >= len) pos = -1;
+      {  // the next tile's position is fetched one tile ahead
+        const int jn = e_begin + (t + 1) * kTile + e;
+        pos_next = jn < e_end ? idx[jn] : -1;
+      }
       uint4 pk[16];
       uint4 sc0 = make_uint4(0, 0, 0, 0), sc1 = sc0;
       if (pos >= 0) {
@@ -376,15 +382,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     const int h0 = 32 * (warp >> 2);  // first of this thread's 32 heads
     const int e = 32 * q4 + lane;     // tile row (entry) / output dim within a dim tile
     const uint32_t lane_addr = uint32_t(32 * q4) << 16;
+    // bit t: this thread's entry of tile t holds a valid position (at most 32 tiles)
+    griddep_wait();  // the index list comes from the preceding kernel on the stream
+    uint32_t vmask = 0;
+    for (int t0 = 0; t0 < n_tiles; t0 += 8) {
+      int32_t pv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int je = e_begin + (t0 + k) * kTile + e;
+        pv[k] = t0 + k < n_tiles && je < e_end ? idx[je] : -1;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (pv[k] >= 0 && pv[k] < len) vmask |= 1u << (t0 + k);
+    }
     float lsum[32];  // per-head running row sums over this thread's entries
 #pragma unroll
     for (int j = 0; j < 32; ++j) lsum[j] = 0.0f;
     bool fail = false;  // uniform across the softmax warps
     for (int t = 0; t < n_tiles; ++t) {
       const int u = t & 1;
-      const int je = e_begin + t * kTile + e;
-      const int32_t pos = je < e_end ? idx[je] : -1;
-      const bool valid = pos >= 0 && pos < len;
+      const bool valid = (vmask >> t) & 1u;
       bool f = !mbar_wait_timed(&bars[B_SFULL + u], (t >> 1) & 1);
       f = __any_sync(0xffffffffu, f);
       float z[32];
@@ -501,25 +519,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       }
       softmax_sync();
       const bool split = n_chunks > 1;
-      float f_out[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float L = sL[h0 + j];
-        f_out[j] = L > 0.0f ? (split ? 1.0f : 1.0f / (kPScale * L)) : 0.0f;
+      if (q4 == 0) {  // per-head factor: 1 for a partial, 1 / (2^6 L) for a final row, 0 if empty
+        const int h = h0 + lane;
+        const float L = sL[h];
+        sA[h] = L > 0.0f ? (split ? 1.0f : 1.0f / (kPScale * L)) : 0.0f;
       }
-      float* stage = reinterpret_cast<float*>(smem + kOffV);  // [64 heads][512 dims]
+      softmax_sync();
+      // O^T -> staging [64 heads][512 dims] fp32 in the V_hat region (rolled: runs once per CTA)
+      float* stage = reinterpret_cast<float*>(smem + kOffV);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
+      for (int cj = 0; cj < 16; ++cj) {
+        const int c = cj >> 2, j0 = h0 + 8 * (cj & 3);
+        uint32_t r[8];
         if (n_tiles > 0) {
-          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
+          tmem_ld8(tmem + lane_addr + 64u * c + j0, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = 0u;
+          for (int k = 0; k < 8; ++k) r[k] = 0u;
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) stage[(h0 + j) * kD + 128 * c + e] = __uint_as_float(r[j]) * f_out[j];
+        for (int k = 0; k < 8; ++k) stage[(j0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[j0 + k];
       }
       fence_proxy_async_smem();
       softmax_sync();
@@ -641,22 +661,26 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t st
   cudaError_t e = cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAttn));
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_chunks, n_hg, p.B);
-  k_sparse_attn_tc<<<grid, kAttnThreads, kSmemAttn, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_chunks == 1) return e;
-  // launched as a programmatic dependent of the attention grid: its CTAs are scheduled while
-  // the attention grid runs and wait in griddep_wait(), which hides the launch gap
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kHeadsPerCta, n_hg, p.B);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
+  // Both kernels are programmatic dependents of the kernel before them on the stream: their
+  // CTAs may be scheduled while that kernel finishes (an SM it has left idle can run the
+  // attention prologue: barriers, TMEM, Q conversion) and wait in griddep_wait() before
+  // reading what it produced. A predecessor that never signals early simply completes first.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_chunks, n_hg, p.B);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = kSmemAttn;
+  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_sparse_attn_tc, p);
+  if (e != cudaSuccess) return e;
+  if (p.n_chunks == 1) return cudaSuccess;
+  cfg.gridDim = dim3(kHeadsPerCta, n_hg, p.B);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, k_attn_combine, p, n_hg);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

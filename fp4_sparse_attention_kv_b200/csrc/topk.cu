@@ -19,6 +19,7 @@
 //     workspace ready for the next call. No CTA ever waits on another.
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
+#include "fp4kv_sm100.cuh"
 
 namespace fp4kv {
 namespace {
@@ -178,21 +179,6 @@ __device__ void block_sort(T* s) {
   __syncthreads();
 }
 
-// Warp-aggregated append of `take` lanes' values into list[counter++]; slots at or beyond
-// `capacity` are never written (the counter still counts them).
-template <typename T>
-FP4KV_DEV void warp_append(bool take, T v, uint32_t* counter, T* list, uint32_t capacity) {
-  const uint32_t m = __ballot_sync(0xffffffffu, take);
-  if (m == 0) return;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(m)));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
-  if (take && slot < capacity) list[slot] = v;
-}
-
 // candidate = (order key << 32) | value index
 FP4KV_DEV uint32_t cand_key(uint64_t c) { return static_cast<uint32_t>(c >> 32); }
 FP4KV_DEV int32_t cand_idx(uint64_t c) { return static_cast<int32_t>(c & 0xffffffffu); }
@@ -261,20 +247,32 @@ __device__ void resolve_candidates(const SelectProblem& P, int b, const uint64_t
   }
 }
 
+// Appends the taken candidates to s_sel at *s_cnt (one shared atomic per warp).
 template <bool kShared>
 __device__ void collect_candidates(const SelectProblem& P, int b, const uint64_t* cand,
                                    uint32_t n_cand, bool take_all, uint32_t ustar,
                                    int64_t pos_star, uint64_t* s_sel, uint32_t* s_cnt) {
-  for (uint32_t c = threadIdx.x; c < n_cand; c += kSelThreads) {
-    const uint64_t cv = load_cand<kShared>(cand, c);
-    const int32_t i = cand_idx(cv);
-    const int64_t pos = position_of(P, b, i);
-    const uint32_t key = cand_key(cv);
-    const bool take = take_all || key > ustar || (key == ustar && pos <= pos_star);
-    if (take) {
-      const uint32_t slot = atomicAdd(s_cnt, 1u);
-      if (slot < kMaxSel) s_sel[slot] = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
+  const int lane = threadIdx.x & 31;
+  for (uint32_t c0 = 0; c0 < n_cand; c0 += kSelThreads) {
+    const uint32_t c = c0 + threadIdx.x;
+    bool take = false;
+    uint64_t item = 0;
+    if (c < n_cand) {
+      const uint64_t cv = load_cand<kShared>(cand, c);
+      const int32_t i = cand_idx(cv);
+      const int64_t pos = position_of(P, b, i);
+      const uint32_t key = cand_key(cv);
+      take = take_all || key > ustar || (key == ustar && pos <= pos_star);
+      item = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
     }
+    const uint32_t m = __ballot_sync(0xffffffffu, take);
+    if (m == 0) continue;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if (lane == leader) base = atomicAdd(s_cnt, static_cast<uint32_t>(__popc(m)));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    const uint32_t slot = base + static_cast<uint32_t>(__popc(m & ((1u << lane) - 1u)));
+    if (take && slot < kMaxSel) s_sel[slot] = item;
   }
 }
 
@@ -295,6 +293,9 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   __shared__ uint32_t s_cnt;
   __shared__ bool s_last;
   const int tid = threadIdx.x;
+  // a kernel launched after this one as a programmatic dependent may start its own
+  // prologue now (it waits for this grid's completion before reading the results)
+  griddep_launch_dependents();
 
   const int64_t n = n_values(P, b);
   const float* vals = P.values + int64_t(b) * P.vstride;
@@ -314,9 +315,14 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   // 2. filter this CTA's slice
   const int64_t lo = n * blockIdx.x / P.slices;
   const int64_t hi = n * (blockIdx.x + 1) / P.slices;
-  // all loads of a batch are issued before any append (whose atomics would otherwise keep
-  // the next load from being hoisted, costing one memory round trip per 512 values)
+  // Each batch of 8 values per thread is classified in registers; one block-wide prefix
+  // sum of the (sure, candidate) counts then gives every thread its output slots, and one
+  // global atomic per list and batch reserves the CTA's range (appends racing on the
+  // per-sequence counters would cost a memory round trip each).
   constexpr int kBatch = 8;
+  __shared__ uint32_t s_wsum[kSelThreads / 32];
+  __shared__ uint32_t s_base[2];
+  const int lane = tid & 31, warp = tid >> 5;
   for (int64_t base = lo; base < hi; base += int64_t(kSelThreads) * kBatch) {
     float v[kBatch];
 #pragma unroll
@@ -324,21 +330,58 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
       const int64_t i = base + int64_t(u) * kSelThreads + tid;
       v[u] = i < hi ? __ldg(vals + i) : -INFINITY;
     }
+    uint32_t smask = 0, cmask = 0, keys[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int64_t i = base + int64_t(u) * kSelThreads + tid;
-      bool is_sure = false, is_cand = false;
-      uint32_t key = 0;
+      keys[u] = 0;
       if (i < hi && (v[u] != -INFINITY || P.mode != 2)) {
-        key = order_key(v[u]);
-        const int digit = static_cast<int>(key >> (32 - kHistBits));
-        is_sure = digit > bstar;
-        is_cand = digit == bstar;
+        keys[u] = order_key(v[u]);
+        const int digit = static_cast<int>(keys[u] >> (32 - kHistBits));
+        if (digit > bstar) smask |= 1u << u;
+        else if (digit == bstar) cmask |= 1u << u;
       }
-      warp_append<int32_t>(is_sure, static_cast<int32_t>(i), &ctr[0], sure, static_cast<uint32_t>(P.k));
-      warp_append<uint64_t>(is_cand, (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(i),
-                            &ctr[1], cand, static_cast<uint32_t>(P.vstride));
     }
+    // counts packed as (sure << 16) | candidates: a batch holds at most 4096 of each
+    const uint32_t cnt = (static_cast<uint32_t>(__popc(smask)) << 16) | static_cast<uint32_t>(__popc(cmask));
+    uint32_t x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t t = lane < kSelThreads / 32 ? s_wsum[lane] : 0u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      if (lane < kSelThreads / 32) s_wsum[lane] = t;  // inclusive prefix over warps
+      if (lane == kSelThreads / 32 - 1) {
+        s_base[0] = (t >> 16) ? atomicAdd(&ctr[0], t >> 16) : 0u;
+        s_base[1] = (t & 0xffffu) ? atomicAdd(&ctr[1], t & 0xffffu) : 0u;
+      }
+    }
+    __syncthreads();
+    const uint32_t excl = x - cnt + (warp > 0 ? s_wsum[warp - 1] : 0u);
+    uint32_t so = s_base[0] + (excl >> 16), co = s_base[1] + (excl & 0xffffu);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t i = base + int64_t(u) * kSelThreads + tid;
+      if ((smask >> u) & 1u) {
+        if (so < static_cast<uint32_t>(P.k)) sure[so] = static_cast<int32_t>(i);
+        ++so;
+      }
+      if ((cmask >> u) & 1u) {
+        if (co < static_cast<uint32_t>(P.vstride))
+          cand[co] = (static_cast<uint64_t>(keys[u]) << 32) | static_cast<uint32_t>(i);
+        ++co;
+      }
+    }
+    __syncthreads();  // s_wsum and s_base are reused by the next batch
   }
 
   // 3. ticket: the last CTA of this sequence finalises
@@ -371,15 +414,14 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
       resolve_candidates<false>(P, b, cand, n_cand, r, bstar, s_hist, s_scan, &ustar, &pos_star);
   }
 
-  // collect the selected (position, value index) pairs
-  if (tid == 0) s_cnt = 0;
-  __syncthreads();
+  // collect the selected (position, value index) pairs: the sure list is compact and all
+  // of it is taken (n_sure <= K <= kMaxSel); taken candidates are appended after it
+  if (tid == 0) s_cnt = n_sure;
   for (uint32_t c = tid; c < n_sure; c += kSelThreads) {
     const int32_t i = __ldcg(sure + c);
-    const uint32_t slot = atomicAdd(&s_cnt, 1u);
-    if (slot < kMaxSel)
-      s_sel[slot] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
+    s_sel[c] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
   }
+  __syncthreads();
   if (r > 0 || take_all) {
     if (in_smem)
       collect_candidates<true>(P, b, s_cand, n_cand, take_all, ustar, pos_star, s_sel, &s_cnt);
@@ -432,7 +474,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
 }  // namespace
 
 int select_slices(int64_t n_values, int B, int num_sms) {
-  int64_t s = (2 * int64_t(num_sms) + B - 1) / B;
+  int64_t s = (2 * int64_t(num_sms)) / B;  // two CTAs per SM: one wave
   const int64_t cap = (n_values + 4095) / 4096;
   if (s > cap) s = cap;
   if (s < 1) s = 1;
