@@ -100,7 +100,7 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Workspace layouts
 // ---------------------------------------------------------------------------------------
 struct IndexerLayout {
-  size_t status = 0, scores = 0, bmax = 0, hist = 0, counters = 0, sure = 0, cand = 0;
+  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist2 = 0, counters = 0, cnt = 0, list = 0;
   size_t total = 0;
   int64_t score_stride = 0, bmax_stride = 0;
   int n_probs = 0;
@@ -112,11 +112,11 @@ struct IndexerLayout {
 IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, int64_t npb) {
   IndexerLayout L;
   size_t off = kAlign;  // status header
-  L.score_stride = (kind == 1) ? npb * 8 : (cap + 3) / 4 * 4;
+  L.score_stride = (kind == 1) ? npb * 8 : (cap + 7) / 8 * 8;
   L.scores = off;
   off += up(sizeof(float) * B * L.score_stride);
   if (kind == 2) {
-    L.bmax_stride = ((cap + 7) / 8 + 3) / 4 * 4;
+    L.bmax_stride = ((cap + 7) / 8 + 7) / 8 * 8;
     L.bmax = off;
     off += up(sizeof(float) * B * L.bmax_stride);
   }
@@ -132,13 +132,16 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
     L.k[1] = npb;
     L.vstride[1] = L.bmax_stride;
   }
+  // hist, hist2 and counters are contiguous: the region that must start at zero
   L.hist = off;
   off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
+  L.hist2 = off;
+  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
   L.counters = off;
-  off += up(sizeof(uint32_t) * L.n_probs * B * 4);
-  L.sure = off;
-  for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(int32_t) * B * L.k[i]);
-  L.cand = off;
+  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kSelCounters);
+  L.cnt = off;
+  off += up(sizeof(uint32_t) * L.n_probs * 2 * B * fp4kv::kMaxSlices);
+  L.list = off;
   for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(uint64_t) * B * L.vstride[i]);
   L.total = off;
   return L;
@@ -328,7 +331,7 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
   if (e != cudaSuccess) return cuda_fail(e, "indexer scoring");
 
   fp4kv::SelectProblem probs[2];
-  size_t sure_off = L.sure, cand_off = L.cand;
+  size_t list_off = L.list;
   for (int i = 0; i < L.n_probs; ++i) {
     fp4kv::SelectProblem& P = probs[i];
     P = fp4kv::SelectProblem{};
@@ -340,11 +343,12 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
     P.npb = n_pool_blocks;
     P.k = static_cast<int>(L.k[i]);
     P.hist = p.hist + int64_t(i) * B * fp4kv::kHistBins;
-    P.counters = reinterpret_cast<uint32_t*>(base + L.counters) + int64_t(i) * B * 4;
-    P.sure = reinterpret_cast<int32_t*>(base + sure_off);
-    P.cand = reinterpret_cast<int32_t*>(base + cand_off);
-    sure_off += up(sizeof(int32_t) * B * L.k[i]);
-    cand_off += up(sizeof(uint64_t) * B * L.vstride[i]);
+    P.hist2 = reinterpret_cast<uint32_t*>(base + L.hist2) + int64_t(i) * B * fp4kv::kHistBins;
+    P.counters = reinterpret_cast<uint32_t*>(base + L.counters) + int64_t(i) * B * fp4kv::kSelCounters;
+    P.cnt1 = reinterpret_cast<uint32_t*>(base + L.cnt) + int64_t(2 * i) * B * fp4kv::kMaxSlices;
+    P.cnt2 = P.cnt1 + int64_t(B) * fp4kv::kMaxSlices;
+    P.list = reinterpret_cast<uint64_t*>(base + list_off);
+    list_off += up(sizeof(uint64_t) * B * L.vstride[i]);
     P.out_idx = (i == 0) ? out_idx : out_pool;
     P.out_score = (i == 0) ? out_score : nullptr;
     const int64_t nvals = (kind == 1) ? int64_t(n_pool_blocks) * 8 : (i == 0 ? cap : (cap + 7) / 8);
@@ -409,9 +413,9 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
   if (top_k < 1 || top_k > 4096) return fail(FP4KV_ERR_UNSUPPORTED, "top_k=%d outside [1, 4096]", top_k);
   if (cap < 1 || cap > (int64_t(1) << 31) - 8)
     return fail(FP4KV_ERR_UNSUPPORTED, "cap=%lld outside [1, 2^31 - 8]", (long long)cap);
-  if (!aligned(q, 16) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(out, 8) ||
+  if (!aligned(q, 16) || !aligned(packed, 16) || !aligned(scales, 16) || !aligned(out, 8) ||
       !aligned(ws, kAlign))
-    return fail(FP4KV_ERR_INVALID_ARG, "misaligned q/packed (16 B), scales (2 B), out (8 B) or ws (256 B)");
+    return fail(FP4KV_ERR_INVALID_ARG, "misaligned q/packed/scales (16 B), out (8 B) or ws (256 B)");
   const int sms = num_sms();
   const AttnLayout L = attn_layout(B, H, top_k, sms);
   if (ws_bytes < L.total) return fail(FP4KV_ERR_WORKSPACE_TOO_SMALL, "ws_bytes %zu < %zu", ws_bytes, L.total);
@@ -511,7 +515,7 @@ fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H
   // the status word and the histogram + counters must start at zero
   cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
   if (e == cudaSuccess)
-    e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.sure - L.hist, s);
+    e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.cnt - L.hist, s);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: clearing scratch");
   return run_indexer(kind, q, w, H_I, keys, key_dtype, key_scale, cap, seq_lens, B, pool,
                      pool ? n_pool_blocks : 0, top_k, out_idx, nullptr, out_score, ws, L.total, s);

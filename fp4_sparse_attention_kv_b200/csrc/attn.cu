@@ -142,6 +142,27 @@ FP4KV_DEV float butterfly32(const float (&v)[32]) {
   return kMax ? fmaxf(keep, r) : keep + r;
 }
 
+// Wait policies (all return the same value in every lane of the warp). The gather warps
+// wait for buffers during the softmax and the MMAs: they poll rarely. The softmax warps
+// wait on the critical path.
+#ifndef ATTN_GATHER_SLEEP_NS
+#define ATTN_GATHER_SLEEP_NS 128
+#endif
+FP4KV_DEV bool gather_wait(uint64_t* bar, uint32_t parity) {
+#if ATTN_GATHER_SLEEP_NS > 0
+  return __all_sync(0xffffffffu, mbar_wait_sleepy(bar, parity, ATTN_GATHER_SLEEP_NS));
+#else
+  return __all_sync(0xffffffffu, mbar_wait_timed(bar, parity));
+#endif
+}
+FP4KV_DEV bool softmax_wait(uint64_t* bar, uint32_t parity) {
+#ifdef ATTN_SOFTMAX_LANE0
+  return mbar_wait_warp(bar, parity);
+#else
+  return __all_sync(0xffffffffu, mbar_wait_timed(bar, parity));
+#endif
+}
+
 FP4KV_DEV void fail_wait(const AttnParams& p, volatile uint32_t* abort_flag) {
   atomicOr(p.status, kFlagWaitTimeout);
   *abort_flag = 1;
@@ -203,63 +224,99 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 
   if (warp >= kSoftWarps && warp < kMmaWarp) {
     // ------------------------------ gather + dequantize ------------------------------
-    const int e = tid - kSoftThreads;  // tile row of this thread
+    // Gather warp g handles tile rows 32 g + 8 i + qd (i = 0..3, qd = lane / 4): the four
+    // lanes of a quad share a row, so one warp load covers the same 64-byte slice of eight
+    // rows (32 different rows per load would multiply the requests the SM has in flight,
+    // which every load/store instruction of the CTA then queues behind). Lane j = lane % 4
+    // holds, for chunk pair cp (dims [128 cp, +128) = code bytes [64 cp, +64)), the code
+    // bytes [64 cp + 16 j, +16): dims [128 cp + 32 j, +32), scale groups 8 cp + 2 j and + 1.
+    const int gw = warp - kSoftWarps;
+    const int qd = lane >> 2, j = lane & 3;
     const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
     const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
     griddep_wait();  // the index list comes from the preceding kernel on the stream
-    int32_t pos_next = e_begin + e < e_end ? idx[e_begin + e] : -1;
+    int32_t pos_next[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int je = e_begin + 32 * gw + 8 * i + qd;
+      pos_next[i] = je < e_end ? idx[je] : -1;
+    }
     for (int t = 0; t < n_tiles && !*s_abort; ++t) {
-      int32_t pos = pos_next;
-      if (pos < 0 || pos >= len) pos = -1;
-      {  // the next tile's position is fetched one tile ahead
-        const int jn = e_begin + (t + 1) * kTile + e;
-        pos_next = jn < e_end ? idx[jn] : -1;
+      // Tile t's rows are loaded only once the softmax warps have read tile t - 1's logits
+      // from TMEM: a TMEM load completes behind the global loads the SM has in flight, so
+      // loads issued earlier would stall the softmax. They still overlap the probabilities
+      // and P.V of tile t - 1, ahead of the first chunk they are needed for.
+      if (t > 0 && !gather_wait(&bars[B_SFREE + ((t - 1) & 1)], ((t - 1) >> 1) & 1)) {
+        if (lane == 0) fail_wait(p, s_abort);
+        break;
       }
-      uint4 pk[16];
-      uint4 sc0 = make_uint4(0, 0, 0, 0), sc1 = sc0;
-      if (pos >= 0) {
-        const uint8_t* prow = packed_b + int64_t(pos) * (kD / 2);
-        const uint8_t* srow = scales_b + int64_t(pos) * (kD / kGroup);
+      int32_t pos[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = ld_nc_v4(prow + 16 * i);
-        sc0 = ld_nc_v4(srow);
-        sc1 = ld_nc_v4(srow + 16);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) {
+        pos[i] = (pos_next[i] >= 0 && pos_next[i] < len) ? pos_next[i] : -1;
+        const int jn = e_begin + (t + 1) * kTile + 32 * gw + 8 * i + qd;  // one tile ahead
+        pos_next[i] = jn < e_end ? idx[jn] : -1;
       }
-      const uint32_t scw[8] = {sc0.x, sc0.y, sc0.z, sc0.w, sc1.x, sc1.y, sc1.z, sc1.w};
+      uint4 pk[4][4];  // [chunk pair][row]
+      uint2 s8[4];     // [row]: the row's scale bytes [8 j, +8) (those of chunk pair j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (pos[i] >= 0) {
+          const uint8_t* prow = packed_b + int64_t(pos[i]) * (kD / 2) + 16 * j;
+#pragma unroll
+          for (int cp = 0; cp < 4; ++cp) pk[cp][i] = ld_nc_v4(prow + 64 * cp);
+          s8[i] = ld_nc_v2(scales_b + int64_t(pos[i]) * (kD / kGroup) + 8 * j);
+        } else {
+#pragma unroll
+          for (int cp = 0; cp < 4; ++cp) pk[cp][i] = make_uint4(0, 0, 0, 0);
+          s8[i] = make_uint2(0, 0);
+        }
+      }
       bool ok = true;  // (no break inside this fully unrolled loop: registers stay registers)
 #pragma unroll
-      for (int jc = 0; jc < kChunks; ++jc) {
-        if (ok && !mbar_wait_timed(&bars[B_VFREE + jc], (t & 1) ^ 1)) {
-          fail_wait(p, s_abort);
+      for (int cp = 0; cp < 4; ++cp) {
+        if (ok && (!gather_wait(&bars[B_VFREE + 2 * cp], (t & 1) ^ 1) ||
+                   !gather_wait(&bars[B_VFREE + 2 * cp + 1], (t & 1) ^ 1))) {
+          if (lane == 0) fail_wait(p, s_abort);
           ok = false;
         }
         if (!ok) continue;
-        uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + e * 128;
+        const int jc = 2 * cp + (j >> 1);  // chunk of this lane's 32 dims
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {  // 16 dims per scale group
-          const uint32_t sb = (scw[jc] >> (8 * g)) & 0xffu;
-          const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint16_t>(sb * 0x101u));
-          const uint4 src = pk[2 * jc + (g >> 1)];
-          const uint32_t w0 = (g & 1) ? src.z : src.x;
-          const uint32_t w1 = (g & 1) ? src.w : src.y;
-          uint4 o0, o1;
-          o0.x = hmul2_f16(e2m1x2_to_f16x2(w0 & 0xffu), s2);
-          o0.y = hmul2_f16(e2m1x2_to_f16x2((w0 >> 8) & 0xffu), s2);
-          o0.z = hmul2_f16(e2m1x2_to_f16x2((w0 >> 16) & 0xffu), s2);
-          o0.w = hmul2_f16(e2m1x2_to_f16x2(w0 >> 24), s2);
-          o1.x = hmul2_f16(e2m1x2_to_f16x2(w1 & 0xffu), s2);
-          o1.y = hmul2_f16(e2m1x2_to_f16x2((w1 >> 8) & 0xffu), s2);
-          o1.z = hmul2_f16(e2m1x2_to_f16x2((w1 >> 16) & 0xffu), s2);
-          o1.w = hmul2_f16(e2m1x2_to_f16x2(w1 >> 24), s2);
-          *reinterpret_cast<uint4*>(vrow + (((2 * g) ^ (e & 7)) << 4)) = o0;
-          *reinterpret_cast<uint4*>(vrow + (((2 * g + 1) ^ (e & 7)) << 4)) = o1;
+        for (int i = 0; i < 4; ++i) {
+          const int r = 32 * gw + 8 * i + qd;
+          // scale bytes 8 cp + 2 j, + 1 of row r: held by quad lane cp, word j / 2
+          const uint32_t w0 = __shfl_sync(0xffffffffu, s8[i].x, 4 * qd + cp);
+          const uint32_t w1 = __shfl_sync(0xffffffffu, s8[i].y, 4 * qd + cp);
+          const uint32_t sw = ((j >> 1) ? w1 : w0) >> (16 * (j & 1));
+          const uint32_t sA = e4m3x2_to_f16x2(static_cast<uint16_t>((sw & 0xffu) * 0x101u));
+          const uint32_t sB = e4m3x2_to_f16x2(static_cast<uint16_t>(((sw >> 8) & 0xffu) * 0x101u));
+          const uint4 src = pk[cp][i];
+          uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + r * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            // 8-dim unit uu of this lane's 32 dims; lanes j and j + 2 (same units, different
+            // chunks) go in a staggered order so that a store phase hits distinct banks
+            const bool st = (j & 2) != 0;
+            const int uu0 = k, uu1 = k ^ 2;
+            const uint32_t w = st ? (uu1 == 0 ? src.x : uu1 == 1 ? src.y : uu1 == 2 ? src.z : src.w)
+                                  : (uu0 == 0 ? src.x : uu0 == 1 ? src.y : uu0 == 2 ? src.z : src.w);
+            const uint32_t s2 = (st ? uu1 : uu0) < 2 ? sA : sB;
+            uint4 o;
+            o.x = hmul2_f16(e2m1x2_to_f16x2(w & 0xffu), s2);
+            o.y = hmul2_f16(e2m1x2_to_f16x2((w >> 8) & 0xffu), s2);
+            o.z = hmul2_f16(e2m1x2_to_f16x2((w >> 16) & 0xffu), s2);
+            o.w = hmul2_f16(e2m1x2_to_f16x2(w >> 24), s2);
+            const int unit = 4 * (j & 1) + (st ? uu1 : uu0);
+            *reinterpret_cast<uint4*>(vrow + ((unit ^ (r & 7)) << 4)) = o;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_VREADY + jc]);
+        if (lane == 0) {
+          mbar_arrive(&bars[B_VREADY + 2 * cp]);
+          mbar_arrive(&bars[B_VREADY + 2 * cp + 1]);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -267,8 +324,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     if (lane == 0) {
       constexpr uint32_t kIdescQK = umma_idesc(0u, 128, kHeadsPerCta, 0u, 0u);
       constexpr uint32_t kIdescPV = umma_idesc(0u, 128, kHeadsPerCta, 1u, 1u);
-      const uint32_t q0 = smem_u32(smem + kOffQ), v0 = smem_u32(smem + kOffV);
-      const uint32_t ph0 = smem_u32(smem + kOffPh), pl0 = smem_u32(smem + kOffPl);
+      // Descriptors are built once; each MMA adds its operand offset in 16-byte units to the
+      // start-address field (shared-memory addresses stay below 2^18 bytes, so the 14-bit
+      // field never carries). A single thread issues ~50 cycles apart at best for N = 64,
+      // so the issue path is kept to constant adds.
+      const uint64_t dq = sw128_kmajor_desc(smem_u32(smem + kOffQ));
+      const uint64_t dvk = sw128_kmajor_desc(smem_u32(smem + kOffV));
+      const uint64_t dvm = sw128_mnmajor_desc(smem_u32(smem + kOffV), kVChunkBytes);
+      const uint64_t dph = sw128_mnmajor_desc(smem_u32(smem + kOffPh), kPBytes);
+      const uint64_t dpl = sw128_mnmajor_desc(smem_u32(smem + kOffPl), kPBytes);
       bool ok = mbar_wait_timed(&bars[B_QREADY], 0);
       if (!ok) fail_wait(p, s_abort);
       for (int t = 0; ok && t < n_tiles; ++t) {
@@ -286,10 +350,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_f16(ds, sw128_kmajor_desc(v0 + jc * kVChunkBytes + 32 * k),
-                     sw128_kmajor_desc(q0 + jc * kQChunkBytes + 32 * k), kIdescQK, (jc | k) != 0);
+          const uint64_t a = dvk + static_cast<uint64_t>((jc * kVChunkBytes) >> 4);
+          const uint64_t bq = dq + static_cast<uint64_t>((jc * kQChunkBytes) >> 4);
+          umma_f16(ds, a, bq, kIdescQK, jc != 0);  // K steps of 16 elements = 32 bytes
+          umma_f16(ds, a + 2, bq + 2, kIdescQK, true);
+          umma_f16(ds, a + 4, bq + 4, kIdescQK, true);
+          umma_f16(ds, a + 6, bq + 6, kIdescQK, true);
         }
         if (!ok) {
           fail_wait(p, s_abort);
@@ -301,14 +367,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
           break;
         }
         tc_fence_after();
-#pragma unroll 1
+        const bool acc0 = t > 0;
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t d = tmem + 64u * c;
 #pragma unroll
-          for (int s = 0; s < kTile / 16; ++s) {
-            const uint64_t a = sw128_mnmajor_desc(v0 + 2 * c * kVChunkBytes + 2048 * s, kVChunkBytes);
-            umma_f16(d, a, sw128_mnmajor_desc(ph0 + 2048 * s, kPBytes), kIdescPV, t > 0 || s > 0);
-            umma_f16(d, a, sw128_mnmajor_desc(pl0 + 2048 * s, kPBytes), kIdescPV, true);
+          for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
+            const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
+            const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
+            umma_f16(d, a, dph + ko, kIdescPV, acc0 || s > 0);
+            umma_f16(d, a, dpl + ko, kIdescPV, true);
           }
           umma_commit(&bars[B_VFREE + 2 * c]);
           umma_commit(&bars[B_VFREE + 2 * c + 1]);
@@ -403,8 +471,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     for (int t = 0; t < n_tiles; ++t) {
       const int u = t & 1;
       const bool valid = (vmask >> t) & 1u;
-      bool f = !mbar_wait_timed(&bars[B_SFULL + u], (t >> 1) & 1);
-      f = __any_sync(0xffffffffu, f);
+      bool f = !softmax_wait(&bars[B_SFULL + u], (t >> 1) & 1);
       float z[32];
       bool over = false;
       if (!f) {
@@ -422,8 +489,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         }
         // the previous tile's P.V must be complete before P is rewritten or O rescaled
         // (it precedes this tile's S in the tensor pipe, so this wait is normally free)
-        f = !mbar_wait_timed(&bars[B_PFREE], (t & 1) ^ 1);
-        f = __any_sync(0xffffffffu, f);
+        f = !softmax_wait(&bars[B_PFREE], (t & 1) ^ 1);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) z[j] = -INFINITY;
@@ -502,8 +568,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     }
     // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----
     if (!fail && n_tiles > 0) {
-      bool f = !mbar_wait_timed(&bars[B_PFREE], (n_tiles - 1) & 1);
-      f = __any_sync(0xffffffffu, f);
+      const bool f = !softmax_wait(&bars[B_PFREE], (n_tiles - 1) & 1);
       fail = softmax_any(f);
     }
     if (fail) {

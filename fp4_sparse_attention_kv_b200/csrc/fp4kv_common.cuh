@@ -167,6 +167,11 @@ FP4KV_DEV uint4 ld_nc_v4(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
+FP4KV_DEV uint2 ld_nc_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
 FP4KV_DEV uint4 ld_stream_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"

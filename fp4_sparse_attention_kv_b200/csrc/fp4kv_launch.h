@@ -41,8 +41,10 @@ cudaError_t launch_index_score(const IndexScoreParams& p, int num_sms, cudaStrea
 // ----------------------------------------------------------------------------------------
 // Exact top-K select over per-segment fp32 values, given the first-level histogram.
 // ----------------------------------------------------------------------------------------
+constexpr int kMaxSlices = 512;   // CTAs per sequence in the top-K select kernels
+constexpr int kSelCounters = 4;   // per sequence: n_sure, digit 1 + 1, ticket, spare
 struct SelectProblem {
-  const float* values;      // [B][vstride]
+  const float* values;      // [B][vstride], vstride a multiple of 8
   int64_t vstride;
   const int32_t* seq_lens;  // [B]
   int mode;                 // 0: n = seq_len; 1: n = ceil(seq_len / 8) (block ids);
@@ -50,14 +52,17 @@ struct SelectProblem {
   const int32_t* pool;      // mode 2
   int npb;
   int k;
-  uint32_t* hist;           // [B][4096], zeroed by the last CTA of each segment
-  uint32_t* counters;       // [B][4]: n_sure, n_cand, ticket, spare
-  int32_t* sure;            // [B][k]
-  int32_t* cand;            // [B][vstride] 8-byte candidates ((order key << 32) | index)
+  uint32_t* hist;           // [B][4096] digit-1 histogram (from the scoring kernel)
+  uint32_t* hist2;          // [B][4096] digit-2 histogram
+  uint32_t* counters;       // [B][kSelCounters]
+  uint32_t* cnt1;           // [B][kMaxSlices] kept entries per slice after filter
+  uint32_t* cnt2;           // [B][kMaxSlices] ... after finish
+  uint64_t* list;           // [B][vstride] (order key << 32) | value index, per-slice regions
   int32_t* out_idx;         // [B][k]
   float* out_score;         // nullable [B][k]
   int slices;
 };
+// hist, hist2 and counters must be zero on entry; the kernels leave them zero.
 cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
                                cudaStream_t stream);
 int select_slices(int64_t n_values, int B, int num_sms);

@@ -339,9 +339,11 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<FP8, N>::kCtasPerSm)
 #pragma unroll
         for (int h = 0; h < N; ++h) wv[h] = h < p.H_I ? p.w[int64_t(cur_b) * p.H_I + h] : 0.0f;
       }
-      if (!mbar_wait_timed(&tfull[acc], aph)) {
-        atomicOr(p.status, kFlagWaitTimeout);
-        *s_abort = 1;
+      if (!mbar_wait_warp(&tfull[acc], aph)) {
+        if (lane == 0) {
+          atomicOr(p.status, kFlagWaitTimeout);
+          *s_abort = 1;
+        }
         break;
       }
       tc_fence_after();

@@ -6,17 +6,23 @@
 // layer produces its own top-K indices) and for the candidate pool (section "계층적 희소
 // 인덱서로 인덱싱 비용을 컨텍스트 길이에서 분리하기": the blocks with the highest block max).
 //
-// Values are mapped to order-preserving 32-bit keys. The scoring kernel has already built
-// a histogram of the top 12 key bits per sequence. This kernel, launched with several CTAs
-// per sequence:
-//  1. finds the digit b* of the K-th largest key from that histogram (suffix sums);
-//  2. streams its slice of the values: keys with digit > b* are certainly selected
-//     ("sure", fewer than K in total), keys with digit == b* are candidates;
-//  3. takes a ticket; the last CTA of the sequence resolves the candidates exactly with
-//     three more radix passes on the key (8+8+4 bits) and, if the K-th key is tied, radix
-//     passes on the position (lowest positions win), then bitonic-sorts the selected
-//     positions and writes them. It also zeroes the histogram and counters, leaving the
-//     workspace ready for the next call. No CTA ever waits on another.
+// Values are mapped to order-preserving 32-bit keys. The scoring kernel has already built a
+// histogram of the top 12 key bits (digit 1) per sequence. Two kernels follow, each with
+// several CTAs per sequence, every CTA owning one slice of the values:
+//  filter  finds the digit-1 value b1 of the K-th largest key, keeps the keys with digit 1
+//          >= b1 (in position order, in its slice's own region of the list array), counts
+//          those above b1 ("sure") and builds a histogram of the next 12 bits (digit 2) of
+//          the keys with digit 1 == b1;
+//  finish  (a programmatic dependent of filter) finds the digit-2 value b2 of the K-th key,
+//          drops from its slice list the keys with digit 1 == b1 and digit 2 < b2, and takes
+//          a ticket; the last CTA of the sequence resolves the few keys left in the (b1, b2)
+//          bin exactly (the last 8 key bits, then the lowest positions among equal keys),
+//          and writes the selection by one ordered compaction of the slice lists. Slices are
+//          in position order and each list is in position order, so positions come out
+//          ascending without a sort (the pool mode, whose positions need not grow with the
+//          value index, sorts its at most 4096 selected pairs). That CTA also zeroes the
+//          histograms and counters, leaving the workspace ready for the next call.
+// No CTA ever waits on another CTA.
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
 #include "fp4kv_sm100.cuh"
@@ -25,8 +31,12 @@ namespace fp4kv {
 namespace {
 
 constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kPer = 8;                         // consecutive values per thread and batch
+constexpr int kBatchVals = kSelThreads * kPer;  // 4096
 constexpr int kMaxSel = 4096;
 constexpr int kMaxProblems = 2;
+constexpr int kStage = 6144;  // kept entries the finishing CTA stages in shared memory
 
 struct SelectArgs {
   SelectProblem p[kMaxProblems];
@@ -43,10 +53,61 @@ FP4KV_DEV int64_t n_values(const SelectProblem& P, int b) {
   return int64_t(P.npb) * 8;
 }
 
+// Slice s of n values: [s * per, min(n, (s + 1) * per)), per a multiple of 8.
+FP4KV_DEV int64_t slice_per(int64_t n, int slices) {
+  const int64_t q = int64_t(slices) * 8;
+  return (n + q - 1) / q * 8;
+}
+
 FP4KV_DEV int64_t position_of(const SelectProblem& P, int b, int64_t i) {
   if (P.mode != 2) return i;
   const int64_t j = P.pool[int64_t(b) * P.npb + i / 8];
   return j * 8 + (i % 8);
+}
+
+// entry = (order key << 32) | value index
+FP4KV_DEV uint32_t ent_key(uint64_t c) { return static_cast<uint32_t>(c >> 32); }
+FP4KV_DEV int32_t ent_idx(uint64_t c) { return static_cast<int32_t>(c & 0xffffffffu); }
+FP4KV_DEV int digit1(uint32_t key) { return static_cast<int>(key >> 20); }
+FP4KV_DEV int digit2(uint32_t key) { return static_cast<int>((key >> 8) & 0xfffu); }
+
+// Block-wide exclusive prefix sum in thread order; *total receives the block sum.
+// Every thread of the block must call it (it contains barriers).
+FP4KV_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* s_wsum, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = lane < kSelWarps ? s_wsum[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kSelWarps) s_wsum[lane] = t;
+  }
+  __syncthreads();
+  const uint32_t excl = x - v + (warp > 0 ? s_wsum[warp - 1] : 0u);
+  *total = s_wsum[kSelWarps - 1];
+  __syncthreads();
+  return excl;
+}
+
+// Copies a 4096-bin histogram from global memory into shared memory: 8 bins (two 16-byte
+// loads) per thread, all in flight at once.
+FP4KV_DEV void load_hist(uint32_t* s_dst, const uint32_t* g_src) {
+  static_assert(kHistBins == kSelThreads * 8, "8 bins per thread");
+  const uint4* src = reinterpret_cast<const uint4*>(g_src) + threadIdx.x * 2;
+  const uint4 a = __ldcg(src), c = __ldcg(src + 1);
+  uint4* dst = reinterpret_cast<uint4*>(s_dst) + threadIdx.x * 2;
+  dst[0] = a;
+  dst[1] = c;
 }
 
 // Block-wide: find the digit d (scanning from the highest digit down) at which the running
@@ -60,7 +121,6 @@ __device__ void find_digit_desc(const uint32_t* h, int nbins, uint32_t r, int* d
   const int hi = nbins - tid * per;
   uint32_t sum = 0;
   for (int d = hi - 1; d >= hi - per && d >= 0; --d) sum += h[d];
-  // inclusive scan over threads (thread 0 = highest digits)
   const int lane = tid & 31, w = tid >> 5;
   uint32_t x = sum;
 #pragma unroll
@@ -71,18 +131,18 @@ __device__ void find_digit_desc(const uint32_t* h, int nbins, uint32_t r, int* d
   if (lane == 31) s_scan[w] = x;
   __syncthreads();
   if (w == 0) {
-    uint32_t v = lane < kSelThreads / 32 ? s_scan[lane] : 0;
+    uint32_t v = lane < kSelWarps ? s_scan[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += y;
     }
-    if (lane < kSelThreads / 32) s_scan[32 + lane] = v;  // inclusive warp prefix
+    if (lane < kSelWarps) s_scan[32 + lane] = v;  // inclusive warp prefix
   }
   __syncthreads();
   const uint32_t incl = x + (w > 0 ? s_scan[32 + w - 1] : 0u);
   const uint32_t excl = incl - sum;
-  const uint32_t total = s_scan[32 + kSelThreads / 32 - 1];
+  const uint32_t total = s_scan[32 + kSelWarps - 1];
   if (tid == 0) {
     s_scan[64] = 0xffffffffu;  // digit
     s_scan[65] = total;
@@ -127,7 +187,7 @@ __device__ void find_digit_asc(const uint32_t* h, int nbins, uint32_t r, int* d_
 // Block-wide ascending bitonic sort of N = kSelThreads * E keys held in shared memory.
 // Each thread keeps E consecutive keys in registers: strides below E are exchanged inside
 // the thread, strides up to 16 E through warp shuffles, and only the widest strides through
-// shared memory (one barrier pair each). Every stage is unrolled at compile time.
+// shared memory (one barrier pair each).
 template <typename T, int E>
 __device__ void block_sort(T* s) {
   constexpr int N = kSelThreads * E;
@@ -179,214 +239,168 @@ __device__ void block_sort(T* s) {
   __syncthreads();
 }
 
-// candidate = (order key << 32) | value index
-FP4KV_DEV uint32_t cand_key(uint64_t c) { return static_cast<uint32_t>(c >> 32); }
-FP4KV_DEV int32_t cand_idx(uint64_t c) { return static_cast<int32_t>(c & 0xffffffffu); }
-
-template <bool kShared>
-FP4KV_DEV uint64_t load_cand(const uint64_t* c, uint32_t i) {
-  if constexpr (kShared) return c[i];
-  return __ldcg(reinterpret_cast<const unsigned long long*>(c) + i);
-}
-
-// Exact resolution of the candidates (all sharing the top 12 key bits `bstar`): finds the
-// r-th largest key ustar among them and, when that key is tied, the largest position
-// pos_star that is still taken (lowest positions win). Candidates live in shared memory
-// (kShared) or, when too many, in global memory.
-template <bool kShared>
-__device__ void resolve_candidates(const SelectProblem& P, int b, const uint64_t* cand,
-                                   uint32_t n_cand, uint32_t r, int bstar, uint32_t* s_hist,
-                                   uint32_t* s_scan, uint32_t* ustar_out, int64_t* pos_star_out) {
-  const int tid = threadIdx.x;
-  uint32_t prefix = static_cast<uint32_t>(bstar);
-  int consumed = kHistBits;
-  const int widths[3] = {8, 8, 4};
-  uint32_t cnt_eq = 0;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int wbits = widths[pass];
-    const int shift = 32 - consumed - wbits;
-    const int nb = 1 << wbits;
-    for (int i = tid; i < nb; i += kSelThreads) s_hist[i] = 0;
-    __syncthreads();
-    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-      const uint32_t key = cand_key(load_cand<kShared>(cand, c));
-      if ((key >> (shift + wbits)) == prefix) atomicAdd(&s_hist[(key >> shift) & (nb - 1)], 1u);
-    }
-    __syncthreads();
-    int d;
-    uint32_t ab;
-    find_digit_desc(s_hist, nb, r, &d, &ab, s_scan);
-    r -= ab;
-    cnt_eq = s_hist[d];
-    prefix = (prefix << wbits) | static_cast<uint32_t>(d);
-    consumed += wbits;
-    __syncthreads();
-  }
-  *ustar_out = prefix;
-  *pos_star_out = INT64_MAX;
-  if (r < cnt_eq) {
-    // lowest r positions among the keys equal to ustar: passes of 8 bits over 32 bits
-    uint64_t pprefix = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelThreads) s_hist[i] = 0;
-      __syncthreads();
-      for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-        const uint64_t cv = load_cand<kShared>(cand, c);
-        if (cand_key(cv) != prefix) continue;
-        const uint64_t pos = static_cast<uint64_t>(position_of(P, b, cand_idx(cv)));
-        if ((pos >> (shift + 8)) == pprefix) atomicAdd(&s_hist[(pos >> shift) & 255], 1u);
-      }
-      __syncthreads();
-      int d;
-      uint32_t below;
-      find_digit_asc(s_hist, 256, r, &d, &below, s_scan);
-      r -= below;
-      pprefix = (pprefix << 8) | static_cast<uint64_t>(d);
-    }
-    *pos_star_out = static_cast<int64_t>(pprefix);
-  }
-}
-
-// Appends the taken candidates to s_sel at *s_cnt (one shared atomic per warp).
-template <bool kShared>
-__device__ void collect_candidates(const SelectProblem& P, int b, const uint64_t* cand,
-                                   uint32_t n_cand, bool take_all, uint32_t ustar,
-                                   int64_t pos_star, uint64_t* s_sel, uint32_t* s_cnt) {
-  const int lane = threadIdx.x & 31;
-  for (uint32_t c0 = 0; c0 < n_cand; c0 += kSelThreads) {
-    const uint32_t c = c0 + threadIdx.x;
-    bool take = false;
-    uint64_t item = 0;
-    if (c < n_cand) {
-      const uint64_t cv = load_cand<kShared>(cand, c);
-      const int32_t i = cand_idx(cv);
-      const int64_t pos = position_of(P, b, i);
-      const uint32_t key = cand_key(cv);
-      take = take_all || key > ustar || (key == ustar && pos <= pos_star);
-      item = (static_cast<uint64_t>(pos) << 32) | static_cast<uint32_t>(i);
-    }
-    const uint32_t m = __ballot_sync(0xffffffffu, take);
-    if (m == 0) continue;
-    const int leader = __ffs(m) - 1;
-    uint32_t base = 0;
-    if (lane == leader) base = atomicAdd(s_cnt, static_cast<uint32_t>(__popc(m)));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    const uint32_t slot = base + static_cast<uint32_t>(__popc(m & ((1u << lane) - 1u)));
-    if (take && slot < kMaxSel) s_sel[slot] = item;
-  }
-}
-
-constexpr int kCandSmem = 6144;  // candidates staged in shared memory when they fit
-constexpr size_t kSelSmem = size_t(kMaxSel) * 8 + size_t(kCandSmem) * 8;
-
-__global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs args) {
-  const SelectProblem& P = args.p[blockIdx.z];
-  const int b = blockIdx.y;
-  if (static_cast<int>(blockIdx.x) >= P.slices) return;
-  // s_sel: the selected (position, index) pairs; its first 16 KiB also serve as the
-  // histogram of phase 1 and of the radix passes (never live at the same time).
-  extern __shared__ __align__(16) uint8_t sel_smem[];
-  uint64_t* s_sel = reinterpret_cast<uint64_t*>(sel_smem);
-  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_sel);
-  uint64_t* s_cand = s_sel + kMaxSel;
-  __shared__ uint32_t s_scan[96];
-  __shared__ uint32_t s_cnt;
-  __shared__ bool s_last;
-  const int tid = threadIdx.x;
-  // a kernel launched after this one as a programmatic dependent may start its own
-  // prologue now (it waits for this grid's completion before reading the results)
+// --------------------------------------------------------------------------------------
+// filter
+// --------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSelThreads) k_select_filter(const SelectArgs args) {
+  // the finishing kernel is a programmatic dependent: it may be scheduled from now on
   griddep_launch_dependents();
+  const SelectProblem& P = args.p[blockIdx.z];
+  const int b = blockIdx.y, s = blockIdx.x;
+  if (s >= P.slices) return;
+  __shared__ __align__(16) uint32_t s_h[kHistBins];  // digit-1 histogram, then this slice's digit-2 one
+  __shared__ uint32_t s_scan[96];
+  __shared__ uint32_t s_wsum[kSelWarps];
+  const int tid = threadIdx.x;
 
   const int64_t n = n_values(P, b);
+  const int64_t per = slice_per(n, P.slices);
+  const int64_t lo = per * s;
+  const int64_t hi = lo + per < n ? lo + per : n;
   const float* vals = P.values + int64_t(b) * P.vstride;
-  uint32_t* hist = P.hist + int64_t(b) * kHistBins;
-  uint32_t* ctr = P.counters + int64_t(b) * 4;
-  int32_t* sure = P.sure + int64_t(b) * P.k;
-  uint64_t* cand = reinterpret_cast<uint64_t*>(P.cand) + int64_t(b) * P.vstride;
+  uint32_t* ctr = P.counters + int64_t(b) * kSelCounters;
+  uint64_t* list = P.list + int64_t(b) * P.vstride;
 
-  // 1. digit of the K-th largest key
-  for (int i = tid; i < kHistBins; i += kSelThreads) s_hist[i] = __ldcg(hist + i);
+  // digit 1 of the K-th largest key (b1 = -1: fewer than K valid values, all are kept)
+  load_hist(s_h, P.hist + int64_t(b) * kHistBins);
   __syncthreads();
-  int bstar;
+  int b1;
   uint32_t above;
-  find_digit_desc(s_hist, kHistBins, static_cast<uint32_t>(P.k), &bstar, &above, s_scan);
-  // bstar == -1: fewer than K valid values; every valid value is "sure"
+  find_digit_desc(s_h, kHistBins, static_cast<uint32_t>(P.k), &b1, &above, s_scan);
+  for (int i = tid; i < kHistBins; i += kSelThreads) s_h[i] = 0;
+  __syncthreads();
 
-  // 2. filter this CTA's slice
-  const int64_t lo = n * blockIdx.x / P.slices;
-  const int64_t hi = n * (blockIdx.x + 1) / P.slices;
-  // Each batch of 8 values per thread is classified in registers; one block-wide prefix
-  // sum of the (sure, candidate) counts then gives every thread its output slots, and one
-  // global atomic per list and batch reserves the CTA's range (appends racing on the
-  // per-sequence counters would cost a memory round trip each).
-  constexpr int kBatch = 8;
-  __shared__ uint32_t s_wsum[kSelThreads / 32];
-  __shared__ uint32_t s_base[2];
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int64_t base = lo; base < hi; base += int64_t(kSelThreads) * kBatch) {
-    float v[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t i = base + int64_t(u) * kSelThreads + tid;
-      v[u] = i < hi ? __ldg(vals + i) : -INFINITY;
+  // keys with digit 1 >= b1, in position order, into list[lo ..)
+  uint32_t run = 0, n_sure = 0;
+  for (int64_t base = lo; base < hi; base += kBatchVals) {
+    const int64_t i0 = base + int64_t(tid) * kPer;
+    float v[kPer];
+    if (i0 < hi) {  // i0 is a multiple of 8 and below vstride (a multiple of 4)
+      const float4 a = __ldg(reinterpret_cast<const float4*>(vals + i0));
+      const float4 c = __ldg(reinterpret_cast<const float4*>(vals + i0 + 4));
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
     }
-    uint32_t smask = 0, cmask = 0, keys[kBatch];
+    uint32_t keep = 0, keys[kPer];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t i = base + int64_t(u) * kSelThreads + tid;
+    for (int u = 0; u < kPer; ++u) {
       keys[u] = 0;
-      if (i < hi && (v[u] != -INFINITY || P.mode != 2)) {
+      if (i0 + u < hi && (P.mode != 2 || v[u] != -INFINITY)) {
         keys[u] = order_key(v[u]);
-        const int digit = static_cast<int>(keys[u] >> (32 - kHistBits));
-        if (digit > bstar) smask |= 1u << u;
-        else if (digit == bstar) cmask |= 1u << u;
+        const int d = digit1(keys[u]);
+        if (d > b1) {
+          keep |= 1u << u;
+          ++n_sure;
+        } else if (d == b1) {
+          keep |= 1u << u;
+          atomicAdd(&s_h[digit2(keys[u])], 1u);
+        }
       }
     }
-    // counts packed as (sure << 16) | candidates: a batch holds at most 4096 of each
-    const uint32_t cnt = (static_cast<uint32_t>(__popc(smask)) << 16) | static_cast<uint32_t>(__popc(cmask));
-    uint32_t x = cnt;
+    uint32_t total;
+    uint32_t o = run + block_excl_scan(static_cast<uint32_t>(__popc(keep)), s_wsum, &total);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_wsum[warp] = x;
+    for (int u = 0; u < kPer; ++u)
+      if ((keep >> u) & 1u)
+        list[lo + o++] = (static_cast<uint64_t>(keys[u]) << 32) | static_cast<uint32_t>(i0 + u);
+    run += total;
+  }
+  uint32_t sure_total;
+  block_excl_scan(n_sure, s_wsum, &sure_total);  // (block sum)
+  if (tid == 0) {
+    P.cnt1[int64_t(b) * kMaxSlices + s] = run;
+    if (sure_total) atomicAdd(&ctr[0], sure_total);
+    if (s == 0) ctr[1] = static_cast<uint32_t>(b1 + 1);
+  }
+  // merge this slice's digit-2 histogram into the sequence's
+  uint32_t* h2 = P.hist2 + int64_t(b) * kHistBins;
+  for (int i = tid; i < kHistBins; i += kSelThreads) {
+    const uint32_t c = s_h[i];
+    if (c) atomicAdd(&h2[i], c);
+  }
+}
+
+// --------------------------------------------------------------------------------------
+// finish
+// --------------------------------------------------------------------------------------
+// Entry j (0 <= j < total) of the concatenated slice lists.
+FP4KV_DEV uint64_t kept_entry(const uint64_t* list, const uint32_t* s_off, int slices, int64_t per,
+                              uint32_t j) {
+  int lo = 0, hi = slices - 1;  // last slice with s_off[slice] <= j
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_off[mid] <= j) lo = mid;
+    else hi = mid - 1;
+  }
+  return __ldcg(reinterpret_cast<const unsigned long long*>(list) + per * lo + (j - s_off[lo]));
+}
+
+constexpr size_t kFinSmem = size_t(kStage) * 8 + size_t(kMaxSel) * 8 + size_t(kMaxSlices + 1) * 4;
+
+__global__ void __launch_bounds__(kSelThreads) k_select_finish(const SelectArgs args) {
+  griddep_wait();  // the filter grid has completed and its writes are visible
+  griddep_launch_dependents();
+  const SelectProblem& P = args.p[blockIdx.z];
+  const int b = blockIdx.y, s = blockIdx.x;
+  if (s >= P.slices) return;
+  extern __shared__ __align__(16) uint8_t fin_smem[];
+  uint64_t* s_stage = reinterpret_cast<uint64_t*>(fin_smem);       // [kStage]
+  uint64_t* s_sel = s_stage + kStage;                              // [kMaxSel]
+  uint32_t* s_h = reinterpret_cast<uint32_t*>(s_sel);              // digit-2 histogram (aliases s_sel)
+  uint32_t* s_off = reinterpret_cast<uint32_t*>(s_sel + kMaxSel);  // [kMaxSlices + 1]
+  __shared__ uint32_t s_scan[96];
+  __shared__ uint32_t s_wsum[kSelWarps];
+  __shared__ uint32_t s_hist8[256];
+  __shared__ bool s_last;
+  const int tid = threadIdx.x;
+
+  const int64_t n = n_values(P, b);
+  const int64_t per = slice_per(n, P.slices);
+  const int64_t lo = per * s;
+  uint32_t* ctr = P.counters + int64_t(b) * kSelCounters;
+  uint64_t* list = P.list + int64_t(b) * P.vstride;
+  uint32_t* h2g = P.hist2 + int64_t(b) * kHistBins;
+  const int b1 = static_cast<int>(__ldcg(&ctr[1])) - 1;
+  const uint32_t n_sure = __ldcg(&ctr[0]);
+  const uint32_t k = static_cast<uint32_t>(P.k);
+  const uint32_t r = k > n_sure ? k - n_sure : 0u;  // keys still to take from digit 1 == b1
+
+  // digit 2 of the K-th key: b2 = -1 takes every key of the b1 bin; b2 = 4096 takes none
+  int b2 = kHistBins;
+  uint32_t above2 = 0, bin_count = 0;
+  if (r > 0 && b1 >= 0) {
+    load_hist(s_h, h2g);
     __syncthreads();
-    if (warp == 0) {
-      uint32_t t = lane < kSelThreads / 32 ? s_wsum[lane] : 0u;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
-        if (lane >= o) t += y;
-      }
-      if (lane < kSelThreads / 32) s_wsum[lane] = t;  // inclusive prefix over warps
-      if (lane == kSelThreads / 32 - 1) {
-        s_base[0] = (t >> 16) ? atomicAdd(&ctr[0], t >> 16) : 0u;
-        s_base[1] = (t & 0xffffu) ? atomicAdd(&ctr[1], t & 0xffffu) : 0u;
-      }
-    }
+    find_digit_desc(s_h, kHistBins, r, &b2, &above2, s_scan);
+    if (b2 >= 0) bin_count = s_h[b2];
     __syncthreads();
-    const uint32_t excl = x - cnt + (warp > 0 ? s_wsum[warp - 1] : 0u);
-    uint32_t so = s_base[0] + (excl >> 16), co = s_base[1] + (excl & 0xffffu);
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int64_t i = base + int64_t(u) * kSelThreads + tid;
-      if ((smask >> u) & 1u) {
-        if (so < static_cast<uint32_t>(P.k)) sure[so] = static_cast<int32_t>(i);
-        ++so;
-      }
-      if ((cmask >> u) & 1u) {
-        if (co < static_cast<uint32_t>(P.vstride))
-          cand[co] = (static_cast<uint64_t>(keys[u]) << 32) | static_cast<uint32_t>(i);
-        ++co;
-      }
-    }
-    __syncthreads();  // s_wsum and s_base are reused by the next batch
   }
 
-  // 3. ticket: the last CTA of this sequence finalises
+  // drop the keys of the b1 bin below b2 from this slice's list (in place, order kept)
+  const uint32_t cnt = __ldcg(P.cnt1 + int64_t(b) * kMaxSlices + s);
+  uint32_t run = 0;
+  for (uint32_t j0 = 0; j0 < cnt; j0 += kSelThreads * 4) {
+    uint64_t e[4];
+    uint32_t keep = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = j0 + tid * 4 + u;
+      e[u] = 0;
+      if (j < cnt) {
+        e[u] = __ldcg(reinterpret_cast<const unsigned long long*>(list) + lo + j);
+        const uint32_t key = ent_key(e[u]);
+        if (digit1(key) != b1 || digit2(key) >= b2) keep |= 1u << u;
+      }
+    }
+    uint32_t total;
+    uint32_t o = run + block_excl_scan(static_cast<uint32_t>(__popc(keep)), s_wsum, &total);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if ((keep >> u) & 1u) list[lo + o++] = e[u];
+    run += total;
+  }
   __syncthreads();
   if (tid == 0) {
+    P.cnt2[int64_t(b) * kMaxSlices + s] = run;
     __threadfence();
     const uint32_t t = atomicAdd(&ctr[2], 1u);
     s_last = (t == static_cast<uint32_t>(P.slices - 1));
@@ -395,90 +409,142 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const SelectArgs ar
   if (!s_last) return;
   __threadfence();
 
-  const uint32_t n_sure = min(__ldcg(&ctr[0]), static_cast<uint32_t>(P.k));
-  const uint32_t n_cand = min(__ldcg(&ctr[1]), static_cast<uint32_t>(P.vstride));
-  const uint32_t r = static_cast<uint32_t>(P.k) > n_sure ? static_cast<uint32_t>(P.k) - n_sure : 0u;
-  const bool take_all = n_cand <= r;
-  const bool in_smem = n_cand <= static_cast<uint32_t>(kCandSmem);
-  if (in_smem) {
-    for (uint32_t c = tid; c < n_cand; c += kSelThreads)
-      s_cand[c] = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + c);
+  // ---- last CTA of the sequence: offsets of the slice lists ----
+  uint32_t total_kept;
+  {
+    const uint32_t c = tid < P.slices ? __ldcg(P.cnt2 + int64_t(b) * kMaxSlices + tid) : 0u;
+    const uint32_t ex = block_excl_scan(c, s_wsum, &total_kept);
+    if (tid < P.slices) s_off[tid] = ex;
+    if (tid == 0) s_off[P.slices] = total_kept;
     __syncthreads();
   }
+  const bool staged = total_kept <= static_cast<uint32_t>(kStage);
+  if (staged) {
+    for (uint32_t j = tid; j < total_kept; j += kSelThreads)
+      s_stage[j] = kept_entry(list, s_off, P.slices, per, j);
+    __syncthreads();
+  }
+  auto entry = [&](uint32_t j) -> uint64_t {
+    return staged ? s_stage[j] : kept_entry(list, s_off, P.slices, per, j);
+  };
+
+  // ---- the (b1, b2) bin: r2 of its keys are taken ----
+  const uint32_t r2 = r > above2 ? r - above2 : 0u;
+  const bool in_range = b1 >= 0 && b2 >= 0 && b2 < kHistBins;
+  const bool bin_all = !in_range || r2 >= bin_count;
+  const uint32_t pre24 = in_range ? (static_cast<uint32_t>(b1) << 12) | static_cast<uint32_t>(b2) : 0u;
   uint32_t ustar = 0;
   int64_t pos_star = INT64_MAX;
-  if (!take_all && r > 0) {
-    if (in_smem)
-      resolve_candidates<true>(P, b, s_cand, n_cand, r, bstar, s_hist, s_scan, &ustar, &pos_star);
-    else
-      resolve_candidates<false>(P, b, cand, n_cand, r, bstar, s_hist, s_scan, &ustar, &pos_star);
+  if (in_range && !bin_all && r2 > 0) {
+    // the last 8 key bits
+    for (int i = tid; i < 256; i += kSelThreads) s_hist8[i] = 0;
+    __syncthreads();
+    for (uint32_t j = tid; j < total_kept; j += kSelThreads) {
+      const uint32_t key = ent_key(entry(j));
+      if ((key >> 8) == pre24) atomicAdd(&s_hist8[key & 255u], 1u);
+    }
+    __syncthreads();
+    int d3;
+    uint32_t above3;
+    find_digit_desc(s_hist8, 256, r2, &d3, &above3, s_scan);
+    ustar = (pre24 << 8) | static_cast<uint32_t>(d3);
+    uint32_t rr = r2 - above3;
+    const uint32_t cnt_eq = s_hist8[d3];
+    __syncthreads();
+    if (rr < cnt_eq) {
+      // the rr lowest positions among the keys equal to ustar: 8-bit passes over 32 bits
+      uint64_t pprefix = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kSelThreads) s_hist8[i] = 0;
+        __syncthreads();
+        for (uint32_t j = tid; j < total_kept; j += kSelThreads) {
+          const uint64_t cv = entry(j);
+          if (ent_key(cv) != ustar) continue;
+          const uint64_t pos = static_cast<uint64_t>(position_of(P, b, ent_idx(cv)));
+          if ((pos >> (shift + 8)) == pprefix) atomicAdd(&s_hist8[(pos >> shift) & 255], 1u);
+        }
+        __syncthreads();
+        int d;
+        uint32_t below;
+        find_digit_asc(s_hist8, 256, rr, &d, &below, s_scan);
+        rr -= below;
+        pprefix = (pprefix << 8) | static_cast<uint64_t>(d);
+      }
+      pos_star = static_cast<int64_t>(pprefix);
+    }
   }
 
-  // collect the selected (position, value index) pairs: the sure list is compact and all
-  // of it is taken (n_sure <= K <= kMaxSel); taken candidates are appended after it
-  if (tid == 0) s_cnt = n_sure;
-  for (uint32_t c = tid; c < n_sure; c += kSelThreads) {
-    const int32_t i = __ldcg(sure + c);
-    s_sel[c] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
-  }
-  __syncthreads();
-  if (r > 0 || take_all) {
-    if (in_smem)
-      collect_candidates<true>(P, b, s_cand, n_cand, take_all, ustar, pos_star, s_sel, &s_cnt);
-    else
-      collect_candidates<false>(P, b, cand, n_cand, take_all, ustar, pos_star, s_sel, &s_cnt);
-  }
-  __syncthreads();
-  int m = static_cast<int>(s_cnt);
-  if (m > P.k) m = P.k;
-  const int nsort = m <= kSelThreads * 4 ? kSelThreads * 4 : kSelThreads * 8;
+  // ---- ordered compaction of the selected keys ----
   int32_t* oi = P.out_idx + int64_t(b) * P.k;
   float* os = P.out_score ? P.out_score + int64_t(b) * P.k : nullptr;
-  if (P.mode != 2) {
-    // position == value index: sort 32-bit positions (padding sorts last)
-    uint32_t* s_pos = reinterpret_cast<uint32_t*>(s_cand);
-    for (int i = tid; i < nsort; i += kSelThreads)
-      s_pos[i] = i < m ? static_cast<uint32_t>(s_sel[i] >> 32) : 0xffffffffu;
-    __syncthreads();
-    if (nsort == kSelThreads * 4) block_sort<uint32_t, 4>(s_pos);
-    else block_sort<uint32_t, 8>(s_pos);
-    for (int j = tid; j < P.k; j += kSelThreads) {
-      if (j < m) {
-        oi[j] = static_cast<int32_t>(s_pos[j]);
-        if (os) os[j] = vals[s_pos[j]];
-      } else {
-        oi[j] = -1;
-        if (os) os[j] = -INFINITY;
+  uint32_t m = 0;
+  for (uint32_t j0 = 0; j0 < total_kept; j0 += kSelThreads * 4) {
+    uint64_t e[4];
+    uint32_t take = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = j0 + tid * 4 + u;
+      e[u] = 0;
+      if (j < total_kept) {
+        e[u] = entry(j);
+        const uint32_t key = ent_key(e[u]);
+        bool t = true;  // digit 1 > b1, or digit 2 > b2, or the whole (b1, b2) bin
+        if (!bin_all && (key >> 8) == pre24)
+          t = r2 > 0 && (key > ustar || (key == ustar && position_of(P, b, ent_idx(e[u])) <= pos_star));
+        if (t) take |= 1u << u;
       }
     }
-  } else {
-    for (int i = m + tid; i < nsort; i += kSelThreads) s_sel[i] = ~0ull;
+    uint32_t total;
+    uint32_t o = m + block_excl_scan(static_cast<uint32_t>(__popc(take)), s_wsum, &total);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!((take >> u) & 1u)) continue;
+      if (o < k) {
+        const int32_t i = ent_idx(e[u]);
+        if (P.mode != 2) {
+          oi[o] = i;
+          if (os) os[o] = key_to_float(ent_key(e[u]));
+        } else {
+          s_sel[o] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
+        }
+      }
+      ++o;
+    }
+    m += total;
+  }
+  if (m > k) m = k;
+  if (P.mode == 2) {
+    // pool slots: positions need not grow with the value index, sort (position, index)
+    const int nsort = m <= static_cast<uint32_t>(kSelThreads * 4) ? kSelThreads * 4 : kSelThreads * 8;
+    for (int i = static_cast<int>(m) + tid; i < nsort; i += kSelThreads) s_sel[i] = ~0ull;
     __syncthreads();
     if (nsort == kSelThreads * 4) block_sort<uint64_t, 4>(s_sel);
     else block_sort<uint64_t, 8>(s_sel);
-    for (int j = tid; j < P.k; j += kSelThreads) {
-      if (j < m) {
-        oi[j] = static_cast<int32_t>(s_sel[j] >> 32);
-        if (os) os[j] = vals[static_cast<uint32_t>(s_sel[j] & 0xffffffffu)];
-      } else {
-        oi[j] = -1;
-        if (os) os[j] = -INFINITY;
-      }
+    for (uint32_t j = tid; j < m; j += kSelThreads) {
+      oi[j] = static_cast<int32_t>(s_sel[j] >> 32);
+      if (os) os[j] = P.values[int64_t(b) * P.vstride + static_cast<uint32_t>(s_sel[j] & 0xffffffffu)];
     }
   }
+  for (uint32_t j = m + tid; j < k; j += kSelThreads) {
+    oi[j] = -1;
+    if (os) os[j] = -INFINITY;
+  }
   // leave the workspace zeroed for the next call
-  for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
-  if (tid < 4) ctr[tid] = 0;
+  for (int i = tid; i < kHistBins; i += kSelThreads) {
+    P.hist[int64_t(b) * kHistBins + i] = 0;
+    h2g[i] = 0;
+  }
+  if (tid < kSelCounters) ctr[tid] = 0;
 }
 
 }  // namespace
 
 int select_slices(int64_t n_values, int B, int num_sms) {
   int64_t s = (2 * int64_t(num_sms)) / B;  // two CTAs per SM: one wave
-  const int64_t cap = (n_values + 4095) / 4096;
+  const int64_t cap = (n_values + kBatchVals - 1) / kBatchVals;
   if (s > cap) s = cap;
+  if (s > kMaxSlices) s = kMaxSlices;
   if (s < 1) s = 1;
-  if (s > 65535) s = 65535;
   return static_cast<int>(s);
 }
 
@@ -492,10 +558,24 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
     if (probs[i].slices > gx) gx = probs[i].slices;
   }
   dim3 grid(gx, B, n_probs);
-  cudaError_t e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSelSmem));
+  k_select_filter<<<grid, kSelThreads, 0, stream>>>(args);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_topk_select<<<grid, kSelThreads, kSelSmem, stream>>>(args);
+  e = cudaFuncSetAttribute(k_select_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kFinSmem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = kFinSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_select_finish, args);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -165,7 +165,7 @@ fp4kv_status fp4kv_hier_pool_select(const void* q, const float* w, int32_t H_I, 
  * before attention; [ingu627]: 64 query heads over one shared KV head).
  * Reuse mode is this call with the previous layer's idx ([PyTorchKR] CSA2 mode table).
  * q        : bf16 bits [B][H][d], 16-byte aligned.   d == 512.
- * packed, scales : the cache planes (see layout above).
+ * packed, scales : the cache planes (see layout above), both 16-byte aligned here.
  * idx      : int32 [B][top_k]; entries < 0 or >= seq_lens[b] are skipped; duplicates count.
  * out      : fp32 [B][H][d].   lse : nullable fp32 [B][H] (-inf when no entry is valid,
  *            in which case out is 0).

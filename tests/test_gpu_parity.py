@@ -201,6 +201,36 @@ def test_indexer_topk_ties_go_to_the_lowest_positions(fk):
     assert idx2[0].tolist() == list(range(3000)) + [-1] * 1096
 
 
+def test_indexer_topk_all_equal_scores_beyond_the_staging_buffer(fk):
+    # 20000 equal scores: every entry survives both radix digits, so the final selection
+    # runs over more entries than the finishing CTA stages in shared memory and is decided
+    # by position alone
+    cap = 20000
+    q, w, _ = _indexer_inputs(9, 1, cap, 32, True)
+    row = synth.indexer_keys(9, 0, torch.arange(1, dtype=torch.int64), 128, True)
+    keys = row.repeat(cap, 1).reshape(1, cap, 128).to(DEV).contiguous()
+    lens = torch.tensor([cap], dtype=torch.int32, device=DEV)
+    for k in (1, 100, 4096):
+        idx = fk.indexer_topk(q, w, keys, lens, k).cpu().numpy()
+        assert idx[0].tolist() == list(range(k)), k
+
+
+def test_reindex_with_a_pool_in_arbitrary_order(fk):
+    # pool blocks listed out of position order: the output is still ascending positions
+    B, cap, k, npb = 2, 20000, 300, 96
+    q, w, keys = _indexer_inputs(14, B, cap, 32, True)
+    lens = torch.tensor([20000, 15000], dtype=torch.int32, device=DEV)
+    rng = np.random.default_rng(14)
+    pools = [rng.permutation(int(lens[b]) // 8)[:npb].astype(np.int32) for b in range(B)]
+    pool = torch.tensor(np.stack(pools), dtype=torch.int32, device=DEV)
+    idx = fk.indexer_topk(q, w, keys, lens, k, pool=pool).cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        pos = O.pool_positions(pools[b], L, 8)
+        ref = P.oracle_scores_seq(q[b], w[b], keys[b], L)[pos]
+        P.check_topk(idx[b], ref, pos, k, f"unordered pool b={b}")
+
+
 def test_hier_pool_select_matches_oracle(fk):
     B, cap, k, npb = 2, 20000, 256, 64
     q, w, keys = _indexer_inputs(11, B, cap, 32, True)
