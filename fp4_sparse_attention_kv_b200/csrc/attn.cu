@@ -242,11 +242,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       pos_next[i] = je < e_end ? idx[je] : -1;
     }
     for (int t = 0; t < n_tiles && !*s_abort; ++t) {
-      // Tile t's rows are loaded only once the softmax warps have read tile t - 1's logits
-      // from TMEM: a TMEM load completes behind the global loads the SM has in flight, so
-      // loads issued earlier would stall the softmax. They still overlap the probabilities
-      // and P.V of tile t - 1, ahead of the first chunk they are needed for.
-      if (t > 0 && !gather_wait(&bars[B_SFREE + ((t - 1) & 1)], ((t - 1) >> 1) & 1)) {
+      // Tile t's rows are loaded only once the softmax warps have written tile t - 1's
+      // probabilities: TMEM and shared-memory accesses queue behind the global loads the
+      // SM has in flight, so loads issued earlier would stall the softmax. They overlap
+      // the P.V of tile t - 1 instead, which frees the buffers they are needed for.
+      if (t > 0 && !gather_wait(&bars[B_PREADY], (t - 1) & 1)) {
         if (lane == 0) fail_wait(p, s_abort);
         break;
       }
