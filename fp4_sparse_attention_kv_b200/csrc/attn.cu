@@ -168,6 +168,83 @@ FP4KV_DEV void fail_wait(const AttnParams& p, volatile uint32_t* abort_flag) {
   *abort_flag = 1;
 }
 
+// Loads the rows of tile t at `pos` (rows row0 + 8 i + qd of the tile, qd = lane / 4,
+// i < NG; pos < 0: an all-zero row) and dequantizes them into the V_hat chunk buffers, one
+// chunk pair at a time as the P.V of the previous tile frees it. The four lanes of a quad
+// share a row, so one warp load covers the same 64-byte slice of eight rows (32 different
+// rows per load would multiply the requests in flight, which every load/store instruction
+// of the CTA then queues behind). Lane j = lane % 4 holds, for chunk pair cp (dims
+// [128 cp, +128) = code bytes [64 cp, +64)), the code bytes [64 cp + 16 j, +16): dims
+// [128 cp + 32 j, +32), scale groups 8 cp + 2 j and + 1. Warp-collective; returns false
+// (in every lane) if a wait timed out.
+template <int NG>
+FP4KV_DEV bool load_dequant(uint8_t* smem, uint64_t* bars, const uint8_t* packed_b,
+                            const uint8_t* scales_b, const int32_t (&pos)[NG], int row0, int t) {
+  const int lane = threadIdx.x & 31, qd = lane >> 2, j = lane & 3;
+  uint4 pk[4][NG];  // [chunk pair][row group]
+  uint2 s8[NG];     // [row group]: the row's scale bytes [8 j, +8) (those of chunk pair j)
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    if (pos[i] >= 0) {
+      const uint8_t* prow = packed_b + int64_t(pos[i]) * (kD / 2) + 16 * j;
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) pk[cp][i] = ld_nc_v4(prow + 64 * cp);
+      s8[i] = ld_nc_v2(scales_b + int64_t(pos[i]) * (kD / kGroup) + 8 * j);
+    } else {
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) pk[cp][i] = make_uint4(0, 0, 0, 0);
+      s8[i] = make_uint2(0, 0);
+    }
+  }
+  bool ok = true;  // (no break inside this fully unrolled loop: registers stay registers)
+#pragma unroll
+  for (int cp = 0; cp < 4; ++cp) {
+    // (both chunks of the pair are released by the same commit point of P.V; this wait is
+    // on the critical path, so it polls without sleeping)
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_VFREE + 2 * cp], (t & 1) ^ 1) &&
+                                           mbar_wait_timed(&bars[B_VFREE + 2 * cp + 1], (t & 1) ^ 1)))
+      ok = false;
+    if (!ok) continue;
+    const int jc = 2 * cp + (j >> 1);  // chunk of this lane's 32 dims
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      const int r = row0 + 8 * i + qd;
+      // scale bytes 8 cp + 2 j, + 1 of row r: held by quad lane cp, word j / 2
+      const uint32_t w0 = __shfl_sync(0xffffffffu, s8[i].x, 4 * qd + cp);
+      const uint32_t w1 = __shfl_sync(0xffffffffu, s8[i].y, 4 * qd + cp);
+      const uint32_t sw = ((j >> 1) ? w1 : w0) >> (16 * (j & 1));
+      const uint32_t sA = e4m3x2_to_f16x2(static_cast<uint16_t>((sw & 0xffu) * 0x101u));
+      const uint32_t sB = e4m3x2_to_f16x2(static_cast<uint16_t>(((sw >> 8) & 0xffu) * 0x101u));
+      const uint4 src = pk[cp][i];
+      uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + r * 128;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // 8-dim unit uu of this lane's 32 dims; lanes j and j + 2 (same units, different
+        // chunks) go in a staggered order so that a store phase hits distinct banks
+        const bool st = (j & 2) != 0;
+        const int uu0 = k, uu1 = k ^ 2;
+        const uint32_t w = st ? (uu1 == 0 ? src.x : uu1 == 1 ? src.y : uu1 == 2 ? src.z : src.w)
+                              : (uu0 == 0 ? src.x : uu0 == 1 ? src.y : uu0 == 2 ? src.z : src.w);
+        const uint32_t s2 = (st ? uu1 : uu0) < 2 ? sA : sB;
+        uint4 o;
+        o.x = hmul2_f16(e2m1x2_to_f16x2(w & 0xffu), s2);
+        o.y = hmul2_f16(e2m1x2_to_f16x2((w >> 8) & 0xffu), s2);
+        o.z = hmul2_f16(e2m1x2_to_f16x2((w >> 16) & 0xffu), s2);
+        o.w = hmul2_f16(e2m1x2_to_f16x2(w >> 24), s2);
+        const int unit = 4 * (j & 1) + (st ? uu1 : uu0);
+        *reinterpret_cast<uint4*>(vrow + ((unit ^ (r & 7)) << 4)) = o;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bars[B_VREADY + 2 * cp]);
+      mbar_arrive(&bars[B_VREADY + 2 * cp + 1]);
+    }
+  }
+  return ok;
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled operand layouts need 1 KiB alignment
@@ -199,7 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 
   if (tid == 0) {
     for (int j = 0; j < kChunks; ++j) {
-      mbar_init(&bars[B_VREADY + j], kGatherWarps);
+      mbar_init(&bars[B_VREADY + j], kGatherWarps + kSoftWarps);
       mbar_init(&bars[B_VFREE + j], 1);
     }
     for (int u = 0; u < 2; ++u) {
@@ -224,21 +301,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 
   if (warp >= kSoftWarps && warp < kMmaWarp) {
     // ------------------------------ gather + dequantize ------------------------------
-    // Gather warp g handles tile rows 32 g + 8 i + qd (i = 0..3, qd = lane / 4): the four
-    // lanes of a quad share a row, so one warp load covers the same 64-byte slice of eight
-    // rows (32 different rows per load would multiply the requests the SM has in flight,
-    // which every load/store instruction of the CTA then queues behind). Lane j = lane % 4
-    // holds, for chunk pair cp (dims [128 cp, +128) = code bytes [64 cp, +64)), the code
-    // bytes [64 cp + 16 j, +16): dims [128 cp + 32 j, +32), scale groups 8 cp + 2 j and + 1.
-    const int gw = warp - kSoftWarps;
-    const int qd = lane >> 2, j = lane & 3;
+    // Gather warp g loads and dequantizes tile rows 16 g + 8 i + lane / 4 (i = 0, 1); the
+    // softmax warps take rows 64 .. 127.
+    const int row0 = 16 * (warp - kSoftWarps);
+    const int qd = lane >> 2;
     const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
     const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
     griddep_wait();  // the index list comes from the preceding kernel on the stream
-    int32_t pos_next[4];
+    int32_t pos_next[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int je = e_begin + 32 * gw + 8 * i + qd;
+    for (int i = 0; i < 2; ++i) {
+      const int je = e_begin + row0 + 8 * i + qd;
       pos_next[i] = je < e_end ? idx[je] : -1;
     }
     for (int t = 0; t < n_tiles && !*s_abort; ++t) {
@@ -250,73 +323,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         if (lane == 0) fail_wait(p, s_abort);
         break;
       }
-      int32_t pos[4];
+      int32_t pos[2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         pos[i] = (pos_next[i] >= 0 && pos_next[i] < len) ? pos_next[i] : -1;
-        const int jn = e_begin + (t + 1) * kTile + 32 * gw + 8 * i + qd;  // one tile ahead
+        const int jn = e_begin + (t + 1) * kTile + row0 + 8 * i + qd;  // one tile ahead
         pos_next[i] = jn < e_end ? idx[jn] : -1;
       }
-      uint4 pk[4][4];  // [chunk pair][row]
-      uint2 s8[4];     // [row]: the row's scale bytes [8 j, +8) (those of chunk pair j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (pos[i] >= 0) {
-          const uint8_t* prow = packed_b + int64_t(pos[i]) * (kD / 2) + 16 * j;
-#pragma unroll
-          for (int cp = 0; cp < 4; ++cp) pk[cp][i] = ld_nc_v4(prow + 64 * cp);
-          s8[i] = ld_nc_v2(scales_b + int64_t(pos[i]) * (kD / kGroup) + 8 * j);
-        } else {
-#pragma unroll
-          for (int cp = 0; cp < 4; ++cp) pk[cp][i] = make_uint4(0, 0, 0, 0);
-          s8[i] = make_uint2(0, 0);
-        }
-      }
-      bool ok = true;  // (no break inside this fully unrolled loop: registers stay registers)
-#pragma unroll
-      for (int cp = 0; cp < 4; ++cp) {
-        if (ok && (!gather_wait(&bars[B_VFREE + 2 * cp], (t & 1) ^ 1) ||
-                   !gather_wait(&bars[B_VFREE + 2 * cp + 1], (t & 1) ^ 1))) {
-          if (lane == 0) fail_wait(p, s_abort);
-          ok = false;
-        }
-        if (!ok) continue;
-        const int jc = 2 * cp + (j >> 1);  // chunk of this lane's 32 dims
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 32 * gw + 8 * i + qd;
-          // scale bytes 8 cp + 2 j, + 1 of row r: held by quad lane cp, word j / 2
-          const uint32_t w0 = __shfl_sync(0xffffffffu, s8[i].x, 4 * qd + cp);
-          const uint32_t w1 = __shfl_sync(0xffffffffu, s8[i].y, 4 * qd + cp);
-          const uint32_t sw = ((j >> 1) ? w1 : w0) >> (16 * (j & 1));
-          const uint32_t sA = e4m3x2_to_f16x2(static_cast<uint16_t>((sw & 0xffu) * 0x101u));
-          const uint32_t sB = e4m3x2_to_f16x2(static_cast<uint16_t>(((sw >> 8) & 0xffu) * 0x101u));
-          const uint4 src = pk[cp][i];
-          uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + r * 128;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            // 8-dim unit uu of this lane's 32 dims; lanes j and j + 2 (same units, different
-            // chunks) go in a staggered order so that a store phase hits distinct banks
-            const bool st = (j & 2) != 0;
-            const int uu0 = k, uu1 = k ^ 2;
-            const uint32_t w = st ? (uu1 == 0 ? src.x : uu1 == 1 ? src.y : uu1 == 2 ? src.z : src.w)
-                                  : (uu0 == 0 ? src.x : uu0 == 1 ? src.y : uu0 == 2 ? src.z : src.w);
-            const uint32_t s2 = (st ? uu1 : uu0) < 2 ? sA : sB;
-            uint4 o;
-            o.x = hmul2_f16(e2m1x2_to_f16x2(w & 0xffu), s2);
-            o.y = hmul2_f16(e2m1x2_to_f16x2((w >> 8) & 0xffu), s2);
-            o.z = hmul2_f16(e2m1x2_to_f16x2((w >> 16) & 0xffu), s2);
-            o.w = hmul2_f16(e2m1x2_to_f16x2(w >> 24), s2);
-            const int unit = 4 * (j & 1) + (st ? uu1 : uu0);
-            *reinterpret_cast<uint4*>(vrow + ((unit ^ (r & 7)) << 4)) = o;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars[B_VREADY + 2 * cp]);
-          mbar_arrive(&bars[B_VREADY + 2 * cp + 1]);
-        }
+      if (!load_dequant<2>(smem, bars, packed_b, scales_b, pos, row0, t)) {
+        if (lane == 0) fail_wait(p, s_abort);
+        break;
       }
     }
   } else if (warp == kMmaWarp) {
@@ -452,6 +468,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     const uint32_t lane_addr = uint32_t(32 * q4) << 16;
     // bit t: this thread's entry of tile t holds a valid position (at most 32 tiles)
     griddep_wait();  // the index list comes from the preceding kernel on the stream
+    // this warp also loads and dequantizes tile rows 64 + 8 warp + lane / 4 of every tile
+    const int drow = 64 + 8 * warp;
+    const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
+    const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
+    auto dq_pos = [&](int tt) -> int32_t {
+      const int je = e_begin + tt * kTile + drow + (lane >> 2);
+      return (tt < n_tiles && je < e_end) ? idx[je] : -1;
+    };
+    int32_t dpos_next = dq_pos(0);
     uint32_t vmask = 0;
     for (int t0 = 0; t0 < n_tiles; t0 += 8) {
       int32_t pv[8];
@@ -468,6 +493,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
     for (int j = 0; j < 32; ++j) lsum[j] = 0.0f;
     bool fail = false;  // uniform across the softmax warps
+    bool dq_fail = false;  // this warp's share of the dequantization timed out
+    if (n_tiles > 0) {
+      int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
+      dpos_next = dq_pos(1);
+      dq_fail = !load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0);
+    }
     for (int t = 0; t < n_tiles; ++t) {
       const int u = t & 1;
       const bool valid = (vmask >> t) & 1u;
@@ -494,6 +525,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
         for (int j = 0; j < 32; ++j) z[j] = -INFINITY;
       }
+      f = f || dq_fail;
       if (softmax_any(over || f)) {
         if (softmax_any(f)) {
           fail = true;
@@ -565,6 +597,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PREADY]);
+      if (t + 1 < n_tiles) {  // this warp's rows of the next tile, as P.V(t) frees V_hat
+        int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
+        dpos_next = dq_pos(t + 2);
+        dq_fail = !load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1);
+      }
     }
     // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----
     if (!fail && n_tiles > 0) {

@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<FP8, N>::kCtasPerSm)
   uint32_t* s_tmem = s_hist_all + 2 * kEpiGroups * kHistBins;
   volatile uint32_t* s_abort = s_tmem + 1;
 
+  // the top-K select that follows may be scheduled as CTAs of this grid finish
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Tiles T;
   T.per_seq = tiles_per_seq;
@@ -153,6 +155,9 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<FP8, N>::kCtasPerSm)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // launched as a programmatic dependent: the prologue above overlapped the previous kernel
+  // on the stream; everything it wrote is visible past this point
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------- TMA producer ----------------------------------
@@ -463,7 +468,18 @@ cudaError_t launch_n(const IndexScoreParams& p, int num_sms, cudaStream_t stream
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Cfg::kSmem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cfg::kSmem, stream>>>(p, tk, tq, tiles_per_seq, total);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p, tk, tq, tiles_per_seq, total);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

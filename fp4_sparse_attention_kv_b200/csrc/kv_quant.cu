@@ -22,6 +22,7 @@
 // Memory: one warp per row, one 16-channel group per lane: 32 B read, 8 B + 1 B written per
 // lane; a warp reads 1 KiB and writes 256 B + 32 B contiguous.
 #include "fp4kv_common.cuh"
+#include "fp4kv_sm100.cuh"
 #include "fp4kv_launch.h"
 
 namespace fp4kv {
@@ -75,6 +76,9 @@ __global__ void __launch_bounds__(256) k_kv_quant_fp4(const uint16_t* __restrict
                                                       uint8_t* __restrict__ packed,
                                                       uint8_t* __restrict__ scales,
                                                       int64_t cap_rows) {
+  // the indexer scan that follows on the stream may start its prologue now (it waits for
+  // this grid before reading anything)
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);

@@ -245,6 +245,7 @@ __device__ void block_sort(T* s) {
 __global__ void __launch_bounds__(kSelThreads) k_select_filter(const SelectArgs args) {
   // the finishing kernel is a programmatic dependent: it may be scheduled from now on
   griddep_launch_dependents();
+  griddep_wait();  // this grid is one too: the scores and histograms are complete past here
   const SelectProblem& P = args.p[blockIdx.z];
   const int b = blockIdx.y, s = blockIdx.x;
   if (s >= P.slices) return;
@@ -558,22 +559,23 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
     if (probs[i].slices > gx) gx = probs[i].slices;
   }
   dim3 grid(gx, B, n_probs);
-  k_select_filter<<<grid, kSelThreads, 0, stream>>>(args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(k_select_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kFinSmem));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_select_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kFinSmem));
-  if (e != cudaSuccess) return e;
+  // both kernels are programmatic dependents of the kernel before them on the stream
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = kFinSmem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_select_filter, args);
+  if (e != cudaSuccess) return e;
+  cfg.dynamicSmemBytes = kFinSmem;
   e = cudaLaunchKernelEx(&cfg, k_select_finish, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
