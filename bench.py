@@ -238,8 +238,8 @@ class DecodeWorkload:
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
         self.inputs = [self.q, self.qi, self.w, self.x_new]
         self.outputs = [self.out, self.lse]
-        # quantize, scan, select, attention (+ the chunk combine when attention splits)
-        self.launches_per_step = 4 + attn_split(fk, B, cap, H, K)
+        # quantize, scan, select (filter + finish), attention (+ the chunk merge when split)
+        self.launches_per_step = 5 + attn_split(fk, B, cap, H, K)
         self.tokens_per_step = B
 
     def step(self):
@@ -297,7 +297,9 @@ class HierWorkload:
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
         self.inputs = self.q + self.qi + self.w + self.x_new
         self.outputs = self.out + self.lse
-        self.launches_per_step = L + 2 + (L // 2) * 2 + L * (1 + attn_split(fk, B, cap, H, K))
+        # per layer a quantize and an attention (+ merge); the Full layer and each Reindex layer
+        # add a scan and the two select kernels
+        self.launches_per_step = L + 3 + (L // 2) * 3 + L * (1 + attn_split(fk, B, cap, H, K))
         self.tokens_per_step = B
 
     def step(self):
