@@ -1,0 +1,70 @@
+"""Host-side logic of bench.py on the CPU: the multi-rank plumbing (gloo, two ranks) and the
+reference arm's output contract. No GPU is used."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    ws, r, _ = bench.dist_env()
+    dist = bench.init_dist(ws, "gloo")
+    bench.barrier(ws)
+    # each rank times a different duration: the job's time is the slowest rank's
+    got = bench.max_over_ranks(1.0 + 2.5 * r, ws)
+    bench.barrier(ws)
+    out[r] = got
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+        assert dict(out) == {0: 3.5, 1: 3.5}
+
+
+def test_max_over_ranks_is_identity_on_one_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(4.25, 1) == 4.25
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_prints_one_line_on_rank0_only():
+    """The reference arm (the oracle on the host cores) prints one JSON line on rank 0 and
+    exits 0 without work on the other ranks."""
+    outs = []
+    for rank in (0, 1):
+        env = dict(os.environ, WORLD_SIZE="2", RANK=str(rank), LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+        r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny",
+                            "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                           capture_output=True, text=True, timeout=280)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs.append([ln for ln in r.stdout.splitlines() if ln.strip()])
+    assert outs[1] == []
+    assert len(outs[0]) == 1
+    line = json.loads(outs[0][0])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak"
