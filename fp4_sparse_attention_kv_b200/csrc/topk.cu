@@ -99,17 +99,6 @@ FP4KV_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* s_wsum, uint32_t* total
   return excl;
 }
 
-// Copies a 4096-bin histogram from global memory into shared memory: 8 bins (two 16-byte
-// loads) per thread, all in flight at once.
-FP4KV_DEV void load_hist(uint32_t* s_dst, const uint32_t* g_src) {
-  static_assert(kHistBins == kSelThreads * 8, "8 bins per thread");
-  const uint4* src = reinterpret_cast<const uint4*>(g_src) + threadIdx.x * 2;
-  const uint4 a = __ldcg(src), c = __ldcg(src + 1);
-  uint4* dst = reinterpret_cast<uint4*>(s_dst) + threadIdx.x * 2;
-  dst[0] = a;
-  dst[1] = c;
-}
-
 // Block-wide: find the digit d (scanning from the highest digit down) at which the running
 // count of `h[0..nbins)` reaches `r` (r >= 1). Returns d and the count strictly above d.
 // If the total is below r, returns d = -1 and above = total.
@@ -162,6 +151,70 @@ __device__ void find_digit_desc(const uint32_t* h, int nbins, uint32_t r, int* d
   __syncthreads();
   *d_out = s_scan[64] == 0xffffffffu ? -1 : static_cast<int>(s_scan[64]);
   *above_out = s_scan[65];
+  __syncthreads();
+}
+
+// The same search over a 4096-bin histogram in global memory, read straight into registers:
+// thread t owns the 8 bins [4096 - 8 (t + 1), 4096 - 8 t) (two 16-byte loads), so no
+// shared-memory copy is made and the crossing thread finds the digit in its own registers.
+// Also returns the count of the found bin (0 if none).
+__device__ void find_digit_desc_g(const uint32_t* g_hist, uint32_t r, int* d_out, uint32_t* above_out,
+                                  uint32_t* count_out, uint32_t* s_scan) {
+  static_assert(kHistBins == kSelThreads * 8, "8 bins per thread");
+  const int tid = threadIdx.x;
+  const int lo = kHistBins - 8 * (tid + 1);
+  const uint4 a = __ldcg(reinterpret_cast<const uint4*>(g_hist + lo));
+  const uint4 c = __ldcg(reinterpret_cast<const uint4*>(g_hist + lo + 4));
+  const uint32_t h[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+  uint32_t sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum += h[i];
+  const int lane = tid & 31, w = tid >> 5;
+  uint32_t x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_scan[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    uint32_t v = lane < kSelWarps ? s_scan[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < kSelWarps) s_scan[32 + lane] = v;  // inclusive warp prefix
+    if (lane == 0) {
+      s_scan[64] = 0xffffffffu;  // digit
+      s_scan[65] = 0;            // count above it
+      s_scan[66] = 0;            // its count
+    }
+  }
+  __syncthreads();
+  const uint32_t incl = x + (w > 0 ? s_scan[32 + w - 1] : 0u);
+  const uint32_t excl = incl - sum;
+  const uint32_t total = s_scan[32 + kSelWarps - 1];
+  if (total < r) {
+    if (tid == 0) s_scan[65] = total;
+  } else if (excl < r && incl >= r) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      if (acc + h[i] >= r) {
+        s_scan[64] = static_cast<uint32_t>(lo + i);
+        s_scan[65] = acc;
+        s_scan[66] = h[i];
+        break;
+      }
+      acc += h[i];
+    }
+  }
+  __syncthreads();
+  *d_out = s_scan[64] == 0xffffffffu ? -1 : static_cast<int>(s_scan[64]);
+  *above_out = s_scan[65];
+  *count_out = s_scan[66];
   __syncthreads();
 }
 
@@ -263,23 +316,27 @@ __global__ void __launch_bounds__(kSelThreads) k_select_filter(const SelectArgs 
   uint64_t* list = P.list + int64_t(b) * P.vstride;
 
   // digit 1 of the K-th largest key (b1 = -1: fewer than K valid values, all are kept)
-  load_hist(s_h, P.hist + int64_t(b) * kHistBins);
-  __syncthreads();
-  int b1;
-  uint32_t above;
-  find_digit_desc(s_h, kHistBins, static_cast<uint32_t>(P.k), &b1, &above, s_scan);
   for (int i = tid; i < kHistBins; i += kSelThreads) s_h[i] = 0;
-  __syncthreads();
+  int b1;
+  uint32_t above, b1_count;
+  find_digit_desc_g(P.hist + int64_t(b) * kHistBins, static_cast<uint32_t>(P.k), &b1, &above, &b1_count, s_scan);
+  (void)above;
+  (void)b1_count;
 
   // keys with digit 1 >= b1, in position order, into list[lo ..)
   uint32_t run = 0, n_sure = 0;
+  // the next batch's values are loaded before this batch is classified and compacted
+  float4 na = make_float4(0.f, 0.f, 0.f, 0.f), nc = na;
+  if (lo + int64_t(tid) * kPer < hi) {  // a multiple of 8 below vstride (a multiple of 8)
+    na = __ldg(reinterpret_cast<const float4*>(vals + lo + int64_t(tid) * kPer));
+    nc = __ldg(reinterpret_cast<const float4*>(vals + lo + int64_t(tid) * kPer + 4));
+  }
   for (int64_t base = lo; base < hi; base += kBatchVals) {
     const int64_t i0 = base + int64_t(tid) * kPer;
-    float v[kPer];
-    if (i0 < hi) {  // i0 is a multiple of 8 and below vstride (a multiple of 4)
-      const float4 a = __ldg(reinterpret_cast<const float4*>(vals + i0));
-      const float4 c = __ldg(reinterpret_cast<const float4*>(vals + i0 + 4));
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+    const float v[kPer] = {na.x, na.y, na.z, na.w, nc.x, nc.y, nc.z, nc.w};
+    if (i0 + kBatchVals < hi) {
+      na = __ldg(reinterpret_cast<const float4*>(vals + i0 + kBatchVals));
+      nc = __ldg(reinterpret_cast<const float4*>(vals + i0 + kBatchVals + 4));
     }
     uint32_t keep = 0, keys[kPer];
 #pragma unroll
@@ -368,12 +425,12 @@ __global__ void __launch_bounds__(kSelThreads) k_select_finish(const SelectArgs 
   // digit 2 of the K-th key: b2 = -1 takes every key of the b1 bin; b2 = 4096 takes none
   int b2 = kHistBins;
   uint32_t above2 = 0, bin_count = 0;
-  if (r > 0 && b1 >= 0) {
-    load_hist(s_h, h2g);
-    __syncthreads();
-    find_digit_desc(s_h, kHistBins, r, &b2, &above2, s_scan);
-    if (b2 >= 0) bin_count = s_h[b2];
-    __syncthreads();
+  if (r > 0 && b1 >= 0) find_digit_desc_g(h2g, r, &b2, &above2, &bin_count, s_scan);
+  // the digit-1 histogram has been read by the filter grid (complete): zero this CTA's share
+  {
+    const int per_cta = (kHistBins + P.slices - 1) / P.slices;
+    uint32_t* h1 = P.hist + int64_t(b) * kHistBins;
+    for (int i = s * per_cta + tid; i < min(kHistBins, (s + 1) * per_cta); i += kSelThreads) h1[i] = 0;
   }
 
   // drop the keys of the b1 bin below b2 from this slice's list (in place, order kept)
@@ -420,9 +477,13 @@ __global__ void __launch_bounds__(kSelThreads) k_select_finish(const SelectArgs 
     __syncthreads();
   }
   const bool staged = total_kept <= static_cast<uint32_t>(kStage);
-  if (staged) {
-    for (uint32_t j = tid; j < total_kept; j += kSelThreads)
-      s_stage[j] = kept_entry(list, s_off, P.slices, per, j);
+  if (staged) {  // one warp per slice list
+    const int lane = tid & 31;
+    for (int sl = tid >> 5; sl < P.slices; sl += kSelWarps) {
+      const uint32_t o = s_off[sl], n_sl = s_off[sl + 1] - o;
+      const unsigned long long* src = reinterpret_cast<const unsigned long long*>(list) + per * sl;
+      for (uint32_t j = lane; j < n_sl; j += 32) s_stage[o + j] = __ldcg(src + j);
+    }
     __syncthreads();
   }
   auto entry = [&](uint32_t j) -> uint64_t {
@@ -530,11 +591,9 @@ __global__ void __launch_bounds__(kSelThreads) k_select_finish(const SelectArgs 
     oi[j] = -1;
     if (os) os[j] = -INFINITY;
   }
-  // leave the workspace zeroed for the next call
-  for (int i = tid; i < kHistBins; i += kSelThreads) {
-    P.hist[int64_t(b) * kHistBins + i] = 0;
-    h2g[i] = 0;
-  }
+  // leave the workspace zeroed for the next call (the digit-1 histogram was zeroed by all
+  // the finishing CTAs)
+  for (int i = tid; i < kHistBins; i += kSelThreads) h2g[i] = 0;
   if (tid < kSelCounters) ctr[tid] = 0;
 }
 
