@@ -627,21 +627,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         sA[h] = L > 0.0f ? (split ? 1.0f : 1.0f / (kPScale * L)) : 0.0f;
       }
       softmax_sync();
-      // O^T -> staging [64 heads][512 dims] fp32 in the V_hat region (rolled: runs once per CTA)
+      // O^T -> staging [64 heads][512 dims] fp32 in the V_hat region: one 32-column TMEM load
+      // (this thread's heads) per dim tile
       float* stage = reinterpret_cast<float*>(smem + kOffV);
 #pragma unroll 1
-      for (int cj = 0; cj < 16; ++cj) {
-        const int c = cj >> 2, j0 = h0 + 8 * (cj & 3);
-        uint32_t r[8];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
         if (n_tiles > 0) {
-          tmem_ld8(tmem + lane_addr + 64u * c + j0, r);
+          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) r[k] = 0u;
+          for (int k = 0; k < 32; ++k) r[k] = 0u;
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) stage[(j0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[j0 + k];
+        for (int k = 0; k < 32; ++k) stage[(h0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[h0 + k];
       }
       fence_proxy_async_smem();
       softmax_sync();
@@ -681,8 +681,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 }
 
 // Merge of the chunk partials (log-sum-exp combine). Grid (64 heads, head groups, B), 128
-// threads: the chunk weights 2^(m_c - M) are computed once into shared memory, then every
-// thread accumulates 4 of the 512 dims over the chunks, four chunks' loads in flight at once.
+// threads: every thread accumulates 4 of the 512 dims over the chunks; the first chunks'
+// rows are loaded while the weights 2^(m_c - M) are computed into shared memory.
 constexpr int kMaxChunks = 256;
 __global__ void __launch_bounds__(128) k_attn_combine(const AttnParams p, int n_hg) {
   __shared__ float s_w[kMaxChunks];
@@ -694,10 +694,17 @@ __global__ void __launch_bounds__(128) k_attn_combine(const AttnParams p, int n_
   if (hh >= nh) return;
   const int n_chunks = p.n_chunks;
   const int64_t base = (int64_t(b) * n_hg + hg) * n_chunks;
+  const float4* src = reinterpret_cast<const float4*>(p.part_o + (base * kHeadsPerCta + hh) * kD) + tid;
+  const int64_t cstride = int64_t(kHeadsPerCta) * kD / 4;  // float4s between chunks
+  // the first chunks' partial rows are loaded before the weights are known (independent)
+  constexpr int kPre = 8;
+  float4 v[kPre];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) v[u] = u < n_chunks ? __ldcg(src + u * cstride) : make_float4(0.f, 0.f, 0.f, 0.f);
   float mloc = -INFINITY;
   for (int c = tid; c < n_chunks; c += 128) {
-    const float mc = p.part_ml[((base + c) * kHeadsPerCta + hh) * 2];
-    const float lc = p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1];
+    const float mc = __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2]);
+    const float lc = __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1]);
     s_w[c] = lc > 0.0f ? mc : -INFINITY;
     if (lc > 0.0f) mloc = fmaxf(mloc, mc);
   }
@@ -711,31 +718,24 @@ __global__ void __launch_bounds__(128) k_attn_combine(const AttnParams p, int n_
     const float mc = s_w[c];
     const float w = mc == -INFINITY ? 0.0f : exp2f(mc - M);
     s_w[c] = w;
-    lsum += w * p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1];
+    lsum += w * __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
   if (lane == 0) s_red[1][warp] = lsum;
   __syncthreads();
   const float Lt = s_red[1][0] + s_red[1][1] + s_red[1][2] + s_red[1][3];
-  const float4* src = reinterpret_cast<const float4*>(p.part_o + (base * kHeadsPerCta + hh) * kD) + tid;
-  const int64_t cstride = int64_t(kHeadsPerCta) * kD / 4;  // float4s between chunks
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int c = 0;
-  for (; c + 4 <= n_chunks; c += 4) {
-    float4 v[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = src[(c + u) * cstride];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float w = s_w[c + u];
-      acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
-    }
+  for (int u = 0; u < kPre; ++u) {
+    if (u >= n_chunks) break;
+    const float w = s_w[u];
+    acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
   }
-  for (; c < n_chunks; ++c) {
-    const float4 v = src[c * cstride];
+  for (int c = kPre; c < n_chunks; ++c) {
+    const float4 x = __ldcg(src + c * cstride);
     const float w = s_w[c];
-    acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+    acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
   }
   const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
   float4* dst = reinterpret_cast<float4*>(p.out + (int64_t(b) * p.H + hg * kHeadsPerCta + hh) * kD) + tid;
