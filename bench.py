@@ -203,7 +203,40 @@ def attn_split(fk, B, cap, H, K) -> int:
     return 1 if fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K) > 256 else 0
 
 
-class DecodeWorkload:
+class TwoSets:
+    """Per-step inputs and outputs in two buffer sets, so that the end-to-end run can copy one
+    step's data while another step computes. `in_attrs` / `out_attrs` name the attributes
+    (tensors or lists of tensors) that hold them; `use_set(k)` rebinds them to set k."""
+
+    in_attrs: tuple = ()
+    out_attrs: tuple = ()
+
+    def _flat(self, names, k):
+        out = []
+        for a in names:
+            v = self._sets[k][a]
+            out.extend(v if isinstance(v, list) else [v])
+        return out
+
+    def make_second_set(self):
+        if getattr(self, "_sets", None) is not None:
+            return
+        first = {a: getattr(self, a) for a in self.in_attrs + self.out_attrs}
+        second = {a: ([t.clone() for t in v] if isinstance(v, list) else v.clone()) for a, v in first.items()}
+        self._sets = [first, second]
+
+    def use_set(self, k):
+        for a, v in self._sets[k].items():
+            setattr(self, a, v)
+
+    def inputs_of(self, k):
+        return self._flat(self.in_attrs, k)
+
+    def outputs_of(self, k):
+        return self._flat(self.out_attrs, k)
+
+
+class DecodeWorkload(TwoSets):
     """Tiny / decode32 / long: one decoder layer per step (write the new row, Full-mode
     indexer top-K over the whole cache, attention over the selected rows)."""
 
@@ -238,6 +271,7 @@ class DecodeWorkload:
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
         self.inputs = [self.q, self.qi, self.w, self.x_new]
         self.outputs = [self.out, self.lse]
+        self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
         # quantize, scan, select (filter + finish), attention (+ the chunk merge when split)
         self.launches_per_step = 5 + attn_split(fk, B, cap, H, K)
         self.tokens_per_step = B
@@ -256,7 +290,7 @@ class DecodeWorkload:
                 "kv_quant_fp4": self.B * (2 * D + ROW_BYTES)}
 
 
-class HierWorkload:
+class HierWorkload(TwoSets):
     """Hierarchical: 20 layers per step. Layer 1 (Full): hier_pool_select over all entries
     -> top-K + pool; layers 2, 4, .., 20 (Reindex): own indexer query scored inside the pool
     over layer 1's keys; layers 3, 5, .., 19 (Reuse): the previous layer's indices. Every
@@ -297,6 +331,7 @@ class HierWorkload:
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
         self.inputs = self.q + self.qi + self.w + self.x_new
         self.outputs = self.out + self.lse
+        self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
         # per layer a quantize and an attention (+ merge); the Full layer and each Reindex layer
         # add a scan and the two select kernels
         self.launches_per_step = L + 3 + (L // 2) * 3 + L * (1 + attn_split(fk, B, cap, H, K))
@@ -328,7 +363,7 @@ class HierWorkload:
                 "kv_quant_fp4": L * B * (2 * D + ROW_BYTES)}
 
 
-class QuantWorkload:
+class QuantWorkload(TwoSets):
     """Quantize-on-write sweep: 131,072 tokens x 20 layers of bf16 rows -> FP4 + scales."""
 
     def __init__(self, cfg, fk, device, rank=0):
@@ -346,6 +381,7 @@ class QuantWorkload:
         self.n = n
         self.inputs = [self.x]
         self.outputs = [self.packed, self.scales]
+        self.in_attrs, self.out_attrs = ("x",), ("packed", "scales")
         self.launches_per_step = 1
         self.tokens_per_step = cfg["tokens"]
 
@@ -398,30 +434,54 @@ def timed_steps(wl, steps, warmup, flush, sampler, fk):
 
 
 def e2e_steps(wl, steps, warmup):
-    """Same step through the public API with host buffers: the per-step inputs are copied
-    from pinned host memory and the outputs read back inside the timed region."""
-    h_in = [t.detach().cpu().pin_memory() for t in wl.inputs]
-    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.outputs]
-    s = torch.cuda.current_stream()
+    """Same step through the public API with host buffers: every step copies its inputs from
+    pinned host memory and reads its outputs back inside the timed region. As in a serving
+    loop, the copies run on an upload and a download stream against two buffer sets, so step
+    i's inputs travel while step i - 1 computes and its outputs while step i + 1 computes;
+    events order each set's upload, compute and read-back."""
+    wl.make_second_set()
+    dev = wl.inputs_of(0)[0].device
+    h_in = [t.detach().cpu().pin_memory() for t in wl.inputs_of(0)]
+    h_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.outputs_of(0)] for _ in range(2)]
+    torch.cuda.synchronize()
+    # non-blocking streams of their own (no implicit ordering with the legacy default stream)
+    comp, up, down = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for h, d in zip(h_in, wl.inputs):
-            d.copy_(h, non_blocking=True)
-        wl.step()
-        for h, d in zip(h_out, wl.outputs):
-            h.copy_(d, non_blocking=True)
+    def run(n):
+        for i in range(n):
+            k = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev_free[k])  # set k's previous step has been read back
+                for h, d in zip(h_in, wl.inputs_of(k)):
+                    d.copy_(h, non_blocking=True)
+                ev_up[k].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(ev_up[k])
+                wl.use_set(k)
+                wl.step()  # the library enqueues on the current stream
+                ev_comp[k].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_comp[k])
+                for h, d in zip(h_out[k], wl.outputs_of(k)):
+                    h.copy_(d, non_blocking=True)
+                ev_free[k].record(down)
 
-    for _ in range(max(1, warmup)):
-        one()
+    run(max(2, warmup))
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(s)
-    for _ in range(steps):
-        one()
-    b.record(s)
+    a.record(up)
+    run(steps)
+    down.wait_stream(up)
+    down.wait_stream(comp)
+    b.record(down)
     torch.cuda.synchronize()
-    h2d = sum(t.numel() * t.element_size() for t in wl.inputs)
-    d2h = sum(t.numel() * t.element_size() for t in wl.outputs)
+    wl.use_set(0)
+    h2d = sum(t.numel() * t.element_size() for t in wl.inputs_of(0))
+    d2h = sum(t.numel() * t.element_size() for t in wl.outputs_of(0))
     return a.elapsed_time(b), h2d, d2h
 
 
