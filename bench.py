@@ -232,6 +232,40 @@ class TwoSets:
     def inputs_of(self, k):
         return self._flat(self.in_attrs, k)
 
+    graphs = None
+
+    def capture_graphs(self):
+        """Capture one step per buffer set in a CUDA graph (the library enqueues on the
+        current stream and allocates nothing, so a step is capturable); on any failure the
+        steps stay eager."""
+        self.make_second_set()
+        try:
+            gs = []
+            for k in range(2):
+                self.use_set(k)
+                cs = torch.cuda.Stream()
+                cs.wait_stream(torch.cuda.current_stream())
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cs, capture_error_mode="relaxed"):
+                    self.step()
+                torch.cuda.current_stream().wait_stream(cs)
+                gs.append(g)
+            torch.cuda.synchronize()
+            self.graphs = gs
+        except Exception as e:  # noqa: BLE001 - any capture failure falls back to eager steps
+            phase(f"graph capture failed, eager steps: {e}")
+            self.graphs = None
+        self.use_set(0)
+
+    def run_step(self, k=0):
+        """One step on buffer set k: a graph replay when captured, else eager launches."""
+        if getattr(self, "_sets", None) is not None:
+            self.use_set(k)
+        if self.graphs is not None:
+            self.graphs[k].replay()
+        else:
+            self.step()
+
     def outputs_of(self, k):
         return self._flat(self.out_attrs, k)
 
@@ -407,17 +441,20 @@ def timed_steps(wl, steps, warmup, flush, sampler, fk):
     dependent of the first, so they stay out of the headline timing."""
     s = torch.cuda.current_stream()
     for _ in range(warmup):
-        wl.step()
+        wl.run_step(0)
     torch.cuda.synchronize()
 
-    def run(n):
+    def run(n, prof_pass=False):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(n)]
         for a, b in evs:
             if flush is not None:
                 flush.zero_()
             a.record(s)
-            wl.step()
+            if prof_pass:
+                wl.step()  # eager: the library records its per-launch events as it launches
+            else:
+                wl.run_step(0)
             b.record(s)
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in evs)
@@ -426,7 +463,7 @@ def timed_steps(wl, steps, warmup, flush, sampler, fk):
     total_ms = run(steps)
     fk.profile_read()  # drop earlier records
     fk.profile_enable(True)
-    run(steps)
+    run(steps, prof_pass=True)
     fk.profile_enable(False)
     sampler.stop()
     prof = fk.profile_read()
@@ -461,8 +498,7 @@ def e2e_steps(wl, steps, warmup):
                 ev_up[k].record(up)
             with torch.cuda.stream(comp):
                 comp.wait_event(ev_up[k])
-                wl.use_set(k)
-                wl.step()  # the library enqueues on the current stream
+                wl.run_step(k)  # the library enqueues on the current stream
                 ev_comp[k].record(comp)
             with torch.cuda.stream(down):
                 down.wait_event(ev_comp[k])
@@ -603,6 +639,8 @@ def main(argv=None):
     ap.add_argument("--config", default="decode32", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch each step eagerly instead of "
+                    "replaying a captured CUDA graph")
     args = ap.parse_args(argv)
     cfg_name, cfg = args.config, CONFIGS[args.config]
     if args.impl == "reference":
@@ -637,6 +675,12 @@ def main(argv=None):
         flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
         l2_note = "flushed (256 MiB write) before every timed step"
     torch.cuda.synchronize()
+    for _ in range(2):  # the library's first launches set kernel attributes
+        wl.step()
+    torch.cuda.synchronize()
+    if not args.no_graph:
+        phase("graph capture")
+        wl.capture_graphs()
 
     phase("clock sampler")
     sampler = ClockSampler(local)
@@ -682,6 +726,8 @@ def main(argv=None):
             "config": {"workload": cfg["workload"], "name": cfg_name,
                        "l2": l2_note,
                        "parallelism": f"dp{world} (independent sequences per GPU)",
+                       "launch": ("one CUDA graph replay per step" if wl.graphs is not None
+                                  else "eager launches"),
                        "tokens_per_step": tokens},
             "hbm_gbs_step": step_bytes * world / (step_ms * 1e-3) / 1e9,
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
