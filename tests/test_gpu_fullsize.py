@@ -1,0 +1,111 @@
+"""Parity at the full workload sizes, in the launch configuration the bench times.
+
+bench.py's own workload classes build the data (the whole cache, quantized by the library)
+and run one step exactly as the bench does; sampled sequences are then checked against the
+oracle. The oracle regenerates every input it needs from the seeded generator (the FP4 rows
+it attends over are quantized by the oracle itself, never read back from the GPU cache), so
+nothing it consumes comes from the CUDA path except the selections whose consumers are
+being checked (the attention is checked over the GPU's indices; the Reindex layer over the
+GPU's pool), each of which is itself checked against the oracle first.
+"""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import fp4kv_oracle as O
+from tests import parity as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+D = 512
+
+
+@pytest.fixture(scope="module")
+def fk(cuda_lib):
+    import fp4_sparse_attention_kv_b200 as fk
+    return fk
+
+
+def _attn_check(seed, layer, b, q_b, idx_b, seq_len, new_row, out_b, lse_b, what):
+    """Oracle attention of one sequence over the given selection; rows regenerated on the
+    host and quantized by the oracle; row seq_len - 1 is the row the step wrote."""
+    sel = np.asarray(idx_b, dtype=np.int64)
+    sel = sel[(sel >= 0) & (sel < seq_len)]
+    rows = P.kv_rows_host(seed, layer, b, sel, D)
+    last = sel == seq_len - 1
+    if last.any():
+        rows[last] = new_row
+    pk, sc = O.kv_quant_fp4(rows)
+    ro, rl = O.sparse_attn_decode_rows(P.to_f64(q_b.cpu()), O.kv_dequant_fp4(pk, sc), 1.0)
+    P.check_attn(out_b, lse_b, ro, rl, what)
+
+
+def _new_row_check(wl, b, layer_packed, layer_scales, x_new, what):
+    pk, sc = O.kv_quant_fp4(P.to_f64(x_new[b:b + 1].cpu()))
+    assert np.array_equal(layer_packed[b, wl.cap - 1].cpu().numpy(), pk[0]), what
+    assert np.array_equal(layer_scales[b, wl.cap - 1].cpu().numpy(), sc[0]), what
+
+
+@pytest.mark.timeout(900)
+@pytest.mark.parametrize("name,seqs", [("decode32", (0, 17, 31)), ("long", (0, 3))])
+def test_decode_step_at_full_size(fk, name, seqs):
+    cfg = bench.CONFIGS[name]
+    wl = bench.DecodeWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    idx = wl.idx.cpu().numpy()
+    out, lse = wl.out.cpu().numpy(), wl.lse.cpu().numpy()
+    seed = cfg["seed"]
+    for b in seqs:
+        sc = P.oracle_scores_seq(wl.qi[b], wl.w[b], wl.keys[b], wl.cap)
+        P.check_topk(idx[b], sc, np.arange(wl.cap), wl.K, f"{name} top-K b={b}")
+        new_row = P.to_f64(wl.x_new[b].cpu())
+        _attn_check(seed, 0, b, wl.q[b], idx[b], wl.cap, new_row, out[b], lse[b], f"{name} attention b={b}")
+        _new_row_check(wl, b, wl.packed, wl.scales, wl.x_new, f"{name} new row b={b}")
+
+
+@pytest.mark.timeout(1200)
+def test_hierarchical_step_at_full_size(fk):
+    cfg = bench.CONFIGS["hier"]
+    wl = bench.HierWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    seed, b, cap, K, npb = cfg["seed"], 0, wl.cap, wl.K, wl.npb
+    # layer 1 (Full): flat top-K and the pool of the best blocks
+    sc = P.oracle_scores_seq(wl.qi[0][b], wl.w[0][b], wl.keys[b], cap)
+    P.check_topk(wl.idx[0][b].cpu().numpy(), sc, np.arange(cap), K, "Full top-K")
+    bm = O.block_max(sc, cap, 8)
+    pool = wl.pool[b].cpu().numpy()
+    P.check_topk(pool, bm, np.arange(bm.size), npb, "pool")
+    # layer 2 (Reindex): this layer's query scored inside the pool
+    pos = O.pool_positions(pool, cap, 8)
+    sc2 = P.oracle_scores_seq(wl.qi[1][b], wl.w[1][b], wl.keys[b], cap)[pos]
+    idx1 = wl.idx[1][b].cpu().numpy()
+    P.check_topk(idx1, sc2, pos, K, "Reindex top-K")
+    # attention of layers 1, 2 (over their own indices) and 3 (Reuse: layer 2's indices)
+    for layer, sel in ((0, wl.idx[0][b]), (1, wl.idx[1][b]), (2, wl.idx[1][b])):
+        new_row = P.to_f64(wl.x_new[layer][b].cpu())
+        _attn_check(seed, layer, b, wl.q[layer][b], sel.cpu().numpy(), cap, new_row,
+                    wl.out[layer][b].cpu().numpy(), wl.lse[layer][b].cpu().numpy(),
+                    f"hier layer {layer + 1} attention")
+        _new_row_check(wl, b, wl.packed[layer], wl.scales[layer], wl.x_new[layer], f"hier layer {layer + 1} new row")
+
+
+@pytest.mark.timeout(900)
+def test_quant_sweep_at_full_size_sampled_rows(fk):
+    cfg = bench.CONFIGS["quant"]
+    wl = bench.QuantWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(wl.n, size=4096, replace=False))
+    rows_t = torch.as_tensor(rows, device="cuda")
+    pk, sc = O.kv_quant_fp4(P.to_f64(wl.x[rows_t].cpu()))
+    assert np.array_equal(wl.packed[rows_t].cpu().numpy(), pk)
+    assert np.array_equal(wl.scales[rows_t].cpu().numpy(), sc)
