@@ -45,6 +45,7 @@ SIGNATURES = [
      [_P, _P, _I32, _P, _I32, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _P, _P, _P]),
     ("fp4kv_profile_enable", ctypes.c_int, [_I32]),
     ("fp4kv_profile_read", ctypes.c_int, [ctypes.POINTER(_I32), ctypes.POINTER(_F32)]),
+    ("fp4kv_selftest_wait_timeout", ctypes.c_int, [_I32, _P, _SZ, _P]),
 ]
 
 KERNEL_KINDS = ("kv_quant_fp4", "index_score", "topk_select", "sparse_attn")
@@ -135,6 +136,12 @@ def workspace_status(ws: torch.Tensor) -> int:
     if st not in (0, 5):
         _check(st)
     return int(out.value)
+
+
+def selftest_wait_timeout(limit_us: int, ws: torch.Tensor):
+    """Test hook: a kernel waits on a barrier nothing signals, bounded by limit_us; the
+    timeout lands in ws's status word (read it with workspace_status)."""
+    _check(lib().fp4kv_selftest_wait_timeout(int(limit_us), _ptr(ws), ws.numel(), _stream(ws.device)))
 
 
 def kv_quant_fp4(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,

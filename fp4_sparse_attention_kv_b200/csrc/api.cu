@@ -12,6 +12,7 @@
 #include "fp4kv.h"
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
+#include "fp4kv_sm100.cuh"
 
 namespace {
 
@@ -206,6 +207,24 @@ fp4kv::IndexScoreParams score_params(const void* q, const float* w, int32_t H_I,
 
 }  // namespace
 
+// Test hook: waits on an mbarrier that nothing ever signals, bounded by limit_ns, then
+// reports the timeout in the status word exactly as the library's kernels do.
+__global__ void k_selftest_wait(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    fp4kv::mbar_init(&bar, 1);
+    fp4kv::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = fp4kv::globaltimer_ns();
+    bool done = false;
+    while (!(done = fp4kv::mbar_try_wait(&bar, 0)) && fp4kv::globaltimer_ns() - t0 <= limit_ns) {
+    }
+    if (!done) atomicOr(status, fp4kv::kFlagWaitTimeout);
+  }
+}
+
 extern "C" {
 
 const char* fp4kv_last_error(void) { return g_last_error.c_str(); }
@@ -239,6 +258,18 @@ fp4kv_status fp4kv_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws_bytes == 0) return ok();
   cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "workspace_init");
+  return ok();
+}
+
+fp4kv_status fp4kv_selftest_wait_timeout(int32_t limit_us, void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return fail(FP4KV_ERR_INVALID_ARG, "null workspace");
+  if (ws_bytes < kAlign) return fail(FP4KV_ERR_INVALID_ARG, "ws_bytes %zu < %zu", ws_bytes, kAlign);
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(FP4KV_ERR_INVALID_ARG, "limit_us=%d outside [1, 1000000]", limit_us);
+  k_selftest_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(ws),
+                                                                    uint64_t(limit_us) * 1000u);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_timeout");
   return ok();
 }
 

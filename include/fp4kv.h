@@ -104,6 +104,16 @@ fp4kv_status fp4kv_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * and synchronises `stream`; then clears the word. For tests and diagnostics. */
 fp4kv_status fp4kv_workspace_status(void* ws, uint32_t* host_status, void* stream);
 
+/* selftest_wait_timeout -- (The pages have no counterpart: a test hook.) Launches one
+ * small kernel that waits on an mbarrier nothing ever signals, bounded by limit_us
+ * microseconds (1 .. 1,000,000), so that the bounded-wait error path every kernel of the
+ * library uses can be exercised without faulting the device: when the bound runs out the
+ * kernel sets bit 0 of the workspace status word and returns, leaving the context usable.
+ * Read the word with fp4kv_workspace_status (which then returns FP4KV_ERR_DEVICE_FLAG).
+ * ws: any workspace of at least 256 bytes (only its status word is touched).
+ * INVALID_ARG for a null ws, a smaller ws_bytes or limit_us outside the range. */
+fp4kv_status fp4kv_selftest_wait_timeout(int32_t limit_us, void* ws, size_t ws_bytes, void* stream);
+
 /* kv_quant_fp4 -- quantize-on-write ([PyTorchKR] FP4 KV section).
  * x        : bf16 rows [n_rows][x_row_stride] (uint16 bits); d channels used per row.
  *            16-byte aligned, x_row_stride a multiple of 8.

@@ -353,3 +353,28 @@ def test_workspace_is_left_clean_and_status_zero(fk):
     b = fk.indexer_topk(q, w, keys, lens, k, ws=ws)
     assert torch.equal(a, b)
     assert fk.workspace_status(ws) == 0
+
+
+def test_bounded_wait_reports_a_timeout_and_the_context_stays_usable(fk):
+    """Failure detection without a device fault: a kernel waits on a barrier that nothing
+    signals, gives up after 20 ms, sets the workspace's wait-timeout bit and returns; the
+    host reads the bit, and the same context then quantizes bit-exactly."""
+    ws = fk.alloc_workspace(256, DEV)
+    fk.selftest_wait_timeout(20000, ws)
+    assert fk.workspace_status(ws) == 1
+    assert fk.workspace_status(ws) == 0  # reading clears the word
+    x = P.kv_rows_dev(17, 0, 1, 64, 512, torch.device(DEV))[0]
+    packed = torch.empty((64, 256), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((64, 32), dtype=torch.uint8, device=DEV)
+    fk.kv_quant_fp4(x, packed, scales)
+    pk, sc = O.kv_quant_fp4(P.to_f64(x.cpu()))
+    assert np.array_equal(packed.cpu().numpy(), pk)
+    assert np.array_equal(scales.cpu().numpy(), sc)
+
+
+def test_selftest_hook_rejects_bad_arguments(fk):
+    ws = fk.alloc_workspace(256, DEV)
+    for bad in (0, -5, 1000001):
+        with pytest.raises(fk.Fp4kvError):
+            fk.selftest_wait_timeout(bad, ws)
+    assert fk.workspace_status(ws) == 0
