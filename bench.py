@@ -5,10 +5,12 @@ One step = one decode pass of the hot path for a batch of sequences, on inputs a
 resident in HBM: quantize-on-write of the new token's KV row, the indexer scan with exact
 top-K, and sparse attention over the selected rows. The hierarchical configuration runs a
 20-layer step (one Full layer that also selects the candidate pool, Reindex layers inside
-the pool, Reuse layers on the previous indices). Prints ONE JSON line (rank 0).
+the pool, Reuse layers on the previous indices); the CSA2 decoder configuration runs the
+pages' own 20-layer schedule (groups of 4 over one shared KV, top-K 512, pool of 2048
+blocks). Prints ONE JSON line (rank 0).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode32|long|hier|
-       tiny|quant] [--impl ours|reference]
+       csa2_decoder|tiny|quant] [--impl ours|reference]
 Under torchrun (N > 1) each rank runs the same per-GPU workload on its own GPU (weak
 scaling; the path has no exchange step, so there is no collective in the data path); the
 step time is the max over ranks.
@@ -53,6 +55,14 @@ CONFIGS = {
                  workload="hierarchical batch 8 x 1,048,576 entries, 20 layers: Full + pool of "
                           "1024 blocks x 8, then Reindex / Reuse alternating, own FP4 KV per "
                           "layer, top-K 2048"),
+    # the decoder schedule of the pages' CSA2 section: 20 layers in 5 groups of 4; the first
+    # group is Full + 3 Reuse, the others Reindex + 3 Reuse; every layer reads the one main
+    # KV and the one set of indexer keys the Full layer owns
+    "csa2_decoder": dict(B=8, cap=1 << 20, H=64, H_I=32, K=512, fp8=True, seed=5, layers=20,
+                         npb=2048, group=4,
+                         workload="CSA2 decoder schedule batch 8 x 1,048,576 entries, 20 layers "
+                                  "in groups of 4 (Full or Reindex, then 3 Reuse) over one shared "
+                                  "FP4 KV and indexer key set, pool of 2048 blocks x 8, top-K 512"),
     "tiny": dict(B=1, cap=4096, H=16, H_I=32, K=256, fp8=False, seed=0,
                  workload="tiny batch 1 x 4096 entries, 16 heads, bf16 indexer keys, top-K 256"),
     "quant": dict(tokens=131072, layers=20, seed=4,
@@ -179,6 +189,23 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense 16-bit tensor-core peak in TFLOP/s: the measured bf16 GEMM burst figure (fp16,
+    which the attention's MMAs use, has the same nominal rate)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured (bf16 burst)"
+    return 1590.0, "fallback"
+
+
+def attn_flops_per_row(H: int) -> int:
+    """Algorithmic flops of the attention per selected row and sequence: q.k and p*v over
+    d channels for each of the H heads (2 flops per multiply-add, twice)."""
+    return 4 * H * D
 
 
 def traffic_record(kernel: str, workload: str):
@@ -397,6 +424,76 @@ class HierWorkload(TwoSets):
                 "kv_quant_fp4": L * B * (2 * D + ROW_BYTES)}
 
 
+class Csa2DecoderWorkload(TwoSets):
+    """The decoder schedule of the pages' CSA2 section: 20 layers in groups of 4. Layer 1
+    (Full) scores every entry -> top-K + candidate pool and is the only layer that writes a
+    KV row; the first layer of every later group (Reindex) re-scores inside the pool with
+    its own indexer query; the other layers (Reuse) take their group's indices. Every layer
+    attends with its own query over the one shared FP4 KV."""
+
+    def __init__(self, cfg, fk, device, rank=0):
+        self.cfg, self.fk, self.dev = cfg, fk, device
+        B, cap, H, H_I, K, L, npb, G = (cfg["B"], cfg["cap"], cfg["H"], cfg["H_I"], cfg["K"],
+                                         cfg["layers"], cfg["npb"], cfg["group"])
+        seed = cfg["seed"] + 1000 * rank
+        self.B, self.cap, self.H, self.H_I, self.K, self.L, self.npb, self.G = B, cap, H, H_I, K, L, npb, G
+        n_src = (L + G - 1) // G
+        self.packed = torch.empty((B, cap, D // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((B, cap, D // 16), dtype=torch.uint8, device=device)
+        self.keys = torch.empty((B, cap, DK), dtype=torch.uint8, device=device)
+        chunk = 1 << 18
+        for b in range(B):
+            for r0 in range(0, cap, chunk):
+                rows = torch.arange(r0, min(cap, r0 + chunk), dtype=torch.int64, device=device)
+                self.keys[b, r0:r0 + rows.numel()] = synth.indexer_keys(seed, b, rows, DK, True)
+                fk.kv_quant_fp4(synth.kv_rows(seed, 0, b, rows, D), self.packed[b, r0:r0 + rows.numel()],
+                                self.scales[b, r0:r0 + rows.numel()])
+        self.q = [synth.attn_query(seed, l, B, H, D, device=device) for l in range(L)]
+        # one indexer query per group (the group's Full or Reindex layer)
+        qw = [synth.indexer_query(seed, g * G, B, H_I, fp8=True, device=device) for g in range(n_src)]
+        self.qi = [a for a, _ in qw]
+        self.w = [b_ for _, b_ in qw]
+        self.x_new = synth.kv_rows(seed, 0, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
+        self.dst = torch.arange(B, dtype=torch.int64, device=device) * cap + (cap - 1)
+        self.lens = torch.full((B,), cap, dtype=torch.int32, device=device)
+        self.idx = [torch.empty((B, K), dtype=torch.int32, device=device) for _ in range(n_src)]
+        self.pool = torch.empty((B, npb), dtype=torch.int32, device=device)
+        self.out = [torch.empty((B, H, D), dtype=torch.float32, device=device) for _ in range(L)]
+        self.lse = [torch.empty((B, H), dtype=torch.float32, device=device) for _ in range(L)]
+        self.ws_h = fk.alloc_workspace(fk.workspace_bytes(fk.OP_HIER_POOL_SELECT, B, cap, H_I, K, npb), device)
+        self.ws_r = fk.alloc_workspace(fk.workspace_bytes(fk.OP_REINDEX_TOPK, B, cap, H_I, K, npb), device)
+        self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
+        self.inputs = self.q + self.qi + self.w + [self.x_new]
+        self.outputs = self.out + self.lse
+        self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
+        # one quantize; a scan and the two select kernels per group; an attention (+ merge)
+        # per layer
+        self.launches_per_step = 1 + 3 * n_src + L * (1 + attn_split(fk, B, cap, H, K))
+        self.tokens_per_step = B
+
+    def step(self):
+        fk, G = self.fk, self.G
+        fk.kv_quant_fp4(self.x_new, self.packed.view(-1, D // 2), self.scales.view(-1, D // 16),
+                        dst_row=self.dst)
+        for l in range(self.L):
+            g = l // G
+            if l == 0:
+                fk.hier_pool_select(self.qi[0], self.w[0], self.keys, self.lens, self.K, self.npb,
+                                    ws=self.ws_h, out_idx=self.idx[0], out_pool=self.pool)
+            elif l % G == 0:
+                fk.indexer_topk(self.qi[g], self.w[g], self.keys, self.lens, self.K, pool=self.pool,
+                                ws=self.ws_r, out_idx=self.idx[g])
+            fk.sparse_attn_decode(self.q[l], self.packed, self.scales, self.lens, self.idx[g], 1.0,
+                                  ws=self.ws_a, out=self.out[l], lse=self.lse[l])
+
+    def algorithmic_bytes(self):
+        B, L, G = self.B, self.L, self.G
+        n_reindex = (L + G - 1) // G - 1
+        return {"index_score": B * self.cap * DK + n_reindex * B * self.npb * 8 * DK,
+                "sparse_attn": L * B * self.K * ROW_BYTES,
+                "kv_quant_fp4": B * (2 * D + ROW_BYTES)}
+
+
 class QuantWorkload(TwoSets):
     """Quantize-on-write sweep: 131,072 tokens x 20 layers of bf16 rows -> FP4 + scales."""
 
@@ -573,20 +670,18 @@ def cpu_baseline(cfg_name, cfg, budget_s=12.0):
         gbs = rows * (2 * D + ROW_BYTES) / el / 1e9
         return {"value": gbs, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
                 "sample": f"{rows} rows of the quant sweep in {el:.1f} s"}
-    if cfg_name == "hier":
-        # one sequence's Full layer (scan + top-K + pool + attention) stands for the step's
-        # dominant work; the 19 pool-bounded layers are not sampled
-        from oracle import fp4kv_oracle as O  # noqa: F401
+    # layered configurations: one sequence's Full layer (scan + top-K + attention) stands for
+    # the step's dominant work; the 19 pool-bounded layers are not sampled
     seqs = 0
     while time.perf_counter() - t0 < budget_s or seqs == 0:
         oracle_sample_decode(cfg, seqs % cfg["B"])
         seqs += 1
     el = time.perf_counter() - t0
     layers = cfg.get("layers", 1)
-    return {"value": seqs / el / (layers if cfg_name == "hier" else 1), "unit": "tokens/s",
+    return {"value": seqs / el / layers, "unit": "tokens/s",
             "cores": oracle_threads(), "kind": "oracle",
             "sample": f"{seqs} of {cfg['B']} sequences (whole decode step per sequence"
-                      f"{', layer 1 only, scaled by 1/20' if cfg_name == 'hier' else ''}) in {el:.1f} s"}
+                      f"{f', layer 1 only, scaled by 1/{layers}' if layers > 1 else ''}) in {el:.1f} s"}
 
 
 # ----------------------------------------------------------------------------------------
@@ -609,7 +704,7 @@ def run_reference(args, cfg_name, cfg):
             work += 1
     el = time.perf_counter() - t0
     value = work / el
-    if cfg_name == "hier":
+    if "layers" in cfg:
         value /= cfg["layers"]
     cores = oracle_threads()
     sample = ("2048 rows per step" if cfg_name == "quant" else
@@ -664,6 +759,8 @@ def main(argv=None):
         wl = QuantWorkload(cfg, fk, device, rank)
     elif cfg_name == "hier":
         wl = HierWorkload(cfg, fk, device, rank)
+    elif cfg_name == "csa2_decoder":
+        wl = Csa2DecoderWorkload(cfg, fk, device, rank)
     else:
         wl = DecodeWorkload(cfg, fk, device, rank)
     streamed = sum(wl.algorithmic_bytes().values())
@@ -709,7 +806,21 @@ def main(argv=None):
     n_l, ms_l = prof[dom]
     per_launch_ms = ms_l / max(1, n_l)
     bytes_per_launch = alg[dom] / max(1, n_l / args.steps)
-    achieved = bytes_per_launch / (per_launch_ms * 1e-3) / 1e9
+    if dom == "sparse_attn":
+        # 4*H*d flops per gathered row of 288 bytes (455 flop/B at H = 64) is above the
+        # ridge point of the measured peaks: the attention is bound by the tensor cores
+        flops_per_launch = bytes_per_launch / ROW_BYTES * attn_flops_per_row(wl.H)
+        tpeak, tpeak_kind = measured_tensor_peak()
+        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": tpeak,
+                "unit": "TFLOP/s", "frac": achieved / tpeak, "peak_kind": tpeak_kind,
+                "algorithmic_flops_per_launch": flops_per_launch}
+    else:
+        achieved = bytes_per_launch / (per_launch_ms * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind}
+    roof.update({"traffic": traffic_record(dom, cfg_name),
+                 "algorithmic_bytes_per_launch": bytes_per_launch, "ms_per_launch": per_launch_ms})
     step_bytes = sum(v for k, v in alg.items())
     kernels = {k: {"launches_per_step": n / args.steps, "ms_per_step": t / args.steps,
                    "algorithmic_bytes_per_step": alg.get(k), "gbs": (alg[k] / (t / args.steps * 1e-3) / 1e9) if k in alg and t > 0 else None}
@@ -730,11 +841,7 @@ def main(argv=None):
                                   else "eager launches"),
                        "tokens_per_step": tokens},
             "hbm_gbs_step": step_bytes * world / (step_ms * 1e-3) / 1e9,
-            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": traffic_record(dom, cfg_name),
-                         "algorithmic_bytes_per_launch": bytes_per_launch,
-                         "ms_per_launch": per_launch_ms},
+            "roofline": roof,
             "kernels": kernels,
             "gpu_launches": wl.launches_per_step * args.steps,
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,

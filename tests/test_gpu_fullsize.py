@@ -109,3 +109,28 @@ def test_quant_sweep_at_full_size_sampled_rows(fk):
     pk, sc = O.kv_quant_fp4(P.to_f64(wl.x[rows_t].cpu()))
     assert np.array_equal(wl.packed[rows_t].cpu().numpy(), pk)
     assert np.array_equal(wl.scales[rows_t].cpu().numpy(), sc)
+
+
+@pytest.mark.timeout(1200)
+def test_csa2_decoder_step_at_full_size(fk):
+    cfg = bench.CONFIGS["csa2_decoder"]
+    wl = bench.Csa2DecoderWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    seed, b, cap, K, npb, G = cfg["seed"], 0, wl.cap, wl.K, wl.npb, wl.G
+    # layer 1 (Full): flat top-K 512 and the pool of 2048 blocks
+    sc = P.oracle_scores_seq(wl.qi[0][b], wl.w[0][b], wl.keys[b], cap)
+    P.check_topk(wl.idx[0][b].cpu().numpy(), sc, np.arange(cap), K, "Full top-K")
+    pool = wl.pool[b].cpu().numpy()
+    P.check_topk(pool, O.block_max(sc, cap, 8), np.arange((cap + 7) // 8), npb, "pool")
+    # the Reindex layers of the second and the last group, inside the pool
+    pos = O.pool_positions(pool, cap, 8)
+    for g in (1, len(wl.qi) - 1):
+        sc2 = P.oracle_scores_seq(wl.qi[g][b], wl.w[g][b], wl.keys[b], cap)[pos]
+        P.check_topk(wl.idx[g][b].cpu().numpy(), sc2, pos, K, f"Reindex group {g + 1}")
+    # attention over the shared KV: Full, a Reuse of it, a Reindex layer, the last Reuse
+    new_row = P.to_f64(wl.x_new[b].cpu())
+    for l in (0, G - 1, G, wl.L - 1):
+        _attn_check(seed, 0, b, wl.q[l][b], wl.idx[l // G][b].cpu().numpy(), cap, new_row,
+                    wl.out[l][b].cpu().numpy(), wl.lse[l][b].cpu().numpy(), f"CSA2 layer {l + 1} attention")
+    _new_row_check(wl, b, wl.packed, wl.scales, wl.x_new, "CSA2 new row")

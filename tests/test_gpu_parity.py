@@ -245,6 +245,29 @@ def test_hier_pool_select_matches_oracle(fk):
         P.check_topk(pool[b], bm, np.arange(bm.size), npb, f"pool b={b}")
 
 
+def test_decoder_sizes_topk_512_pool_2048(fk):
+    # the pages' decoder sizes: top-K 512 and a pool of up to 2048 blocks; sequence 1 has
+    # fewer blocks (1126) than the pool holds, so its pool is every block plus -1 padding
+    B, cap, k, npb = 2, 40000, 512, 2048
+    q, w, keys = _indexer_inputs(15, B, cap, 32, True)
+    q2, w2 = synth.indexer_query(15, 4, B, 32, device=DEV)
+    lens = torch.tensor([40000, 9001], dtype=torch.int32, device=DEV)
+    idx, pool = fk.hier_pool_select(q, w, keys, lens, k, npb)
+    idx, pool_np = idx.cpu().numpy(), pool.cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        ref = P.oracle_scores_seq(q[b], w[b], keys[b], L)
+        P.check_topk(idx[b], ref, np.arange(L), k, f"idx b={b}")
+        P.check_topk(pool_np[b], O.block_max(ref, L, 8), np.arange((L + 7) // 8), npb, f"pool b={b}")
+    assert pool_np[1].tolist() == list(range(1126)) + [-1] * (npb - 1126)
+    idx2 = fk.indexer_topk(q2, w2, keys, lens, k, pool=pool).cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        pos = O.pool_positions(pool_np[b], L, 8)
+        ref = P.oracle_scores_seq(q2[b], w2[b], keys[b], L)[pos]
+        P.check_topk(idx2[b], ref, pos, k, f"reindex b={b}")
+
+
 def test_reindex_matches_oracle_and_full_pool_is_flat(fk):
     B, cap, k, npb = 2, 20000, 256, 64
     q, w, keys = _indexer_inputs(12, B, cap, 32, True)
