@@ -9,7 +9,7 @@ the pool, Reuse layers on the previous indices); the CSA2 decoder configuration 
 pages' own 20-layer schedule (groups of 4 over one shared KV, top-K 512, pool of 2048
 blocks). Prints ONE JSON line (rank 0).
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode32|long|hier|
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode32|decode32_fp4idx|long|hier|
        csa2_decoder|tiny|quant] [--impl ours|reference]
 Under torchrun (N > 1) each rank runs the same per-GPU workload on its own GPU (weak
 scaling; the path has no exchange step, so there is no collective in the data path); the
@@ -48,6 +48,11 @@ CONFIGS = {
     "decode32": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=True, seed=1,
                      workload="decode batch 32 x 65,536 FP4 entries, 64 heads, FP8 indexer "
                               "keys, top-K 2048"),
+    # the same decode step with the indexer query and keys stored in FP4 (E2M1 + one E4M3
+    # scale per 16 dims), the format the pages give the indexer
+    "decode32_fp4idx": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=False, idx="fp4", seed=1,
+                            workload="decode batch 32 x 65,536 FP4 entries, 64 heads, FP4 indexer "
+                                     "query and keys (E2M1 + E4M3 per 16 dims), top-K 2048"),
     "long": dict(B=4, cap=1 << 20, H=64, H_I=32, K=2048, fp8=True, seed=2,
                  workload="long context batch 4 x 1,048,576 FP4 entries, 64 heads, FP8 "
                           "indexer keys, top-K 2048"),
@@ -307,21 +312,32 @@ class DecodeWorkload(TwoSets):
         seed = cfg["seed"] + 1000 * rank
         self.B, self.cap, self.H, self.H_I, self.K = B, cap, H, H_I, K
         fp8 = cfg["fp8"]
-        self.key_bytes = DK * (1 if fp8 else 2)
+        self.fp4_idx = cfg.get("idx") == "fp4"
+        self.key_bytes = DK // 2 + DK // 16 if self.fp4_idx else DK * (1 if fp8 else 2)
         # resident cache: FP4 rows + indexer keys, filled through the library's quantizer
         self.packed = torch.empty((B, cap, D // 2), dtype=torch.uint8, device=device)
         self.scales = torch.empty((B, cap, D // 16), dtype=torch.uint8, device=device)
-        self.keys = torch.empty((B, cap, DK), dtype=torch.uint8 if fp8 else torch.bfloat16, device=device)
+        if self.fp4_idx:
+            self.keys = fk.E2M1Planes(B, cap, device)
+        else:
+            self.keys = torch.empty((B, cap, DK), dtype=torch.uint8 if fp8 else torch.bfloat16, device=device)
         chunk = 1 << 18
         for b in range(B):
             for r0 in range(0, cap, chunk):
                 rows = torch.arange(r0, min(cap, r0 + chunk), dtype=torch.int64, device=device)
                 x = synth.kv_rows(seed, 0, b, rows, D)
                 fk.kv_quant_fp4(x, self.packed[b, r0:r0 + rows.numel()], self.scales[b, r0:r0 + rows.numel()])
-                self.keys[b, r0:r0 + rows.numel()] = synth.indexer_keys(seed, b, rows, DK, fp8)
+                kr = synth.indexer_keys(seed, b, rows, DK, fp8)
+                if self.fp4_idx:  # stored with the library's quantizer (d = 128)
+                    fk.kv_quant_fp4(kr, self.keys.codes[b, r0:r0 + rows.numel()],
+                                    self.keys.scales[b, r0:r0 + rows.numel()])
+                else:
+                    self.keys[b, r0:r0 + rows.numel()] = kr
         # per-step inputs (device copies, and pinned host copies for the end-to-end run)
         self.q = synth.attn_query(seed, 0, B, H, D, device=device)
         self.qi, self.w = synth.indexer_query(seed, 0, B, H_I, fp8=fp8, device=device)
+        # FP4 indexer: the bf16 query is stored as FP4 inside each step
+        self.qi4 = fk.E2M1Planes(B, H_I, device) if self.fp4_idx else None
         self.x_new = synth.kv_rows(seed, 0, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
         self.dst = (torch.arange(B, dtype=torch.int64, device=device) * cap + (cap - 1))
         self.lens = torch.full((B,), cap, dtype=torch.int32, device=device)
@@ -334,14 +350,19 @@ class DecodeWorkload(TwoSets):
         self.outputs = [self.out, self.lse]
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
         # quantize, scan, select (filter + finish), attention (+ the chunk merge when split)
-        self.launches_per_step = 5 + attn_split(fk, B, cap, H, K)
+        # (+ the query's FP4 quantize with an FP4 indexer)
+        self.launches_per_step = 5 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
         self.tokens_per_step = B
 
     def step(self):
         fk = self.fk
         fk.kv_quant_fp4(self.x_new, self.packed.view(-1, D // 2), self.scales.view(-1, D // 16),
                         dst_row=self.dst)
-        fk.indexer_topk(self.qi, self.w, self.keys, self.lens, self.K, ws=self.ws_i, out_idx=self.idx)
+        if self.fp4_idx:
+            self.qi4.quantize_from(self.qi)
+            fk.indexer_topk(self.qi4, self.w, self.keys, self.lens, self.K, ws=self.ws_i, out_idx=self.idx)
+        else:
+            fk.indexer_topk(self.qi, self.w, self.keys, self.lens, self.K, ws=self.ws_i, out_idx=self.idx)
         fk.sparse_attn_decode(self.q, self.packed, self.scales, self.lens, self.idx, 1.0,
                               ws=self.ws_a, out=self.out, lse=self.lse)
 
@@ -632,6 +653,8 @@ def oracle_sample_decode(cfg, seq: int, layer_seed=None):
     qi, w = synth.indexer_query(seed, 0, seq + 1, H_I, fp8=fp8)
     kf = O.fp8_e4m3_to_f64(keys.numpy()) if fp8 else O.bf16_bits_to_f64(keys.view(torch.int16).numpy().astype(np.uint16))
     qf = O.fp8_e4m3_to_f64(qi[seq].numpy()) if fp8 else O.bf16_bits_to_f64(qi[seq].view(torch.int16).numpy().astype(np.uint16))
+    if cfg.get("idx") == "fp4":
+        kf, qf = O.indexer_fp4_values(kf), O.indexer_fp4_values(qf)
     x_new = synth.kv_rows(seed, 0, 10 ** 6, torch.tensor([seq]), D)
     O.kv_quant_fp4(O.bf16_bits_to_f64(x_new.view(torch.int16).numpy().astype(np.uint16)))
     idx, _ = O.indexer_topk(qf, w[seq].double().numpy(), kf, cap, K)

@@ -16,7 +16,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp4kv.so")
 
-KEY_BF16, KEY_E4M3 = 0, 1
+KEY_BF16, KEY_E4M3, KEY_E2M1 = 0, 1, 2
 OP_KV_QUANT, OP_INDEXER_TOPK, OP_REINDEX_TOPK, OP_HIER_POOL_SELECT, OP_SPARSE_ATTN, \
     OP_INDEXER_SCORES = range(6)
 
@@ -88,7 +88,41 @@ def _check(status: int):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    if t is None:
+        return None
+    if isinstance(t, E2M1Planes):
+        t = t.buf
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class E2M1Planes:
+    """An FP4 indexer operand of shape [B, rows, 128]: E2M1 codes [B][rows][64] followed,
+    in the same buffer, by the E4M3 scales [B][rows][8] (the layout of key_dtype E2M1)."""
+
+    DK = 128
+
+    def __init__(self, B: int, rows: int, device):
+        self.B, self.rows = int(B), int(rows)
+        n = self.B * self.rows
+        self.buf = torch.empty(n * (self.DK // 2 + self.DK // 16), dtype=torch.uint8, device=device)
+        self.codes = self.buf[:n * (self.DK // 2)].view(self.B, self.rows, self.DK // 2)
+        self.scales = self.buf[n * (self.DK // 2):].view(self.B, self.rows, self.DK // 16)
+
+    @property
+    def device(self):
+        return self.buf.device
+
+    @property
+    def shape(self):
+        return (self.B, self.rows, self.DK)
+
+    def quantize_from(self, x: torch.Tensor):
+        """Fill from bf16 x [B, rows, 128] with the library's FP4 quantizer."""
+        if tuple(x.shape) != self.shape:
+            raise ValueError(f"x: expected shape {self.shape}, got {tuple(x.shape)}")
+        kv_quant_fp4(x.reshape(-1, self.DK), self.codes.view(-1, self.DK // 2),
+                     self.scales.view(-1, self.DK // 16))
+        return self
 
 
 def _stream(device=None):
@@ -163,17 +197,23 @@ def kv_quant_fp4(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
 
 
 def _key_dtype(keys):
+    if isinstance(keys, E2M1Planes):
+        return KEY_E2M1
     if keys.dtype == torch.uint8:
         return KEY_E4M3
     if keys.dtype == torch.bfloat16:
         return KEY_BF16
-    raise TypeError("keys: expected uint8 (E4M3 codes) or bf16")
+    raise TypeError("keys: expected uint8 (E4M3 codes), bf16 or E2M1Planes")
 
 
 def _check_indexer(q, w, keys, seq_lens, key_scale):
     kd = _key_dtype(keys)
-    _need(q, keys.dtype, "q", keys.device)
-    _need(keys, keys.dtype, "keys")
+    if kd == KEY_E2M1:
+        if not isinstance(q, E2M1Planes) or q.device != keys.device:
+            raise TypeError("q: expected E2M1Planes on the keys' device (keys are E2M1Planes)")
+    else:
+        _need(q, keys.dtype, "q", keys.device)
+        _need(keys, keys.dtype, "keys")
     _need(w, torch.float32, "w", keys.device)
     _need(seq_lens, torch.int32, "seq_lens", keys.device)
     if key_scale is not None:

@@ -181,8 +181,11 @@ fp4kv_status check_indexer_args(const void* q, const float* w, int32_t H_I, cons
     return fail(FP4KV_ERR_UNSUPPORTED, "cap=%lld outside [1, 2^31 - 8]", (long long)cap);
   if (int64_t(B) * cap > (int64_t(1) << 31) - 256)
     return fail(FP4KV_ERR_UNSUPPORTED, "B*cap=%lld must stay below 2^31 rows", (long long)(int64_t(B) * cap));
-  if (key_dtype != FP4KV_KEY_BF16 && key_dtype != FP4KV_KEY_E4M3)
+  if (key_dtype != FP4KV_KEY_BF16 && key_dtype != FP4KV_KEY_E4M3 && key_dtype != FP4KV_KEY_E2M1)
     return fail(FP4KV_ERR_UNSUPPORTED, "key_dtype=%d", key_dtype);
+  if (key_dtype == FP4KV_KEY_E2M1 && ((H_I & 1) || (cap & 1)))
+    return fail(FP4KV_ERR_UNSUPPORTED, "E2M1 keys need an even H_I and cap (H_I=%d, cap=%lld)", H_I,
+                (long long)cap);
   if (!aligned(q, 16) || !aligned(keys, 16) || !aligned(w, 4))
     return fail(FP4KV_ERR_INVALID_ARG, "q and keys must be 16-byte aligned");
   return FP4KV_OK;
@@ -196,7 +199,12 @@ fp4kv::IndexScoreParams score_params(const void* q, const float* w, int32_t H_I,
   p.w = w;
   p.H_I = H_I;
   p.keys = keys;
-  p.keys_fp8 = key_dtype == FP4KV_KEY_E4M3;
+  p.key_type = key_dtype;  // the kernel's numbering follows fp4kv_key_dtype
+  if (key_dtype == FP4KV_KEY_E2M1) {
+    // two planes back to back: codes [rows][64], then scales [rows][8]
+    p.key_sf = static_cast<const uint8_t*>(keys) + int64_t(B) * cap * 64;
+    p.q_sf = static_cast<const uint8_t*>(q) + int64_t(B) * H_I * 64;
+  }
   p.key_scale = key_scale;
   p.cap = cap;
   p.seq_lens = seq_lens;

@@ -15,11 +15,13 @@ cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_
 // top-K select and, for the hierarchical Full layer, the block max over 8 positions.
 // ----------------------------------------------------------------------------------------
 struct IndexScoreParams {
-  const void* q;            // [B][H_I][128] e4m3 codes or bf16 bits
+  const void* q;            // [B][H_I][128] e4m3 codes or bf16 bits, or [B][H_I][64] e2m1 pairs
   const float* w;           // [B][H_I]
   int H_I;
-  const void* keys;         // [B][cap][128]
-  bool keys_fp8;
+  const void* keys;         // [B][cap][128] (bf16, e4m3) or [B][cap][64] (e2m1 pairs)
+  int key_type;             // 0 bf16, 1 e4m3, 2 e2m1 with per-16 e4m3 scales
+  const uint8_t* key_sf;    // e2m1: [B][cap][8] e4m3 scales
+  const uint8_t* q_sf;      // e2m1: [B][H_I][8] e4m3 scales
   const float* key_scale;   // nullable [B][cap]
   int64_t cap;
   const int32_t* seq_lens;  // [B]

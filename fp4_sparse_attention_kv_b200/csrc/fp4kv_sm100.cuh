@@ -136,6 +136,40 @@ __host__ __device__ constexpr uint32_t umma_idesc(uint32_t ab_format, int M, int
   return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
          (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
+// K-major operand, 64-byte swizzle, rows of 64 bytes grouped in 8-row (512 B) atoms:
+// stride byte offset 512 between 8-row groups, layout type 4 (64B swizzle).
+FP4KV_DEV uint64_t sw64_kmajor_desc(uint32_t smem_addr) {
+  return uint64_t((smem_addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(512 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(4) << 61);
+}
+// Unswizzled K-major block of 16-byte rows stored back to back (8-row core matrices 128 B
+// apart): the source of a tcgen05.cp of 32 rows x 128 bits.
+FP4KV_DEV uint64_t rows16_desc(uint32_t smem_addr) {
+  return uint64_t((smem_addr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
+         (uint64_t(1) << 46);
+}
+// Instruction descriptor of the block-scaled FP4 MMA (kind::mxf4nvf4): A and B E2M1
+// (format 1), one unsigned E4M3 scale per 16 elements of K (scale format 0), K = 64 per
+// instruction, both operands K-major, fp32 accumulate, scale-factor byte ids 0.
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T, E2M1 operands with per-16 E4M3 block scales read
+// from TMEM at sfa / sfb; one CTA, issued by a single thread.
+FP4KV_DEV void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                         uint32_t sfa_tmem, uint32_t sfb_tmem, bool acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc ? 1u : 0u), "r"(sfa_tmem),
+        "r"(sfb_tmem) : "memory");
+}
+// Copy 32 rows x 128 bits of shared memory into TMEM columns [taddr, taddr + 4) of lanes
+// 0-31, replicated into the other three 32-lane subpartitions. Asynchronous; ordered
+// before later tcgen05.mma of the same thread and tracked by tcgen05.commit.
+FP4KV_DEV void tmem_cp_32x128_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
 FP4KV_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 FP4KV_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(

@@ -67,7 +67,13 @@ typedef enum {
   FP4KV_ERR_DEVICE_FLAG = 5          /* a kernel reported a timed-out wait (status word)  */
 } fp4kv_status;
 
-typedef enum { FP4KV_KEY_BF16 = 0, FP4KV_KEY_E4M3 = 1 } fp4kv_key_dtype;
+/* Indexer query / key formats. FP4KV_KEY_E2M1 is the FP4 indexer format ([PyTorchKR] FP4
+ * KV section: the indexer query and key were already FP4): each 128-dim vector is 64
+ * bytes of E2M1 codes (two per byte, even dim in the low nibble) plus 8 E4M3 scales (one
+ * per 16 dims), as fp4kv_kv_quant_fp4 with d = 128 writes them. The q and keys buffers
+ * each hold two planes back to back: all codes [B][rows][64], then all scales
+ * [B][rows][8] (rows = H_I for q, cap for keys). Needs an even H_I and an even cap. */
+typedef enum { FP4KV_KEY_BF16 = 0, FP4KV_KEY_E4M3 = 1, FP4KV_KEY_E2M1 = 2 } fp4kv_key_dtype;
 
 typedef enum {
   FP4KV_OP_KV_QUANT = 0,
@@ -128,9 +134,10 @@ fp4kv_status fp4kv_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int32_t d, in
 
 /* indexer_scores -- Full-mode scoring of every visible entry, no selection
  * ([PyTorchKR] CSA2 section: the indexer scores all causally visible positions).
- * q         : [B][H_I][128] E4M3 codes (key_dtype E4M3) or bf16 bits (key_dtype BF16).
+ * q         : [B][H_I][128] E4M3 codes (key_dtype E4M3) or bf16 bits (key_dtype BF16), or
+ *             the two E2M1 planes (key_dtype E2M1, see fp4kv_key_dtype).
  * w         : fp32 [B][H_I] head weights (any query scale folded in).
- * keys      : [B][cap][128], same dtype as q. 16-byte aligned.
+ * keys      : [B][cap][128], same dtype as q (E2M1: the two planes). 16-byte aligned.
  * key_scale : nullable fp32 [B][cap] per-entry key scale ks.
  * seq_lens  : int32 [B] (device); seq_lens[b] <= cap. Entries n >= seq_lens[b] are not
  *             scored and out_score[b][n] is left unwritten for them.

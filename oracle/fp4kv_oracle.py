@@ -31,7 +31,8 @@ Readings where the pages are silent (each is listed in the design notes):
 * E2M1 codes round-to-nearest-even on the code, saturating at 6; the sign of x is kept,
   so a negative value that rounds to zero is stored as 0x8;
 * two codes per byte, the even channel in the low nibble; scales one byte per group;
-* indexer score = ks[n] * sum_h w_h * max(0, q_h . k_n), rounded to fp32;
+* indexer score = ks[n] * sum_h w_h * max(0, q_h . k_n), rounded to fp32; with FP4
+  indexer operands, q and k are first stored with the main KV's quantizer;
 * top-K by (fp32 score descending, index ascending), output in ascending index order,
   padded with -1;
 * attention: softmax(sm_scale * q . v_hat) . v_hat, one latent row serving as K and V.
@@ -195,6 +196,15 @@ def indexer_scores(q, w, keys, key_scale=None) -> np.ndarray:
     if key_scale is not None:
         s = s * np.asarray(key_scale, dtype=np.float64)
     return s.astype(np.float32)
+
+
+def indexer_fp4_values(x) -> np.ndarray:
+    """FP4 indexer operand ([PyTorchKR] FP4 main-KV section: DeepSeek-V4 already kept the
+    indexer query and key in FP4): the values 128-dim query or key rows x [R, 128] (exact
+    bf16 values as fp64) hold once stored as E2M1 codes with one E4M3 scale per 16 dims,
+    quantized exactly as the main KV is. Scores of FP4 operands are indexer_scores of these
+    values."""
+    return kv_dequant_fp4(*kv_quant_fp4(x))
 
 
 def topk_positions(scores, positions, top_k: int) -> np.ndarray:

@@ -401,3 +401,97 @@ def test_selftest_hook_rejects_bad_arguments(fk):
         with pytest.raises(fk.Fp4kvError):
             fk.selftest_wait_timeout(bad, ws)
     assert fk.workspace_status(ws) == 0
+
+
+# ----------------------------------------------------------------------------------------
+# FP4 (E2M1 + per-16 E4M3 scale) indexer query and keys
+# ----------------------------------------------------------------------------------------
+
+def _fp4_indexer_inputs(fk, seed, B, cap, H_I, layer=0):
+    """bf16 indexer query / keys from the generator, stored as FP4 by the library."""
+    qb, w = synth.indexer_query(seed, layer, B, H_I, fp8=False, device=DEV)
+    kb = P.keys_dev(seed, B, cap, False, DEV)
+    q4 = fk.E2M1Planes(B, H_I, DEV).quantize_from(qb)
+    k4 = fk.E2M1Planes(B, cap, DEV).quantize_from(kb)
+    return qb, w, kb, q4, k4
+
+
+def _fp4_oracle_scores(qb_b, w_b, kb_b, L, ks=None):
+    """The oracle's own FP4 storage of the bf16 inputs, then its scores (fp32)."""
+    return O.indexer_scores(O.indexer_fp4_values(P.to_f64(qb_b)), w_b.detach().cpu().double().numpy(),
+                            O.indexer_fp4_values(P.to_f64(kb_b[:L])),
+                            None if ks is None else ks[:L].detach().cpu().double().numpy())
+
+
+def test_fp4_indexer_planes_are_the_quantizer_output(fk):
+    qb, _, kb, q4, k4 = _fp4_indexer_inputs(fk, 21, 2, 600, 32)
+    for x, planes in ((qb, q4), (kb, k4)):
+        pk, sc = O.kv_quant_fp4(P.to_f64(x.reshape(-1, 128)))
+        assert np.array_equal(planes.codes.reshape(-1, 64).cpu().numpy(), pk)
+        assert np.array_equal(planes.scales.reshape(-1, 8).cpu().numpy(), sc)
+
+
+@pytest.mark.parametrize("H_I", [8, 32, 48, 64])
+def test_fp4_indexer_scores_match_oracle(fk, H_I):
+    B, cap = 2, 1000
+    qb, w, kb, q4, k4 = _fp4_indexer_inputs(fk, 22, B, cap, H_I)
+    lens = torch.tensor([1000, 613], dtype=torch.int32, device=DEV)
+    ks = torch.rand((B, cap), generator=torch.Generator().manual_seed(2)).to(DEV) + 0.5
+    for key_scale in (None, ks):
+        got = fk.indexer_scores(q4, w, k4, lens, key_scale=key_scale).cpu().numpy()
+        for b in range(B):
+            L = int(lens[b])
+            ref = _fp4_oracle_scores(qb[b], w[b], kb[b], L, None if key_scale is None else ks[b])
+            err = np.abs(got[b, :L].astype(np.float64) - ref) / np.maximum(np.abs(ref), 1e-3)
+            assert err.max() <= 2e-6, err.max()
+            assert np.all(np.isneginf(got[b, L:]))
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=23, B=3, cap=5000, lens=[5000, 4093, 77], H_I=32, k=300),
+    dict(seed=24, B=2, cap=70000, lens=[70000, 65537], H_I=32, k=2048),
+    dict(seed=25, B=2, cap=3000, lens=[3000, 2999], H_I=8, k=1),
+    dict(seed=26, B=1, cap=9000, lens=[9000], H_I=64, k=4096),
+])
+def test_fp4_indexer_topk_matches_oracle(fk, case):
+    qb, w, kb, q4, k4 = _fp4_indexer_inputs(fk, case["seed"], case["B"], case["cap"], case["H_I"])
+    lens = torch.tensor(case["lens"], dtype=torch.int32, device=DEV)
+    k = case["k"]
+    idx = fk.indexer_topk(q4, w, k4, lens, k).cpu().numpy()
+    for b in range(case["B"]):
+        L = case["lens"][b]
+        P.check_topk(idx[b], _fp4_oracle_scores(qb[b], w[b], kb[b], L), np.arange(L), k, f"b={b}")
+
+
+def test_fp4_hier_pool_select_and_reindex_match_oracle(fk):
+    B, cap, k, npb = 2, 20000, 256, 64
+    qb, w, kb, q4, k4 = _fp4_indexer_inputs(fk, 27, B, cap, 32)
+    q2b, w2 = synth.indexer_query(27, 1, B, 32, fp8=False, device=DEV)
+    q24 = fk.E2M1Planes(B, 32, DEV).quantize_from(q2b)
+    lens = torch.tensor([20000, 12346], dtype=torch.int32, device=DEV)
+    idx, pool = fk.hier_pool_select(q4, w, k4, lens, k, npb)
+    idx, pool_np = idx.cpu().numpy(), pool.cpu().numpy()
+    idx2 = fk.indexer_topk(q24, w2, k4, lens, k, pool=pool).cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        ref = _fp4_oracle_scores(qb[b], w[b], kb[b], L)
+        P.check_topk(idx[b], ref, np.arange(L), k, f"idx b={b}")
+        P.check_topk(pool_np[b], O.block_max(ref, L, 8), np.arange((L + 7) // 8), npb, f"pool b={b}")
+        pos = O.pool_positions(pool_np[b], L, 8)
+        ref2 = _fp4_oracle_scores(q2b[b], w2[b], kb[b], L)[pos]
+        P.check_topk(idx2[b], ref2, pos, k, f"reindex b={b}")
+
+
+def test_fp4_indexer_rejects_odd_sizes(fk):
+    _, w, _, q4, _ = _fp4_indexer_inputs(fk, 28, 1, 64, 32)
+    k_odd = fk.E2M1Planes(1, 63, DEV)
+    k_odd.buf.zero_()
+    lens = torch.tensor([63], dtype=torch.int32, device=DEV)
+    with pytest.raises(fk.Fp4kvError):
+        fk.indexer_topk(q4, w, k_odd, lens, 8)
+    q_odd = fk.E2M1Planes(1, 31, DEV)
+    q_odd.buf.zero_()
+    k_even = fk.E2M1Planes(1, 64, DEV)
+    k_even.buf.zero_()
+    with pytest.raises(fk.Fp4kvError):
+        fk.indexer_topk(q_odd, w[:, :31].contiguous(), k_even, lens, 8)

@@ -189,3 +189,48 @@ def test_attention_with_no_valid_entry():
     packed, scales = _rows(rng, 4, 32)
     out, lse = O.sparse_attn_decode(np.ones((2, 32)), packed, scales, np.array([-1, 9]), 4, 1.0)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+# ----------------------------------------------------------------------------------------
+# FP4 indexer operands
+# ----------------------------------------------------------------------------------------
+
+def test_fp4_indexer_values_leave_fp4_grid_rows_unchanged():
+    """Rows already on the FP4 grid, with each 16-dim group's largest magnitude equal to
+    6 * S for an E4M3 value S, are stored without loss: the FP4 scores equal the plain
+    scores of the same values."""
+    rng = np.random.default_rng(3)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    e4m3_normals = O.e4m3_decode(np.arange(0x08, 0x7F))  # normal E4M3 values
+
+    def grid_rows(n):
+        mags = grid[rng.integers(0, 8, size=(n, 8, 16))]
+        mags[:, :, 0] = 6.0  # the group's amax is 6 * S exactly
+        sign = np.where(rng.random((n, 8, 16)) < 0.5, -1.0, 1.0)
+        S = e4m3_normals[rng.integers(0, e4m3_normals.size, size=(n, 8, 1))]
+        S = np.minimum(S, 2.0)  # keep products well inside the bf16 and fp32 ranges
+        return (sign * mags * S).reshape(n, 128)
+
+    q, keys = grid_rows(4), grid_rows(50)
+    assert np.array_equal(O.indexer_fp4_values(q), q)
+    assert np.array_equal(O.indexer_fp4_values(keys), keys)
+    w = rng.uniform(0.5, 1.5, size=4)
+    assert np.array_equal(O.indexer_scores(O.indexer_fp4_values(q), w, O.indexer_fp4_values(keys)),
+                          O.indexer_scores(q, w, keys))
+
+
+def test_fp4_indexer_one_nonzero_dim_closed_form():
+    """A query and a key with one non-zero dim c: each group holding it quantizes to
+    6 * E4M3(|x| / 6) with x's sign, so the single-head score is
+    w * max(0, sign * 36 * E4M3(|q_c| / 6) * E4M3(|k_c| / 6))."""
+    qs = [0.3, -1.7, 2.5, 0.01171875, 100.0]
+    ks = [1.0, 0.4, -3.3, 7.0, 0.05]
+    for i, (qv, kv) in enumerate(zip(qs, ks)):
+        c = (5 * i + 3) % 128
+        q = np.zeros((1, 128))
+        k = np.zeros((1, 128))
+        q[0, c], k[0, c] = qv, kv
+        want = 0.75 * max(0.0, np.sign(qv * kv) * 36.0 * O.e4m3_decode(O.e4m3_round_sat(abs(qv) / 6.0))
+                          * O.e4m3_decode(O.e4m3_round_sat(abs(kv) / 6.0)))
+        got = O.indexer_scores(O.indexer_fp4_values(q), [0.75], O.indexer_fp4_values(k))
+        assert got[0] == np.float32(want), (qv, kv, got[0], want)
