@@ -9,8 +9,8 @@ the pool, Reuse layers on the previous indices); the CSA2 decoder configuration 
 pages' own 20-layer schedule (groups of 4 over one shared KV, top-K 512, pool of 2048
 blocks). Prints ONE JSON line (rank 0).
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode32|decode32_fp4idx|long|hier|
-       csa2_decoder|tiny|quant] [--impl ours|reference]
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--config decode32|decode32_fp4idx|decode32_swa|long|hier|csa2_decoder|tiny|quant]
 Under torchrun (N > 1) each rank runs the same per-GPU workload on its own GPU (weak
 scaling; the path has no exchange step, so there is no collective in the data path); the
 step time is the max over ranks.
@@ -41,6 +41,7 @@ METRIC = "sparse FP4 decode-attention tokens/s; achieved HBM GB/s (% of B200 pea
 D = 512
 DK = 128
 ROW_BYTES = D // 2 + D // 16  # 288
+SWA_LAYER = 700  # generator stream of the sliding-window rows
 L2_BYTES = 126 * 2 ** 20
 
 CONFIGS = {
@@ -53,6 +54,11 @@ CONFIGS = {
     "decode32_fp4idx": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=False, idx="fp4", seed=1,
                             workload="decode batch 32 x 65,536 FP4 entries, 64 heads, FP4 indexer "
                                      "query and keys (E2M1 + E4M3 per 16 dims), top-K 2048"),
+    # the same decode step with the sliding-window branch: the last 128 positions' KV in FP8,
+    # attended in the same softmax as the selected rows
+    "decode32_swa": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=True, swa=128, seed=1,
+                         workload="decode batch 32 x 65,536 FP4 entries + a 128-token FP8 sliding "
+                                  "window, 64 heads, FP8 indexer keys, top-K 2048"),
     "long": dict(B=4, cap=1 << 20, H=64, H_I=32, K=2048, fp8=True, seed=2,
                  workload="long context batch 4 x 1,048,576 FP4 entries, 64 heads, FP8 "
                           "indexer keys, top-K 2048"),
@@ -338,6 +344,18 @@ class DecodeWorkload(TwoSets):
         self.qi, self.w = synth.indexer_query(seed, 0, B, H_I, fp8=fp8, device=device)
         # FP4 indexer: the bf16 query is stored as FP4 inside each step
         self.qi4 = fk.E2M1Planes(B, H_I, device) if self.fp4_idx else None
+        # sliding window: ring of the last n_win positions' rows (E4M3), slot = position % n_win
+        self.n_win = cfg.get("swa", 0)
+        self.swa = None
+        if self.n_win:
+            nw = self.n_win
+            self.swa = torch.empty((B, nw, D), dtype=torch.uint8, device=device)
+            pos = torch.arange(cap - nw, cap, dtype=torch.int64, device=device)
+            for b in range(B):
+                fk.swa_quant_fp8(synth.kv_rows(seed, SWA_LAYER, b, pos, D), self.swa[b],
+                                 dst_row=pos % nw)
+            self.x_swa_new = synth.kv_rows(seed, SWA_LAYER, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
+            self.swa_dst = torch.arange(B, dtype=torch.int64, device=device) * nw + (cap - 1) % nw
         self.x_new = synth.kv_rows(seed, 0, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
         self.dst = (torch.arange(B, dtype=torch.int64, device=device) * cap + (cap - 1))
         self.lens = torch.full((B,), cap, dtype=torch.int32, device=device)
@@ -347,29 +365,36 @@ class DecodeWorkload(TwoSets):
         self.ws_i = fk.alloc_workspace(fk.workspace_bytes(fk.OP_INDEXER_TOPK, B, cap, H_I, K), device)
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
         self.inputs = [self.q, self.qi, self.w, self.x_new]
-        self.outputs = [self.out, self.lse]
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
+        if self.n_win:
+            self.inputs.append(self.x_swa_new)
+            self.in_attrs = self.in_attrs + ("x_swa_new",)
+        self.outputs = [self.out, self.lse]
         # quantize, scan, select (filter + finish), attention (+ the chunk merge when split)
-        # (+ the query's FP4 quantize with an FP4 indexer)
-        self.launches_per_step = 5 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
+        # (+ the query's FP4 quantize with an FP4 indexer, + the window row's FP8 write)
+        self.launches_per_step = (5 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
+                                  + (1 if self.n_win else 0))
+        self.attn_rows_per_step = B * (K + self.n_win)
         self.tokens_per_step = B
 
     def step(self):
         fk = self.fk
         fk.kv_quant_fp4(self.x_new, self.packed.view(-1, D // 2), self.scales.view(-1, D // 16),
                         dst_row=self.dst)
+        if self.n_win:
+            fk.swa_quant_fp8(self.x_swa_new, self.swa.view(-1, D), dst_row=self.swa_dst)
         if self.fp4_idx:
             self.qi4.quantize_from(self.qi)
             fk.indexer_topk(self.qi4, self.w, self.keys, self.lens, self.K, ws=self.ws_i, out_idx=self.idx)
         else:
             fk.indexer_topk(self.qi, self.w, self.keys, self.lens, self.K, ws=self.ws_i, out_idx=self.idx)
         fk.sparse_attn_decode(self.q, self.packed, self.scales, self.lens, self.idx, 1.0,
-                              ws=self.ws_a, out=self.out, lse=self.lse)
+                              ws=self.ws_a, out=self.out, lse=self.lse, swa=self.swa)
 
     def algorithmic_bytes(self):
         return {"index_score": self.B * self.cap * self.key_bytes,
-                "sparse_attn": self.B * self.K * ROW_BYTES,
-                "kv_quant_fp4": self.B * (2 * D + ROW_BYTES)}
+                "sparse_attn": self.B * (self.K * ROW_BYTES + self.n_win * D),
+                "kv_quant_fp4": self.B * (2 * D + ROW_BYTES) + (self.B * (2 * D + D) if self.n_win else 0)}
 
 
 class HierWorkload(TwoSets):
@@ -662,8 +687,14 @@ def oracle_sample_decode(cfg, seq: int, layer_seed=None):
     xr = synth.kv_rows(seed, 0, seq, torch.as_tensor(sel), D)
     pk, sc = O.kv_quant_fp4(O.bf16_bits_to_f64(xr.view(torch.int16).numpy().astype(np.uint16)))
     q = synth.attn_query(seed, 0, seq + 1, H, D)[seq]
-    O.sparse_attn_decode_rows(O.bf16_bits_to_f64(q.view(torch.int16).numpy().astype(np.uint16)),
-                              O.kv_dequant_fp4(pk, sc), 1.0)
+    qf64 = O.bf16_bits_to_f64(q.view(torch.int16).numpy().astype(np.uint16))
+    nw = cfg.get("swa", 0)
+    if nw:
+        xw = synth.kv_rows(seed, SWA_LAYER, seq, torch.arange(cap - nw, cap, dtype=torch.int64), D)
+        vw = O.e4m3_decode(O.swa_quant_fp8(O.bf16_bits_to_f64(xw.view(torch.int16).numpy().astype(np.uint16))))
+        O.sparse_swa_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), vw, 1.0)
+    else:
+        O.sparse_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), 1.0)
 
 
 def oracle_sample_quant(cfg, rows=2048):
@@ -832,7 +863,8 @@ def main(argv=None):
     if dom == "sparse_attn":
         # 4*H*d flops per gathered row of 288 bytes (455 flop/B at H = 64) is above the
         # ridge point of the measured peaks: the attention is bound by the tensor cores
-        flops_per_launch = bytes_per_launch / ROW_BYTES * attn_flops_per_row(wl.H)
+        rows = getattr(wl, "attn_rows_per_step", alg[dom] / ROW_BYTES)
+        flops_per_launch = rows / max(1, n_l / args.steps) * attn_flops_per_row(wl.H)
         tpeak, tpeak_kind = measured_tensor_peak()
         achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": tpeak,

@@ -46,6 +46,9 @@ SIGNATURES = [
     ("fp4kv_profile_enable", ctypes.c_int, [_I32]),
     ("fp4kv_profile_read", ctypes.c_int, [ctypes.POINTER(_I32), ctypes.POINTER(_F32)]),
     ("fp4kv_selftest_wait_timeout", ctypes.c_int, [_I32, _P, _SZ, _P]),
+    ("fp4kv_sparse_swa_attn_decode", ctypes.c_int,
+     [_P, _I32, _I32, _I32, _P, _P, _I64, _P, _P, _I32, _P, _I32, _F32, _P, _P, _P, _SZ, _P]),
+    ("fp4kv_swa_quant_fp8", ctypes.c_int, [_P, _I64, _I32, _I64, _P, _P, _I64, _P]),
 ]
 
 KERNEL_KINDS = ("kv_quant_fp4", "index_score", "topk_select", "sparse_attn")
@@ -284,9 +287,10 @@ def hier_pool_select(q, w, keys, seq_lens, top_k, n_pool_blocks, block_size=8,
 
 
 def sparse_attn_decode(q, packed, scales, seq_lens, idx, sm_scale=1.0, ws=None, out=None,
-                       lse=None, want_lse=True):
+                       lse=None, want_lse=True, swa=None):
     """q bf16 [B, H, d]; packed uint8 [B, cap, d/2]; scales uint8 [B, cap, d/16];
-    idx int32 [B, top_k]. Returns (out fp32 [B, H, d], lse fp32 [B, H] or None)."""
+    idx int32 [B, top_k]; swa (optional) uint8 [B, n_win, d] E4M3 sliding-window rows, attended
+    in the same softmax. Returns (out fp32 [B, H, d], lse fp32 [B, H] or None)."""
     _need(q, torch.bfloat16, "q")
     dev = q.device
     _need(packed, torch.uint8, "packed", dev)
@@ -304,11 +308,36 @@ def sparse_attn_decode(q, packed, scales, seq_lens, idx, sm_scale=1.0, ws=None, 
         lse = torch.empty((B, H), dtype=torch.float32, device=dev)
     if ws is None:
         ws = alloc_workspace(workspace_bytes(OP_SPARSE_ATTN, B, cap, H, top_k), dev)
-    _check(lib().fp4kv_sparse_attn_decode(_ptr(q), B, H, d, _ptr(packed), _ptr(scales), cap,
-                                          _ptr(seq_lens), _ptr(idx), top_k, float(sm_scale),
-                                          _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
-                                          _stream(dev)))
+    if swa is None:
+        _check(lib().fp4kv_sparse_attn_decode(_ptr(q), B, H, d, _ptr(packed), _ptr(scales), cap,
+                                              _ptr(seq_lens), _ptr(idx), top_k, float(sm_scale),
+                                              _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                              _stream(dev)))
+    else:
+        _need(swa, torch.uint8, "swa", dev)
+        if swa.dim() != 3 or swa.shape[0] != B or swa.shape[2] != d:
+            raise ValueError("swa: expected uint8 [B, n_win, d]")
+        _check(lib().fp4kv_sparse_swa_attn_decode(_ptr(q), B, H, d, _ptr(packed), _ptr(scales), cap,
+                                                  _ptr(seq_lens), _ptr(idx), top_k, _ptr(swa),
+                                                  swa.shape[1], float(sm_scale), _ptr(out), _ptr(lse),
+                                                  _ptr(ws), ws.numel(), _stream(dev)))
     return out, lse
+
+
+def swa_quant_fp8(x: torch.Tensor, out: torch.Tensor, dst_row: torch.Tensor | None = None):
+    """E4M3 codes of bf16 rows x [n, d] into out [cap, d] (uint8), at rows dst_row (int64
+    [n]) or 0..n-1: the sliding-window KV's write."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise TypeError("x: expected a CUDA bf16 [n, d] tensor with unit column stride")
+    _need(out, torch.uint8, "out", x.device)
+    n, d = x.shape
+    cap = out.numel() // d
+    if out.numel() != cap * d:
+        raise ValueError("out does not match d")
+    if dst_row is not None:
+        _need(dst_row, torch.int64, "dst_row", x.device)
+    _check(lib().fp4kv_swa_quant_fp8(_ptr(x), n, d, x.stride(0), _ptr(dst_row), _ptr(out), cap,
+                                     _stream(x.device)))
 
 
 def profile_enable(on: bool = True):

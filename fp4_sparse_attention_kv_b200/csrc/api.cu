@@ -313,6 +313,27 @@ fp4kv_status fp4kv_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int32_t d, in
   return ok();
 }
 
+fp4kv_status fp4kv_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int32_t d, int64_t x_row_stride,
+                                 const int64_t* dst_row, uint8_t* out, int64_t cap_rows, void* stream) {
+  if (n_rows < 0 || cap_rows < 0) return fail(FP4KV_ERR_INVALID_ARG, "negative n_rows or cap_rows");
+  if (d % 16 != 0 || d < 16 || d > 1024) return fail(FP4KV_ERR_UNSUPPORTED, "d=%d must be a multiple of 16 in [16, 1024]", d);
+  if (n_rows == 0) return ok();
+  if (!x || !out) return fail(FP4KV_ERR_INVALID_ARG, "null x or out");
+  if (x_row_stride < d || x_row_stride % 8 != 0)
+    return fail(FP4KV_ERR_INVALID_ARG, "x_row_stride=%lld must be >= d and a multiple of 8", (long long)x_row_stride);
+  if (!aligned(x, 16) || !aligned(out, 16))
+    return fail(FP4KV_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  if (!dst_row && n_rows > cap_rows) return fail(FP4KV_ERR_INVALID_ARG, "n_rows > cap_rows with dst_row == NULL");
+  cudaError_t e;
+  {
+    prof::Scope ps(0, static_cast<cudaStream_t>(stream));
+    e = fp4kv::launch_swa_quant_fp8(x, n_rows, d, x_row_stride, dst_row, out, cap_rows, num_sms(),
+                                    static_cast<cudaStream_t>(stream));
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "swa_quant_fp8");
+  return ok();
+}
+
 fp4kv_status fp4kv_indexer_scores(const void* q, const float* w, int32_t H_I, const void* keys,
                                   int32_t key_dtype, const float* key_scale, int64_t cap,
                                   const int32_t* seq_lens, int32_t B, float* out_score,
@@ -439,11 +460,11 @@ fp4kv_status fp4kv_hier_pool_select(const void* q, const float* w, int32_t H_I, 
                      static_cast<cudaStream_t>(stream));
 }
 
-fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, int32_t d,
-                                      const uint8_t* packed, const uint8_t* scales, int64_t cap,
-                                      const int32_t* seq_lens, const int32_t* idx, int32_t top_k,
-                                      float sm_scale, float* out, float* lse, void* ws,
-                                      size_t ws_bytes, void* stream) {
+static fp4kv_status run_attn(const uint16_t* q, int32_t B, int32_t H, int32_t d, const uint8_t* packed,
+                             const uint8_t* scales, int64_t cap, const int32_t* seq_lens,
+                             const int32_t* idx, int32_t top_k, const uint8_t* swa, int32_t n_win,
+                             float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                             void* stream) {
   if (!q || !packed || !scales || !seq_lens || !idx || !out || !ws)
     return fail(FP4KV_ERR_INVALID_ARG, "null pointer argument");
   if (B < 1 || B > 65535) return fail(FP4KV_ERR_UNSUPPORTED, "B=%d outside [1, 65535]", B);
@@ -470,6 +491,8 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
   p.seq_lens = seq_lens;
   p.idx = idx;
   p.top_k = top_k;
+  p.swa = swa;
+  p.n_win = n_win;
   p.sm_scale = sm_scale;
   p.out = out;
   p.lse = lse;
@@ -484,6 +507,27 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
   }
   if (e != cudaSuccess) return cuda_fail(e, "sparse_attn_decode");
   return ok();
+}
+
+fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, int32_t d,
+                                      const uint8_t* packed, const uint8_t* scales, int64_t cap,
+                                      const int32_t* seq_lens, const int32_t* idx, int32_t top_k,
+                                      float sm_scale, float* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  return run_attn(q, B, H, d, packed, scales, cap, seq_lens, idx, top_k, nullptr, 0, sm_scale, out, lse,
+                  ws, ws_bytes, stream);
+}
+
+fp4kv_status fp4kv_sparse_swa_attn_decode(const uint16_t* q, int32_t B, int32_t H, int32_t d,
+                                          const uint8_t* packed, const uint8_t* scales, int64_t cap,
+                                          const int32_t* seq_lens, const int32_t* idx, int32_t top_k,
+                                          const uint8_t* swa, int32_t n_win, float sm_scale, float* out,
+                                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!swa) return fail(FP4KV_ERR_INVALID_ARG, "null swa");
+  if (n_win < 1 || n_win > 128) return fail(FP4KV_ERR_UNSUPPORTED, "n_win=%d outside [1, 128]", n_win);
+  if (!aligned(swa, 16)) return fail(FP4KV_ERR_INVALID_ARG, "swa must be 16-byte aligned");
+  return run_attn(q, B, H, d, packed, scales, cap, seq_lens, idx, top_k, swa, n_win, sm_scale, out, lse,
+                  ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------------------

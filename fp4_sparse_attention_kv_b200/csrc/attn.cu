@@ -36,6 +36,9 @@
 //    once at the end, when O^T is staged in shared memory and leaves in one bulk store.
 //  Per-chunk barriers let the next tile's dequantization overlap the current tile's P.V.
 //  Chunks of the index list go to different CTAs; k_attn_combine merges their partials.
+//  * With a sliding window (the pages' SWA branch, its KV kept in FP8), the last chunk's CTA
+//    runs one more tile: the window's E4M3 rows (exact in fp16), in the same softmax as the
+//    selected rows, so the window and the sparse selection share one normalisation.
 // Every mbarrier wait is bounded in time. Decisions that lead to a named barrier are made
 // uniform across the softmax warps by a barrier vote, so a timed-out wait cannot strand a
 // warp; on timeout the kernel sets a status bit and winds down.
@@ -245,6 +248,61 @@ FP4KV_DEV bool load_dequant(uint8_t* smem, uint64_t* bars, const uint8_t* packed
   return ok;
 }
 
+// The window tile's rows: E4M3 codes, one byte per dim (row pos of this sequence's window
+// rows), with load_dequant's lane mapping and V_hat layout (lane j of a quad converts dims
+// [128 cp + 32 j, +32) of its row for chunk pair cp). The window tile runs once per CTA, so
+// each chunk pair's bytes are loaded just before they are converted.
+template <int NG>
+FP4KV_DEV bool load_dequant_win(uint8_t* smem, uint64_t* bars, const uint8_t* win_b,
+                                const int32_t (&pos)[NG], int row0, int t) {
+  const int lane = threadIdx.x & 31, qd = lane >> 2, j = lane & 3;
+  bool ok = true;
+#pragma unroll
+  for (int cp = 0; cp < 4; ++cp) {
+    uint4 c8[NG][2];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      if (pos[i] >= 0) {
+        const uint8_t* src = win_b + int64_t(pos[i]) * kD + 128 * cp + 32 * j;
+        c8[i][0] = ld_nc_v4(src);
+        c8[i][1] = ld_nc_v4(src + 16);
+      } else {
+        c8[i][0] = c8[i][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_VFREE + 2 * cp], (t & 1) ^ 1) &&
+                                           mbar_wait_timed(&bars[B_VFREE + 2 * cp + 1], (t & 1) ^ 1)))
+      ok = false;
+    if (!ok) continue;
+    const int jc = 2 * cp + (j >> 1);  // chunk of this lane's 32 dims
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      const int r = row0 + 8 * i + qd;
+      uint8_t* vrow = smem + kOffV + jc * kVChunkBytes + r * 128;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int uu = (j & 2) ? (k ^ 2) : k;  // staggered as in load_dequant
+        const uint4 h = (uu >> 1) ? c8[i][1] : c8[i][0];  // (selects: no local-memory indexing)
+        const uint32_t w0 = (uu & 1) ? h.z : h.x, w1 = (uu & 1) ? h.w : h.y;  // dims [8 uu, +8)
+        uint4 o;
+        o.x = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 & 0xffffu));
+        o.y = e4m3x2_to_f16x2(static_cast<uint16_t>(w0 >> 16));
+        o.z = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 & 0xffffu));
+        o.w = e4m3x2_to_f16x2(static_cast<uint16_t>(w1 >> 16));
+        const int unit = 4 * (j & 1) + uu;
+        *reinterpret_cast<uint4*>(vrow + ((unit ^ (r & 7)) << 4)) = o;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bars[B_VREADY + 2 * cp]);
+      mbar_arrive(&bars[B_VREADY + 2 * cp + 1]);
+    }
+  }
+  return ok;
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled operand layouts need 1 KiB alignment
@@ -271,8 +329,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   if (len > p.cap) len = p.cap;
   const int e_begin = int(int64_t(p.top_k) * chunk / n_chunks);
   const int e_end = int(int64_t(p.top_k) * (chunk + 1) / n_chunks);
-  const int n_tiles = (e_end - e_begin + kTile - 1) / kTile;
+  const int n_sel_tiles = (e_end - e_begin + kTile - 1) / kTile;
+  // the last chunk's CTA also attends over the sliding window: one more tile, after the
+  // selected ones, whose rows are the window slots [0, min(n_win, len))
+  const bool has_win = p.swa != nullptr && chunk == n_chunks - 1;
+  const int n_tiles = n_sel_tiles + (has_win ? 1 : 0);
+  const int n_win_rows = has_win ? int(min(int64_t(p.n_win), len)) : 0;
   const int32_t* idx = p.idx + int64_t(b) * p.top_k;
+  const uint8_t* win_b = has_win ? p.swa + int64_t(b) * p.n_win * kD : nullptr;
+  // cache position (selected tiles) or window slot (window tile) of row `row` of tile tt;
+  // -1 for none
+  auto tile_pos = [&](int tt, int row) -> int32_t {
+    if (tt < n_sel_tiles) {
+      const int je = e_begin + tt * kTile + row;
+      return je < e_end ? idx[je] : -1;
+    }
+    return (tt < n_tiles && row < n_win_rows) ? row : -1;
+  };
 
   if (tid == 0) {
     for (int j = 0; j < kChunks; ++j) {
@@ -310,10 +383,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     griddep_wait();  // the index list comes from the preceding kernel on the stream
     int32_t pos_next[2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int je = e_begin + row0 + 8 * i + qd;
-      pos_next[i] = je < e_end ? idx[je] : -1;
-    }
+    for (int i = 0; i < 2; ++i) pos_next[i] = tile_pos(0, row0 + 8 * i + qd);
     for (int t = 0; t < n_tiles && !*s_abort; ++t) {
       // Tile t's rows are loaded only once the softmax warps have written tile t - 1's
       // probabilities: TMEM and shared-memory accesses queue behind the global loads the
@@ -327,10 +397,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         pos[i] = (pos_next[i] >= 0 && pos_next[i] < len) ? pos_next[i] : -1;
-        const int jn = e_begin + (t + 1) * kTile + row0 + 8 * i + qd;  // one tile ahead
-        pos_next[i] = jn < e_end ? idx[jn] : -1;
+        pos_next[i] = tile_pos(t + 1, row0 + 8 * i + qd);  // one tile ahead
       }
-      if (!load_dequant<2>(smem, bars, packed_b, scales_b, pos, row0, t)) {
+      const bool ld_ok = (t == n_sel_tiles) ? load_dequant_win<2>(smem, bars, win_b, pos, row0, t)
+                                            : load_dequant<2>(smem, bars, packed_b, scales_b, pos, row0, t);
+      if (!ld_ok) {
         if (lane == 0) fail_wait(p, s_abort);
         break;
       }
@@ -466,28 +537,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     const int h0 = 32 * (warp >> 2);  // first of this thread's 32 heads
     const int e = 32 * q4 + lane;     // tile row (entry) / output dim within a dim tile
     const uint32_t lane_addr = uint32_t(32 * q4) << 16;
-    // bit t: this thread's entry of tile t holds a valid position (at most 32 tiles)
     griddep_wait();  // the index list comes from the preceding kernel on the stream
     // this warp also loads and dequantizes tile rows 64 + 8 warp + lane / 4 of every tile
     const int drow = 64 + 8 * warp;
     const uint8_t* packed_b = p.packed + int64_t(b) * p.cap * (kD / 2);
     const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
-    auto dq_pos = [&](int tt) -> int32_t {
-      const int je = e_begin + tt * kTile + drow + (lane >> 2);
-      return (tt < n_tiles && je < e_end) ? idx[je] : -1;
-    };
+    auto dq_pos = [&](int tt) -> int32_t { return tile_pos(tt, drow + (lane >> 2)); };
     int32_t dpos_next = dq_pos(0);
-    uint32_t vmask = 0;
+    uint64_t vmask = 0;  // bit t: this thread's entry of tile t is valid (at most 33 tiles)
     for (int t0 = 0; t0 < n_tiles; t0 += 8) {
       int32_t pv[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int je = e_begin + (t0 + k) * kTile + e;
-        pv[k] = t0 + k < n_tiles && je < e_end ? idx[je] : -1;
-      }
+      for (int k = 0; k < 8; ++k) pv[k] = tile_pos(t0 + k, e);
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        if (pv[k] >= 0 && pv[k] < len) vmask |= 1u << (t0 + k);
+        if (pv[k] >= 0 && pv[k] < len) vmask |= uint64_t(1) << (t0 + k);
     }
     float lsum[32];  // per-head running row sums over this thread's entries
 #pragma unroll
@@ -497,7 +561,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     if (n_tiles > 0) {
       int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
       dpos_next = dq_pos(1);
-      dq_fail = !load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0);
+      dq_fail = !(n_sel_tiles == 0 ? load_dequant_win<1>(smem, bars, win_b, dp, drow, 0)
+                                    : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0));
     }
     for (int t = 0; t < n_tiles; ++t) {
       const int u = t & 1;
@@ -600,7 +665,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       if (t + 1 < n_tiles) {  // this warp's rows of the next tile, as P.V(t) frees V_hat
         int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
         dpos_next = dq_pos(t + 2);
-        dq_fail = !load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1);
+        dq_fail = !(t + 1 == n_sel_tiles ? load_dequant_win<1>(smem, bars, win_b, dp, drow, t + 1)
+                                         : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1));
       }
     }
     // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----

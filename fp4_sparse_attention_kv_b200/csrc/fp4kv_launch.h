@@ -9,6 +9,9 @@ namespace fp4kv {
 cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
                                 const int64_t* dst_row, uint8_t* packed, uint8_t* scales,
                                 int64_t cap_rows, int num_sms, cudaStream_t stream);
+cudaError_t launch_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
+                                 const int64_t* dst_row, uint8_t* out, int64_t cap_rows, int num_sms,
+                                 cudaStream_t stream);
 
 // ----------------------------------------------------------------------------------------
 // Indexer scoring (Full scan or pool gather), fused with the first-level histogram of the
@@ -81,11 +84,15 @@ struct AttnParams {
   const int32_t* seq_lens;
   const int32_t* idx;       // [B][top_k]
   int top_k;
+  // nullable: the sliding window's E4M3 rows [B][n_win][d] (ring slot = position % n_win),
+  // attended in the same softmax as the selected rows by one extra chunk CTA (the last)
+  const uint8_t* swa;
+  int n_win;
   float sm_scale;
   float* out;               // [B][H][d]
   float* lse;               // nullable [B][H]
   // split over chunks of the top_k list; partials merged by a combine kernel
-  int n_chunks;
+  int n_chunks;             // chunks of the index list, plus the window's chunk when swa != nullptr
   float* part_o;            // [B][n_hg][n_chunks][64][d]
   float* part_ml;           // [B][n_hg][n_chunks][64][2]
   uint32_t* status;

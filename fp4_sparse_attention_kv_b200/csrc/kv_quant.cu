@@ -1,4 +1,5 @@
-// kv_quant_fp4: quantize-on-write of bf16 KV rows into packed E2M1 codes + E4M3 scales.
+// kv_quant_fp4: quantize-on-write of bf16 KV rows into packed E2M1 codes + E4M3 scales;
+// swa_quant_fp8: the sliding-window KV's write, bf16 rows into E4M3 codes.
 //
 // Method: [PyTorchKR] "DeepSeek-V4.1-Flash, KV 캐시를 토큰당 890바이트로 줄이고 …", section
 // "890바이트를 만든 나머지 절반, FP4 KV 캐시와 지속 캐시 재설계": the main KV is kept as E2M1
@@ -102,7 +103,58 @@ __global__ void __launch_bounds__(256) k_kv_quant_fp4(const uint16_t* __restrict
   }
 }
 
+// SWA KV write: bf16 rows -> E4M3 codes (round to nearest even, saturating at +-448), one
+// byte per channel ([PyTorchKR] FP4 KV section: the quantization-sensitive SWA KV stays
+// FP8). One warp per row, 16 channels per lane and step: 32 B read, 16 B written per lane.
+__global__ void __launch_bounds__(256) k_swa_quant_fp8(const uint16_t* __restrict__ x, int64_t n_rows,
+                                                       int d, int64_t x_stride,
+                                                       const int64_t* __restrict__ dst_row,
+                                                       uint8_t* __restrict__ out, int64_t cap_rows) {
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = warp; r < n_rows; r += nwarps) {
+    const int64_t dst = dst_row ? dst_row[r] : r;
+    if (dst < 0 || dst >= cap_rows) continue;
+    const uint16_t* xr = x + r * x_stride;
+    uint8_t* orow = out + dst * d;
+    for (int c = 16 * lane; c < d; c += 16 * 32) {
+      const uint4 v0 = ld_stream_v4(xr + c);
+      const uint4 v1 = ld_stream_v4(xr + c + 8);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint16_t lo, hi;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo)
+            : "f"(bf16_bits_to_f32(w[2 * k] >> 16)), "f"(bf16_bits_to_f32(w[2 * k] & 0xffffu)));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi)
+            : "f"(bf16_bits_to_f32(w[2 * k + 1] >> 16)), "f"(bf16_bits_to_f32(w[2 * k + 1] & 0xffffu)));
+        // the sign of x is kept (a negative value that rounds to zero is 0x80)
+        const uint32_t w0 = w[2 * k], w1 = w[2 * k + 1];
+        o[k] = (uint32_t(lo) | ((w0 >> 8) & 0x80u) | ((w0 >> 16) & 0x8000u)) |
+               ((uint32_t(hi) | ((w1 >> 8) & 0x80u) | ((w1 >> 16) & 0x8000u)) << 16);
+      }
+      *reinterpret_cast<uint4*>(orow + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
+                                 const int64_t* dst_row, uint8_t* out, int64_t cap_rows, int num_sms,
+                                 cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const int threads = 256;
+  int64_t blocks = (n_rows + 7) / 8;
+  const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > max_blocks) blocks = max_blocks;
+  k_swa_quant_fp8<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, n_rows, d, x_stride, dst_row, out,
+                                                                          cap_rows);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
                                 const int64_t* dst_row, uint8_t* packed, uint8_t* scales,

@@ -194,6 +194,32 @@ fp4kv_status fp4kv_sparse_attn_decode(const uint16_t* q, int32_t B, int32_t H, i
                                       float sm_scale, float* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* sparse_swa_attn_decode -- fp4kv_sparse_attn_decode plus the sliding-window branch
+ * ([PyTorchKR] "왜 KV 캐시가 에이전트 시대의 병목이 되었나": a global branch over the main KV
+ * and a sliding-window (SWA) branch over a local KV of the last n_win tokens; FP4 KV
+ * section: the SWA KV stays FP8). The window's rows join the selected rows in ONE softmax
+ * (this library's reading of how the two branches combine): out = sum over the selected
+ * entries and the window rows of softmax(sm_scale * q . v) * v, lse over both sets.
+ * swa   : E4M3 codes [B][n_win][d] (fp4kv_swa_quant_fp8 writes them), 16-byte aligned; a ring
+ *         buffer: position pos lives in slot pos % n_win, and slots [0, min(n_win,
+ *         seq_lens[b])) are the window of sequence b (the caller keeps them current).
+ * n_win : 1 .. 128. Other arguments and the workspace as fp4kv_sparse_attn_decode.
+ * Positions that are both selected and in the window count twice. */
+fp4kv_status fp4kv_sparse_swa_attn_decode(const uint16_t* q, int32_t B, int32_t H, int32_t d,
+                                          const uint8_t* packed, const uint8_t* scales, int64_t cap,
+                                          const int32_t* seq_lens, const int32_t* idx, int32_t top_k,
+                                          const uint8_t* swa, int32_t n_win, float sm_scale, float* out,
+                                          float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* swa_quant_fp8 -- the SWA KV's write: bf16 rows x [n_rows][d] (row stride x_row_stride
+ * elements, a multiple of 8) to E4M3 codes, round to nearest even, saturating at +-448
+ * ([PyTorchKR] FP4 KV section: the quantization-sensitive SWA KV stays FP8; a direct cast
+ * without a scale is this library's reading). out: [cap_rows][d] bytes; row i goes to
+ * dst_row[i] (nullable: i), rows outside [0, cap_rows) are skipped. d % 16 == 0, d <= 1024;
+ * x and out 16-byte aligned. */
+fp4kv_status fp4kv_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int32_t d, int64_t x_row_stride,
+                                 const int64_t* dst_row, uint8_t* out, int64_t cap_rows, void* stream);
+
 /* indexer_topk_noalloc -- fp4kv_indexer_topk without a caller workspace. (The pages have
  * no counterpart: this is an integration aid.) For callers that cannot allocate device
  * memory: code inside a host runtime that owns all device memory (a serving engine with a

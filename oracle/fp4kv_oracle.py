@@ -318,6 +318,25 @@ def sparse_attn_decode_rows(q, v_hat, sm_scale: float):
     return (e @ v) / den, m[:, 0] + np.log(den[:, 0])
 
 
+def swa_quant_fp8(x) -> np.ndarray:
+    """The sliding-window KV's storage ([PyTorchKR] FP4 KV section: the SWA KV stays FP8):
+    each value as an E4M3 code, nearest value with ties to the even code, saturating at
+    448, the sign of x kept (a negative value that rounds to zero is 0x80). x: exact bf16
+    values as fp64, any shape; returns uint8 codes of the same shape."""
+    x = np.asarray(x, dtype=np.float64)
+    mag = e4m3_round_sat(np.abs(x))
+    return ((np.signbit(x).astype(np.int64) << 7) | mag).astype(np.uint8)
+
+
+def sparse_swa_attn_decode_rows(q, v_sel, v_win, sm_scale: float):
+    """Attention of the sparse branch and the sliding-window branch in one softmax: the
+    selected rows v_sel [J, d] and the window rows v_win [W, d] (dequantized values) are
+    attended together, as one set of J + W rows. Returns (o [H, d], lse [H])."""
+    v_sel = np.asarray(v_sel, dtype=np.float64).reshape(-1, np.asarray(q).shape[-1])
+    v_win = np.asarray(v_win, dtype=np.float64).reshape(-1, np.asarray(q).shape[-1])
+    return sparse_attn_decode_rows(q, np.concatenate([v_sel, v_win], axis=0), sm_scale)
+
+
 def fp8_e4m3_to_f64(codes) -> np.ndarray:
     """FP8 E4M3 indexer keys / queries (uint8 codes) -> exact fp64 values."""
     return e4m3_decode(np.asarray(codes, dtype=np.uint8))

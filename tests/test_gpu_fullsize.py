@@ -134,3 +134,29 @@ def test_csa2_decoder_step_at_full_size(fk):
         _attn_check(seed, 0, b, wl.q[l][b], wl.idx[l // G][b].cpu().numpy(), cap, new_row,
                     wl.out[l][b].cpu().numpy(), wl.lse[l][b].cpu().numpy(), f"CSA2 layer {l + 1} attention")
     _new_row_check(wl, b, wl.packed, wl.scales, wl.x_new, "CSA2 new row")
+
+
+@pytest.mark.timeout(900)
+def test_decode_step_with_sliding_window_at_full_size(fk):
+    cfg = bench.CONFIGS["decode32_swa"]
+    wl = bench.DecodeWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    idx = wl.idx.cpu().numpy()
+    out, lse = wl.out.cpu().numpy(), wl.lse.cpu().numpy()
+    seed, cap, nw = cfg["seed"], wl.cap, wl.n_win
+    for b in (0, 31):
+        sc = P.oracle_scores_seq(wl.qi[b], wl.w[b], wl.keys[b], cap)
+        P.check_topk(idx[b], sc, np.arange(cap), wl.K, f"top-K b={b}")
+        sel = idx[b][(idx[b] >= 0) & (idx[b] < cap)]
+        rows = P.kv_rows_host(seed, 0, b, sel, D)
+        rows[sel == cap - 1] = P.to_f64(wl.x_new[b].cpu())
+        v_sel = O.kv_dequant_fp4(*O.kv_quant_fp4(rows))
+        # the window: positions cap - nw .. cap - 1, the last one the row this step wrote
+        wrows = P.kv_rows_host(seed, bench.SWA_LAYER, b, np.arange(cap - nw, cap), D)
+        wrows[-1] = P.to_f64(wl.x_swa_new[b].cpu())
+        v_win = O.e4m3_decode(O.swa_quant_fp8(wrows))
+        ro, rl = O.sparse_swa_attn_decode_rows(P.to_f64(wl.q[b].cpu()), v_sel, v_win, 1.0)
+        P.check_attn(out[b], lse[b], ro, rl, f"attention + window b={b}")
+        slot = (cap - 1) % nw
+        assert np.array_equal(wl.swa[b, slot].cpu().numpy(), O.swa_quant_fp8(wrows[-1])), "window write"

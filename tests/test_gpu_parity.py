@@ -495,3 +495,99 @@ def test_fp4_indexer_rejects_odd_sizes(fk):
     k_even.buf.zero_()
     with pytest.raises(fk.Fp4kvError):
         fk.indexer_topk(q_odd, w[:, :31].contiguous(), k_even, lens, 8)
+
+
+# ----------------------------------------------------------------------------------------
+# Sliding-window branch: FP8 window rows in the same softmax as the selected FP4 rows
+# ----------------------------------------------------------------------------------------
+
+SWA_LAYER = 700  # generator stream of the window rows (a different projection than the main KV)
+
+
+def test_swa_quant_fp8_bit_exact_over_all_finite_bf16(fk):
+    bits = np.arange(0, 0x7F80, dtype=np.uint16)
+    v = O.bf16_bits_to_f64(bits)
+    x = np.concatenate([v, -v])
+    x = np.concatenate([x, np.zeros((-x.size) % 512)]).reshape(-1, 512)
+    xd = _bf16_from_f64(x).to(DEV)
+    out = torch.empty(x.shape, dtype=torch.uint8, device=DEV)
+    fk.swa_quant_fp8(xd, out)
+    assert np.array_equal(out.cpu().numpy(), O.swa_quant_fp8(x))
+    # scattered rows (dst_row), rows outside the buffer skipped
+    dst = torch.tensor([3, -1, 0, 10 ** 9], dtype=torch.int64, device=DEV)
+    out2 = torch.zeros((4, 512), dtype=torch.uint8, device=DEV)
+    fk.swa_quant_fp8(xd[:4].contiguous(), out2, dst_row=dst)
+    want = np.zeros((4, 512), dtype=np.uint8)
+    want[3], want[0] = O.swa_quant_fp8(x[0]), O.swa_quant_fp8(x[2])
+    assert np.array_equal(out2.cpu().numpy(), want)
+
+
+def _swa_case(fk, seed, B, cap, H, lens, idx_np, n_win, sm_scale=1.0):
+    """Selected FP4 rows + the window of the last min(n_win, len) positions (E4M3, ring slot
+    = position % n_win), one softmax; checked against the oracle per sequence."""
+    d = 512
+    x = P.kv_rows_dev(seed, 0, B, cap, d, DEV)
+    packed = torch.empty((B, cap, d // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((B, cap, d // 16), dtype=torch.uint8, device=DEV)
+    fk.kv_quant_fp4(x.view(B * cap, d), packed.view(B * cap, d // 2), scales.view(B * cap, d // 16))
+    del x
+    swa = torch.zeros((B, n_win, d), dtype=torch.uint8, device=DEV)
+    win_pos = []
+    for b in range(B):
+        L = lens[b]
+        pos = np.arange(max(0, L - n_win), L, dtype=np.int64)
+        win_pos.append(pos)
+        if pos.size:
+            rows = synth.kv_rows(seed, SWA_LAYER, b, torch.as_tensor(pos, device=DEV), d)
+            dst = torch.as_tensor(b * n_win + pos % n_win, device=DEV)
+            fk.swa_quant_fp8(rows, swa.view(B * n_win, d), dst_row=dst)
+    q = synth.attn_query(seed, 0, B, H, d, device=DEV)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    idx = torch.tensor(idx_np, dtype=torch.int32, device=DEV)
+    out, lse = fk.sparse_attn_decode(q, packed, scales, lens_t, idx, sm_scale, swa=swa)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    qh = P.to_f64(q.cpu())
+    for b in range(B):
+        sel = np.asarray(idx_np[b])
+        sel = sel[(sel >= 0) & (sel < lens[b])]
+        v_sel = np.zeros((0, d))
+        if sel.size:
+            pk, sc = O.kv_quant_fp4(P.kv_rows_host(seed, 0, b, sel, d))
+            v_sel = O.kv_dequant_fp4(pk, sc)
+        v_win = O.e4m3_decode(O.swa_quant_fp8(P.kv_rows_host(seed, SWA_LAYER, b, win_pos[b], d)))
+        if sel.size + win_pos[b].size:
+            ro, rl = O.sparse_swa_attn_decode_rows(qh[b], v_sel, v_win.reshape(-1, d), sm_scale)
+        else:
+            ro, rl = np.zeros((H, d)), np.full(H, -np.inf)
+        P.check_attn(out[b], lse[b], ro, rl, f"b={b}")
+    return out, lse
+
+
+def _rand_idx(rng, B, top_k, lens, pad_frac=0.1):
+    idx = np.full((B, top_k), -1, dtype=np.int64)
+    for b in range(B):
+        m = min(top_k, lens[b])
+        idx[b, :m] = np.sort(rng.choice(lens[b], size=m, replace=False))
+        holes = rng.random(top_k) < pad_frac
+        idx[b, holes] = -1
+    return idx
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=31, B=3, cap=5000, H=64, top_k=300, lens=[5000, 100, 60], n_win=128),
+    dict(seed=32, B=2, cap=9000, H=16, top_k=2048, lens=[9000, 8999], n_win=128),
+    dict(seed=33, B=2, cap=3000, H=64, top_k=512, lens=[3000, 40], n_win=64),
+    dict(seed=34, B=160, cap=300, H=16, top_k=128, lens=[300] * 160, n_win=128),  # one chunk per sequence
+])
+def test_sparse_swa_attention_matches_oracle(fk, case):
+    rng = np.random.default_rng(case["seed"])
+    idx = _rand_idx(rng, case["B"], case["top_k"], case["lens"])
+    _swa_case(fk, case["seed"], case["B"], case["cap"], case["H"], case["lens"], idx, case["n_win"])
+
+
+def test_sparse_swa_attention_window_only_and_nothing(fk):
+    B, cap, H = 2, 1000, 64
+    idx = np.full((B, 256), -1, dtype=np.int64)  # no selected entry: the window alone
+    _swa_case(fk, 35, B, cap, H, [1000, 77], idx, 128)
+    out, lse = _swa_case(fk, 36, 1, cap, H, [0], np.full((1, 128), -1, dtype=np.int64), 128)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))

@@ -234,3 +234,50 @@ def test_fp4_indexer_one_nonzero_dim_closed_form():
                           * O.e4m3_decode(O.e4m3_round_sat(abs(kv) / 6.0)))
         got = O.indexer_scores(O.indexer_fp4_values(q), [0.75], O.indexer_fp4_values(k))
         assert got[0] == np.float32(want), (qv, kv, got[0], want)
+
+
+# ----------------------------------------------------------------------------------------
+# Sliding-window branch (FP8 rows in the same softmax as the selected rows)
+# ----------------------------------------------------------------------------------------
+
+def test_swa_quant_fp8_sign_saturation_and_brute_force():
+    """Codes are the nearest E4M3 value (ties to the even code, |x| > 448 -> 448) with the
+    sign of x, checked against a plain search over all 127 non-negative values."""
+    vals = [float(O.e4m3_decode(c)) for c in range(127)]
+    rng = np.random.default_rng(7)
+    xs = np.concatenate([rng.normal(0, 3, 400), rng.normal(0, 300, 100), [0.0, -0.0, 1e-9, -1e-9, 448, 449, 1e4, -1e4],
+                         [(vals[i] + vals[i + 1]) / 2 for i in range(126)]])  # every midpoint
+    for x in xs:
+        a = abs(float(x))
+        if a >= 448:
+            want = 0x7E
+        else:
+            d = [abs(a - v) for v in vals]
+            best = min(d)
+            ties = [c for c in range(127) if d[c] == best]
+            want = ties[0] if len(ties) == 1 else next(c for c in ties if c % 2 == 0)
+        want |= 0x80 if math.copysign(1.0, float(x)) < 0 else 0
+        assert int(O.swa_quant_fp8(np.float64(x))) == want, x
+
+
+def _lse_merge(o1, l1, o2, l2):
+    m = np.maximum(l1, l2)
+    w1, w2 = np.exp(l1 - m), np.exp(l2 - m)
+    return (w1[:, None] * o1 + w2[:, None] * o2) / (w1 + w2)[:, None], m + np.log(w1 + w2)
+
+
+def test_swa_one_softmax_equals_the_lse_merge_of_the_two_branches():
+    rng = np.random.default_rng(8)
+    q = rng.normal(0, 0.05, (6, 64))
+    sel = rng.normal(0, 1, (20, 64))
+    win = rng.normal(0, 1, (9, 64))
+    o, lse = O.sparse_swa_attn_decode_rows(q, sel, win, 1.3)
+    o1, l1 = O.sparse_attn_decode_rows(q, sel, 1.3)
+    o2, l2 = O.sparse_attn_decode_rows(q, win, 1.3)
+    om, lm = _lse_merge(o1, l1, o2, l2)
+    assert np.allclose(o, om, rtol=1e-12, atol=1e-12) and np.allclose(lse, lm, rtol=1e-12, atol=1e-12)
+    # an empty selection leaves the window's dense attention, an empty window the sparse one
+    ow, lw = O.sparse_swa_attn_decode_rows(q, np.zeros((0, 64)), win, 1.3)
+    assert np.allclose(ow, o2) and np.allclose(lw, l2)
+    os_, ls = O.sparse_swa_attn_decode_rows(q, sel, np.zeros((0, 64)), 1.3)
+    assert np.allclose(os_, o1) and np.allclose(ls, l1)
