@@ -42,6 +42,8 @@
 // Every mbarrier wait is bounded in time. Decisions that lead to a named barrier are made
 // uniform across the softmax warps by a barrier vote, so a timed-out wait cannot strand a
 // warp; on timeout the kernel sets a status bit and winds down.
+#include <type_traits>
+
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
 #include "fp4kv_sm100.cuh"
@@ -303,6 +305,9 @@ FP4KV_DEV bool load_dequant_win(uint8_t* smem, uint64_t* bars, const uint8_t* wi
   return ok;
 }
 
+// kWin: with the sliding-window tile (a separate instantiation, so that the plain sparse
+// attention keeps its code size and registers).
+template <bool kWin>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled operand layouts need 1 KiB alignment
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   const int n_sel_tiles = (e_end - e_begin + kTile - 1) / kTile;
   // the last chunk's CTA also attends over the sliding window: one more tile, after the
   // selected ones, whose rows are the window slots [0, min(n_win, len))
-  const bool has_win = p.swa != nullptr && chunk == n_chunks - 1;
+  const bool has_win = kWin && chunk == n_chunks - 1;
   const int n_tiles = n_sel_tiles + (has_win ? 1 : 0);
   const int n_win_rows = has_win ? int(min(int64_t(p.n_win), len)) : 0;
   const int32_t* idx = p.idx + int64_t(b) * p.top_k;
@@ -340,9 +345,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   // cache position (selected tiles) or window slot (window tile) of row `row` of tile tt;
   // -1 for none
   auto tile_pos = [&](int tt, int row) -> int32_t {
-    if (tt < n_sel_tiles) {
+    if (!kWin || tt < n_sel_tiles) {
       const int je = e_begin + tt * kTile + row;
-      return je < e_end ? idx[je] : -1;
+      return (tt < n_sel_tiles && je < e_end) ? idx[je] : -1;
     }
     return (tt < n_tiles && row < n_win_rows) ? row : -1;
   };
@@ -399,8 +404,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         pos[i] = (pos_next[i] >= 0 && pos_next[i] < len) ? pos_next[i] : -1;
         pos_next[i] = tile_pos(t + 1, row0 + 8 * i + qd);  // one tile ahead
       }
-      const bool ld_ok = (t == n_sel_tiles) ? load_dequant_win<2>(smem, bars, win_b, pos, row0, t)
-                                            : load_dequant<2>(smem, bars, packed_b, scales_b, pos, row0, t);
+      const bool ld_ok = (kWin && t == n_sel_tiles) ? load_dequant_win<2>(smem, bars, win_b, pos, row0, t)
+                                                    : load_dequant<2>(smem, bars, packed_b, scales_b, pos, row0, t);
       if (!ld_ok) {
         if (lane == 0) fail_wait(p, s_abort);
         break;
@@ -544,14 +549,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     const uint8_t* scales_b = p.scales + int64_t(b) * p.cap * (kD / kGroup);
     auto dq_pos = [&](int tt) -> int32_t { return tile_pos(tt, drow + (lane >> 2)); };
     int32_t dpos_next = dq_pos(0);
-    uint64_t vmask = 0;  // bit t: this thread's entry of tile t is valid (at most 33 tiles)
+    // bit t: this thread's entry of tile t is valid (at most 32 tiles, 33 with the window)
+    using VMask = typename std::conditional<kWin, uint64_t, uint32_t>::type;
+    VMask vmask = 0;
     for (int t0 = 0; t0 < n_tiles; t0 += 8) {
       int32_t pv[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) pv[k] = tile_pos(t0 + k, e);
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        if (pv[k] >= 0 && pv[k] < len) vmask |= uint64_t(1) << (t0 + k);
+        if (pv[k] >= 0 && pv[k] < len) vmask |= VMask(1) << (t0 + k);
     }
     float lsum[32];  // per-head running row sums over this thread's entries
 #pragma unroll
@@ -561,8 +568,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     if (n_tiles > 0) {
       int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
       dpos_next = dq_pos(1);
-      dq_fail = !(n_sel_tiles == 0 ? load_dequant_win<1>(smem, bars, win_b, dp, drow, 0)
-                                    : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0));
+      dq_fail = !((kWin && n_sel_tiles == 0) ? load_dequant_win<1>(smem, bars, win_b, dp, drow, 0)
+                                              : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0));
     }
     for (int t = 0; t < n_tiles; ++t) {
       const int u = t & 1;
@@ -665,8 +672,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       if (t + 1 < n_tiles) {  // this warp's rows of the next tile, as P.V(t) frees V_hat
         int32_t dp[1] = {(dpos_next >= 0 && dpos_next < len) ? dpos_next : -1};
         dpos_next = dq_pos(t + 2);
-        dq_fail = !(t + 1 == n_sel_tiles ? load_dequant_win<1>(smem, bars, win_b, dp, drow, t + 1)
-                                         : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1));
+        dq_fail = !((kWin && t + 1 == n_sel_tiles) ? load_dequant_win<1>(smem, bars, win_b, dp, drow, t + 1)
+                                                   : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1));
       }
     }
     // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----
@@ -826,7 +833,8 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t st
   (void)num_sms;
   if (p.B == 0) return cudaSuccess;
   const int n_hg = (p.H + kHeadsPerCta - 1) / kHeadsPerCta;
-  cudaError_t e = cudaFuncSetAttribute(k_sparse_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.swa != nullptr ? k_sparse_attn_tc<true> : k_sparse_attn_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAttn));
   if (e != cudaSuccess) return e;
   // Both kernels are programmatic dependents of the kernel before them on the stream: their
@@ -843,7 +851,7 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t st
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k_sparse_attn_tc, p);
+  e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e != cudaSuccess) return e;
   if (p.n_chunks == 1) return cudaSuccess;
   cfg.gridDim = dim3(kHeadsPerCta, n_hg, p.B);
