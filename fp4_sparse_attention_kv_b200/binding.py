@@ -49,6 +49,9 @@ SIGNATURES = [
     ("fp4kv_sparse_swa_attn_decode", ctypes.c_int,
      [_P, _I32, _I32, _I32, _P, _P, _I64, _P, _P, _I32, _P, _I32, _F32, _P, _P, _P, _SZ, _P]),
     ("fp4kv_swa_quant_fp8", ctypes.c_int, [_P, _I64, _I32, _I64, _P, _P, _I64, _P]),
+    ("fp4kv_topk_merge", ctypes.c_int, [_P, _P, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32, _I32, _I32, _P,
+                                        _P, _P, _P]),
+    ("fp4kv_lse_combine", ctypes.c_int, [_P, _P, _I32, _I32, _I32, _I32, _P, _P, _P]),
 ]
 
 KERNEL_KINDS = ("kv_quant_fp4", "index_score", "topk_select", "sparse_attn")
@@ -374,3 +377,48 @@ def indexer_topk_noalloc(q, w, keys, seq_lens, top_k, pool=None, block_size=8, k
                                             top_k, _ptr(out_idx), _ptr(out_score),
                                             _stream(keys.device)))
     return out_idx
+
+
+def topk_merge(cand_score: torch.Tensor, cand_idx: torch.Tensor, part_base, top_k: int,
+               local_range=None, out_idx=None, out_local=None, out_score=None):
+    """Exact top-K of the union of per-part candidate lists. cand_score fp32 / cand_idx int32
+    [n_parts, B, k_part] (range-local positions, -1 absent); part_base: the first global
+    position of each part's range (host ints). Returns (out_idx [B, top_k] global positions
+    ascending, out_local [B, top_k] positions local to local_range=(lo, hi) or None)."""
+    _need(cand_score, torch.float32, "cand_score")
+    _need(cand_idx, torch.int32, "cand_idx", cand_score.device)
+    R, B, k_part = cand_idx.shape
+    if tuple(cand_score.shape) != (R, B, k_part) or len(part_base) != R:
+        raise ValueError("cand_score / cand_idx must be [n_parts, B, k_part] with one base per part")
+    dev = cand_idx.device
+    if out_idx is None:
+        out_idx = torch.empty((B, top_k), dtype=torch.int32, device=dev)
+    _need(out_idx, torch.int32, "out_idx", dev)
+    lo, hi = (0, 0) if local_range is None else (int(local_range[0]), int(local_range[1]))
+    if local_range is not None and out_local is None:
+        out_local = torch.empty((B, top_k), dtype=torch.int32, device=dev)
+    if out_local is not None:
+        _need(out_local, torch.int32, "out_local", dev)
+    if out_score is not None:
+        _need(out_score, torch.float32, "out_score", dev)
+    bases = (_I32 * R)(*[int(x) for x in part_base])
+    _check(lib().fp4kv_topk_merge(_ptr(cand_score), _ptr(cand_idx), R, k_part, B, bases, top_k, lo, hi,
+                                  _ptr(out_idx), _ptr(out_local), _ptr(out_score), _stream(dev)))
+    return out_idx, out_local
+
+
+def lse_combine(part_out: torch.Tensor, part_lse: torch.Tensor, out=None, lse=None):
+    """Attention over the union of disjoint row sets from the parts: part_out fp32
+    [R, B, H, d], part_lse fp32 [R, B, H]. Returns (out [B, H, d], lse [B, H])."""
+    _need(part_out, torch.float32, "part_out")
+    _need(part_lse, torch.float32, "part_lse", part_out.device)
+    R, B, H, d = part_out.shape
+    if tuple(part_lse.shape) != (R, B, H):
+        raise ValueError("part_lse must be [R, B, H]")
+    dev = part_out.device
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _check(lib().fp4kv_lse_combine(_ptr(part_out), _ptr(part_lse), R, B, H, d, _ptr(out), _ptr(lse), _stream(dev)))
+    return out, lse

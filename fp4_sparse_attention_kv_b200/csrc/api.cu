@@ -313,6 +313,51 @@ fp4kv_status fp4kv_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int32_t d, in
   return ok();
 }
 
+fp4kv_status fp4kv_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_parts, int32_t k_part,
+                              int32_t B, const int32_t* part_base, int32_t top_k, int32_t local_lo,
+                              int32_t local_hi, int32_t* out_idx, int32_t* out_local, float* out_score,
+                              void* stream) {
+  if (!cand_score || !cand_idx || !part_base || !out_idx)
+    return fail(FP4KV_ERR_INVALID_ARG, "null cand_score, cand_idx, part_base or out_idx");
+  if (B < 1 || B > 65535) return fail(FP4KV_ERR_UNSUPPORTED, "B=%d outside [1, 65535]", B);
+  if (n_parts < 1 || n_parts > fp4kv::kMaxShardParts)
+    return fail(FP4KV_ERR_UNSUPPORTED, "n_parts=%d outside [1, %d]", n_parts, fp4kv::kMaxShardParts);
+  if (k_part < 1 || int64_t(n_parts) * k_part > 16384)
+    return fail(FP4KV_ERR_UNSUPPORTED, "n_parts * k_part = %lld outside [1, 16384]", (long long)n_parts * k_part);
+  if (top_k < 1 || top_k > 4096) return fail(FP4KV_ERR_UNSUPPORTED, "top_k=%d outside [1, 4096]", top_k);
+  for (int r = 0; r < n_parts; ++r)
+    if (part_base[r] < 0) return fail(FP4KV_ERR_INVALID_ARG, "part_base[%d] = %d < 0", r, part_base[r]);
+  if (!aligned(cand_score, 4) || !aligned(cand_idx, 4) || !aligned(out_idx, 4) || !aligned(out_local, 4) ||
+      !aligned(out_score, 4))
+    return fail(FP4KV_ERR_INVALID_ARG, "misaligned argument (4 B)");
+  cudaError_t e;
+  {
+    prof::Scope ps(2, static_cast<cudaStream_t>(stream));
+    e = fp4kv::launch_topk_merge(cand_score, cand_idx, n_parts, k_part, part_base, B, top_k, local_lo, local_hi,
+                                 out_idx, out_local, out_score, static_cast<cudaStream_t>(stream));
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "topk_merge");
+  return ok();
+}
+
+fp4kv_status fp4kv_lse_combine(const float* part_out, const float* part_lse, int32_t n_parts, int32_t B, int32_t H,
+                               int32_t d, float* out, float* lse, void* stream) {
+  if (!part_out || !part_lse || !out) return fail(FP4KV_ERR_INVALID_ARG, "null part_out, part_lse or out");
+  if (n_parts < 1 || n_parts > 1024) return fail(FP4KV_ERR_UNSUPPORTED, "n_parts=%d outside [1, 1024]", n_parts);
+  if (B < 1 || B > 65535 || H < 1 || H > 128 || d < 1 || d > 1024)
+    return fail(FP4KV_ERR_UNSUPPORTED, "B=%d, H=%d or d=%d outside the supported range", B, H, d);
+  if (!aligned(part_out, 4) || !aligned(part_lse, 4) || !aligned(out, 4) || !aligned(lse, 4))
+    return fail(FP4KV_ERR_INVALID_ARG, "misaligned argument (4 B)");
+  cudaError_t e;
+  {
+    prof::Scope ps(3, static_cast<cudaStream_t>(stream));
+    e = fp4kv::launch_lse_combine(part_out, part_lse, n_parts, int64_t(B) * H, d, out, lse,
+                                  static_cast<cudaStream_t>(stream));
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "lse_combine");
+  return ok();
+}
+
 fp4kv_status fp4kv_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int32_t d, int64_t x_row_stride,
                                  const int64_t* dst_row, uint8_t* out, int64_t cap_rows, void* stream) {
   if (n_rows < 0 || cap_rows < 0) return fail(FP4KV_ERR_INVALID_ARG, "negative n_rows or cap_rows");

@@ -98,6 +98,17 @@ struct AttnParams {
   uint32_t* status;
 };
 cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream);
+
+// ----------------------------------------------------------------------------------------
+// Context-sharded decode: exact merge of per-range top-K candidates, and the log-sum-exp
+// combine of per-range attention partials (csrc/shard.cu).
+// ----------------------------------------------------------------------------------------
+constexpr int kMaxShardParts = 64;
+cudaError_t launch_topk_merge(const float* cand_score, const int32_t* cand_idx, int n_parts, int k_part,
+                              const int32_t* part_base, int B, int top_k, int lo, int hi, int32_t* out_idx,
+                              int32_t* out_local, float* out_score, cudaStream_t stream);
+cudaError_t launch_lse_combine(const float* part_out, const float* part_lse, int n_parts, int64_t n_bh, int d,
+                               float* out, float* lse, cudaStream_t stream);
 int attn_chunks(int B, int H, int top_k, int num_sms);
 
 }  // namespace fp4kv

@@ -211,6 +211,34 @@ fp4kv_status fp4kv_sparse_swa_attn_decode(const uint16_t* q, int32_t B, int32_t 
                                           const uint8_t* swa, int32_t n_win, float sm_scale, float* out,
                                           float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* topk_merge -- context-sharded decode (no counterpart on the pages: several GPUs split every
+ * sequence's positions into contiguous ranges; part r holds positions [part_base[r], ...) and
+ * runs fp4kv_indexer_topk over its own range with out_score). This call merges the gathered
+ * per-part lists exactly: out_idx[b] = the top_k of the union of the candidates by score
+ * descending, then position ascending, as global positions in ascending order, padded with
+ * -1. The union contains the global top-K (a position among the best K of the whole context
+ * is among the best K of its range, ties being broken by position in both), so the result
+ * equals the indexer top-K of the whole context.
+ * cand_score fp32 / cand_idx int32 [n_parts][B][k_part]: each part's out_score / out_idx
+ *            (range-local positions, -1 absent), as an all-gather lays them out;
+ * part_base  HOST int32 [n_parts], >= 0;   1 <= n_parts <= 64, n_parts * k_part <= 16384;
+ * out_local  nullable int32 [B][top_k]: the selection as positions local to
+ *            [local_lo, local_hi), -1 elsewhere (what this part's attention needs);
+ * out_score  nullable fp32 [B][top_k] (-inf for pads). 1 <= top_k <= 4096. */
+fp4kv_status fp4kv_topk_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_parts, int32_t k_part,
+                              int32_t B, const int32_t* part_base, int32_t top_k, int32_t local_lo,
+                              int32_t local_hi, int32_t* out_idx, int32_t* out_local, float* out_score,
+                              void* stream);
+
+/* lse_combine -- context-sharded decode: joins attention partials computed over disjoint
+ * row sets (each range's fp4kv_sparse_attn_decode over the selected positions it holds).
+ * part_out fp32 [n_parts][B][H][d], part_lse fp32 [n_parts][B][H] (-inf: the part had no
+ * row). out[b][h] = sum_r w_r part_out[r][b][h] / sum_r w_r with w_r = e^(lse_r - max_r lse_r);
+ * lse (nullable) = max + ln(sum w_r), -inf (and out = 0) when every part is empty.
+ * 1 <= n_parts <= 1024, H <= 128, d <= 1024. */
+fp4kv_status fp4kv_lse_combine(const float* part_out, const float* part_lse, int32_t n_parts, int32_t B, int32_t H,
+                               int32_t d, float* out, float* lse, void* stream);
+
 /* swa_quant_fp8 -- the SWA KV's write: bf16 rows x [n_rows][d] (row stride x_row_stride
  * elements, a multiple of 8) to E4M3 codes, round to nearest even, saturating at +-448
  * ([PyTorchKR] FP4 KV section: the quantization-sensitive SWA KV stays FP8; a direct cast

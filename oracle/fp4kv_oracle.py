@@ -337,6 +337,22 @@ def sparse_swa_attn_decode_rows(q, v_sel, v_win, sm_scale: float):
     return sparse_attn_decode_rows(q, np.concatenate([v_sel, v_win], axis=0), sm_scale)
 
 
+def attn_lse_merge(outs, lses):
+    """Attention over the union of disjoint row sets from the attentions over each set:
+    outs [R, H, d], lses [R, H] (-inf for an empty set). out = sum_r e^(lse_r - M) out_r /
+    sum_r e^(lse_r - M), lse = M + ln(sum); (0, -inf) when every set is empty. (Follows from
+    writing each set's softmax numerator and denominator with its lse.)"""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    m = lses.max(axis=0)
+    with np.errstate(invalid="ignore"):
+        wts = np.where(np.isneginf(lses), 0.0, np.exp(lses - np.where(np.isneginf(m), 0.0, m)))
+    den = wts.sum(axis=0)
+    out = np.where(den[:, None] > 0, (wts[..., None] * outs).sum(axis=0) / np.where(den > 0, den, 1.0)[:, None], 0.0)
+    lse = np.where(den > 0, m + np.log(np.where(den > 0, den, 1.0)), -np.inf)
+    return out, lse
+
+
 def fp8_e4m3_to_f64(codes) -> np.ndarray:
     """FP8 E4M3 indexer keys / queries (uint8 codes) -> exact fp64 values."""
     return e4m3_decode(np.asarray(codes, dtype=np.uint8))

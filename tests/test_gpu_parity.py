@@ -591,3 +591,98 @@ def test_sparse_swa_attention_window_only_and_nothing(fk):
     _swa_case(fk, 35, B, cap, H, [1000, 77], idx, 128)
     out, lse = _swa_case(fk, 36, 1, cap, H, [0], np.full((1, 128), -1, dtype=np.int64), 128)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+# ----------------------------------------------------------------------------------------
+# Context-sharded decode: exact merge of per-range top-K lists, LSE combine of partials
+# ----------------------------------------------------------------------------------------
+
+def test_topk_merge_matches_oracle_with_ties_and_holes(fk):
+    rng = np.random.default_rng(51)
+    R, B, kp, K = 3, 4, 300, 256
+    bases = [0, 5000, 9000]
+    idx = np.full((R, B, kp), -1, dtype=np.int32)
+    sc = np.full((R, B, kp), -np.inf, dtype=np.float32)
+    for r in range(R):
+        for b in range(B):
+            m = [300, 120, 0, 37][b]
+            idx[r, b, :m] = rng.choice(4000, size=m, replace=False)
+            sc[r, b, :m] = rng.integers(0, 40, size=m).astype(np.float32) / 8  # many equal scores
+    lo, hi = 5000, 9000
+    out_score = torch.empty((B, K), dtype=torch.float32, device=DEV)
+    got, local = fk.topk_merge(torch.from_numpy(sc).to(DEV), torch.from_numpy(idx).to(DEV), bases, K,
+                               local_range=(lo, hi), out_score=out_score)
+    got, local, out_score = got.cpu().numpy(), local.cpu().numpy(), out_score.cpu().numpy()
+    for b in range(B):
+        s_all, p_all = [], []
+        for r in range(R):
+            ok = idx[r, b] >= 0
+            s_all.append(sc[r, b][ok])
+            p_all.append(idx[r, b][ok].astype(np.int64) + bases[r])
+        s_all, p_all = np.concatenate(s_all), np.concatenate(p_all)
+        want = O.topk_positions(s_all, p_all, K)
+        assert np.array_equal(got[b], want), b
+        assert np.array_equal(local[b], np.where((want >= lo) & (want < hi), want - lo, -1)), b
+        s_of = dict(zip(p_all.tolist(), s_all.tolist()))
+        m = int((want >= 0).sum())
+        assert np.array_equal(out_score[b, :m], np.array([s_of[p] for p in want[:m]], dtype=np.float32))
+        assert np.all(np.isneginf(out_score[b, m:]))
+
+
+def test_lse_combine_matches_oracle(fk):
+    rng = np.random.default_rng(52)
+    R, B, H, d = 4, 3, 64, 512
+    outs = rng.normal(0, 1, (R, B, H, d)).astype(np.float32)
+    lses = rng.normal(5, 3, (R, B, H)).astype(np.float32)
+    lses[1, 0] = -np.inf          # a part without rows
+    lses[:, 2, :5] = -np.inf      # heads with no row anywhere
+    outs[:, 2, :5] = 0
+    out, lse = fk.lse_combine(torch.from_numpy(outs).to(DEV), torch.from_numpy(lses).to(DEV))
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        ro, rl = O.attn_lse_merge(outs[:, b].astype(np.float64), lses[:, b].astype(np.float64))
+        fin = np.isfinite(rl)
+        assert np.allclose(out[b], ro, rtol=1e-5, atol=1e-6)
+        assert np.allclose(lse[b][fin], rl[fin], rtol=1e-6, atol=1e-5) and np.all(np.isneginf(lse[b][~fin]))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_sharded_step_emulated_on_one_gpu(fk, world):
+    """The sharded protocol with the library's kernels, its ranks run one after another on
+    one GPU (no rank waits on another: the exchanges are stacks of the ranks' outputs)."""
+    from fp4_sparse_attention_kv_b200 import shard
+    B, cap, H, K, d = 3, 20000, 64, 512, 512
+    lens = [20000, 13001, 3000]
+    q_idx, w, keys = _indexer_inputs(53, B, cap, 32, True)
+    x = P.kv_rows_dev(53, 0, B, cap, d, DEV)
+    packed = torch.empty((B, cap, d // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((B, cap, d // 16), dtype=torch.uint8, device=DEV)
+    fk.kv_quant_fp4(x.view(B * cap, d), packed.view(B * cap, d // 2), scales.view(B * cap, d // 16))
+    del x
+    q = synth.attn_query(53, 0, B, H, d, device=DEV)
+    ops = shard.LibraryOps(fk)
+    ranges = [shard.shard_range(cap, r, world) for r in range(world)]
+    p1 = [shard.local_topk_phase(ops, world, r, cap, lens, q_idx, w, keys[:, lo:hi].contiguous(), K)
+          for r, (lo, hi) in enumerate(ranges)]
+    all_idx = torch.stack([p[1] for p in p1])
+    all_score = torch.stack([p[2] for p in p1])
+    idxs, outs, lses = [], [], []
+    for r, (lo, hi) in enumerate(ranges):
+        i, o, l = shard.merge_attend_phase(ops, world, r, cap, all_score, all_idx, K, q,
+                                           packed[:, lo:hi].contiguous(), scales[:, lo:hi].contiguous(), p1[r][0], 1.0)
+        idxs.append(i.cpu().numpy())
+        outs.append(o)
+        lses.append(l)
+    out, lse = ops.combine(torch.stack(outs), torch.stack(lses))
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for r in range(1, world):
+        assert np.array_equal(idxs[r], idxs[0])
+    qh = P.to_f64(q.cpu())
+    for b in range(B):
+        L = lens[b]
+        sc = P.oracle_scores_seq(q_idx[b], w[b], keys[b], L)
+        P.check_topk(idxs[0][b], sc, np.arange(L), K, f"sharded top-K b={b}")
+        sel = idxs[0][b][idxs[0][b] >= 0]
+        pk, s8 = O.kv_quant_fp4(P.kv_rows_host(53, 0, b, sel, d))
+        ro, rl = O.sparse_attn_decode_rows(qh[b], O.kv_dequant_fp4(pk, s8), 1.0)
+        P.check_attn(out[b], lse[b], ro, rl, f"sharded attention b={b}")

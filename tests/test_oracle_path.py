@@ -281,3 +281,24 @@ def test_swa_one_softmax_equals_the_lse_merge_of_the_two_branches():
     assert np.allclose(ow, o2) and np.allclose(lw, l2)
     os_, ls = O.sparse_swa_attn_decode_rows(q, sel, np.zeros((0, 64)), 1.3)
     assert np.allclose(os_, o1) and np.allclose(ls, l1)
+
+
+def test_attn_lse_merge_equals_attention_over_the_union():
+    """Context sharding: attention over disjoint row sets merged by their lse equals the
+    attention over all rows (brute force), empty sets included."""
+    rng = np.random.default_rng(9)
+    q = rng.normal(0, 0.05, (5, 32))
+    sets = [rng.normal(0, 1, (7, 32)), np.zeros((0, 32)), rng.normal(0, 1, (12, 32)), rng.normal(0, 2, (1, 32))]
+    outs, lses = [], []
+    for rows in sets:
+        if rows.shape[0]:
+            o, l = O.sparse_attn_decode_rows(q, rows, 0.7)
+        else:
+            o, l = np.zeros((5, 32)), np.full(5, -np.inf)
+        outs.append(o)
+        lses.append(l)
+    om, lm = O.attn_lse_merge(np.stack(outs), np.stack(lses))
+    ow, lw = O.sparse_attn_decode_rows(q, np.concatenate(sets), 0.7)
+    assert np.allclose(om, ow, rtol=1e-12, atol=1e-12) and np.allclose(lm, lw, rtol=1e-12, atol=1e-12)
+    oe, le = O.attn_lse_merge(np.zeros((2, 5, 32)), np.full((2, 5), -np.inf))
+    assert np.all(oe == 0) and np.all(np.isneginf(le))
