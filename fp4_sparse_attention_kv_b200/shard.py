@@ -42,6 +42,9 @@ class LibraryOps:
 
     def local_topk(self, q, w, keys_local, lens_local, top_k):
         B = lens_local.shape[0]
+        if keys_local.shape[1] == 0:  # an empty range (a context shorter than the ranks' split)
+            return (torch.full((B, top_k), -1, dtype=torch.int32, device=lens_local.device),
+                    torch.full((B, top_k), float("-inf"), dtype=torch.float32, device=lens_local.device))
         score = torch.empty((B, top_k), dtype=torch.float32, device=lens_local.device)
         idx = self.fk.indexer_topk(q, w, keys_local, lens_local, top_k, out_score=score)
         return idx, score
@@ -50,6 +53,10 @@ class LibraryOps:
         return self.fk.topk_merge(all_score, all_idx, bases, top_k, local_range=(lo, hi))
 
     def local_attention(self, q, packed_local, scales_local, lens_local, sel_local, sm_scale):
+        if packed_local.shape[1] == 0:  # an empty range holds no row: weight 0 in the combine
+            B, H, d = q.shape
+            return (torch.zeros((B, H, d), dtype=torch.float32, device=q.device),
+                    torch.full((B, H), float("-inf"), dtype=torch.float32, device=q.device))
         return self.fk.sparse_attn_decode(q, packed_local, scales_local, lens_local, sel_local, sm_scale)
 
     def combine(self, all_out, all_lse):

@@ -93,3 +93,54 @@ def test_binding_raises_typed_errors():
     with pytest.raises(binding.Fp4kvError) as ei:
         binding._check(2)
     assert ei.value.status == 2
+
+
+def test_host_validation_of_the_window_shard_and_selftest_calls():
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    f1 = ctypes.c_float(1.0)
+    # sliding-window write: d must be a multiple of 16, pointers 16-byte aligned
+    st, msg = _call("fp4kv_swa_quant_fp8", fake, 4, 40, 40, None, fake, 4, None)
+    assert st == 2 and "d=40" in msg
+    st, msg = _call("fp4kv_swa_quant_fp8", fake, 4, 512, 512, None, P(0x10008), 4, None)
+    assert st == 1 and "aligned" in msg
+    # attention with a window: n_win in [1, 128], swa required
+    st, msg = _call("fp4kv_sparse_swa_attn_decode", fake, 1, 16, 512, fake, fake, 10, fake, fake, 4, fake, 129, f1,
+                    fake, None, fake, 1 << 20, None)
+    assert st == 2 and "n_win" in msg
+    st, msg = _call("fp4kv_sparse_swa_attn_decode", fake, 1, 16, 512, fake, fake, 10, fake, fake, 4, None, 64, f1,
+                    fake, None, fake, 1 << 20, None)
+    assert st == 1 and "swa" in msg
+    # exact merge of per-range lists: at most 64 parts and 16384 candidates, bases >= 0
+    bases = (ctypes.c_int32 * 65)(*([0] * 65))
+    st, msg = _call("fp4kv_topk_merge", fake, fake, 65, 8, 1, bases, 8, 0, 0, fake, None, None, None)
+    assert st == 2 and "n_parts" in msg
+    st, msg = _call("fp4kv_topk_merge", fake, fake, 8, 4096, 1, bases, 8, 0, 0, fake, None, None, None)
+    assert st == 2 and "k_part" in msg
+    neg = (ctypes.c_int32 * 2)(0, -5)
+    st, msg = _call("fp4kv_topk_merge", fake, fake, 2, 8, 1, neg, 8, 0, 0, fake, None, None, None)
+    assert st == 1 and "part_base" in msg
+    st, msg = _call("fp4kv_lse_combine", fake, fake, 0, 1, 16, 512, fake, None, None)
+    assert st == 2 and "n_parts" in msg
+    st, msg = _call("fp4kv_lse_combine", fake, fake, 2, 1, 129, 512, fake, None, None)
+    assert st == 2 and "H=129" in msg
+    # FP4 indexer operands need an even H_I and cap
+    st, msg = _call("fp4kv_indexer_topk", fake, fake, 31, fake, 2, None, 100, fake, 1, None, 0, 8, 16, fake, None,
+                    fake, 1 << 20, None)
+    assert st == 2 and "even" in msg
+    # the bounded-wait test hook checks its limit and workspace before launching anything
+    st, msg = _call("fp4kv_selftest_wait_timeout", 0, fake, 256, None)
+    assert st == 1 and "limit_us" in msg
+    st, msg = _call("fp4kv_selftest_wait_timeout", 1000, None, 256, None)
+    assert st == 1 and "workspace" in msg
+
+
+def test_shard_ranges_cover_the_context_once():
+    from fp4_sparse_attention_kv_b200 import shard
+    for cap in (1, 7, 8, 1000, 65536, 1 << 20):
+        for world in (1, 2, 3, 4, 8):
+            rs = [shard.shard_range(cap, r, world) for r in range(world)]
+            assert rs[0][0] == 0 and rs[-1][1] == cap
+            for (lo, hi), (lo2, _) in zip(rs, rs[1:]):
+                assert hi == lo2 and lo <= hi
+            assert all(lo % 8 == 0 or lo == cap for lo, _ in rs)
