@@ -121,7 +121,7 @@ def test_context_sharded_step_on_two_gloo_ranks_equals_the_whole_context():
     sys.path.insert(0, ROOT)
     from oracle import fp4kv_oracle as O
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         result = m.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), result), nprocs=world, join=True)
         result = dict(result)
