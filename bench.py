@@ -81,6 +81,22 @@ CONFIGS = {
 }
 
 
+# sizes a command line may override (the JSON line then lists them under config.overrides)
+OVERRIDES = (("B", int), ("cap", int), ("H", int), ("H_I", int), ("K", int), ("npb", int), ("seed", int))
+
+
+def apply_overrides(cfg: dict, args) -> dict:
+    cfg = dict(cfg)
+    over = {k: getattr(args, k) for k, _ in OVERRIDES if getattr(args, k, None) is not None}
+    for k, v in over.items():
+        if k not in cfg:
+            raise SystemExit(f"--{k.replace('_', '-')} does not apply to this configuration")
+        cfg[k] = v
+    if over:
+        cfg["overrides"] = over
+    return cfg
+
+
 # ----------------------------------------------------------------------------------------
 # distributed plumbing
 # ----------------------------------------------------------------------------------------
@@ -790,8 +806,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step eagerly instead of "
                     "replaying a captured CUDA graph")
+    for key, kind in OVERRIDES:
+        ap.add_argument("--" + key.replace("_", "-"), type=kind, default=None,
+                        help=f"override the configuration's {key}")
     args = ap.parse_args(argv)
-    cfg_name, cfg = args.config, CONFIGS[args.config]
+    cfg_name, cfg = args.config, apply_overrides(CONFIGS[args.config], args)
     if args.impl == "reference":
         return run_reference(args, cfg_name, cfg)
     if args.warmup < 3:
@@ -889,7 +908,8 @@ def main(argv=None):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp4-e2m1/e4m3 storage; fp16 MMA, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": cfg["workload"], "name": cfg_name,
+            "config": {"workload": cfg["workload"], "name": cfg_name, **({"overrides": cfg["overrides"]}
+                                                                          if "overrides" in cfg else {}),
                        "l2": l2_note,
                        "parallelism": f"dp{world} (independent sequences per GPU)",
                        "launch": ("one CUDA graph replay per step" if wl.graphs is not None

@@ -68,3 +68,15 @@ def test_reference_arm_prints_one_line_on_rank0_only():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["n_gpus"] == 2 and line["scaling"] == "weak"
+
+
+def test_size_overrides_apply_and_are_reported():
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    ns = argparse.Namespace(B=4, cap=None, H=None, H_I=None, K=512, npb=None, seed=None)
+    cfg = bench.apply_overrides(bench.CONFIGS["decode32"], ns)
+    assert (cfg["B"], cfg["K"], cfg["cap"]) == (4, 512, 65536) and cfg["overrides"] == {"B": 4, "K": 512}
+    assert "overrides" not in bench.CONFIGS["decode32"]  # the table itself is unchanged
+    with pytest.raises(SystemExit):
+        bench.apply_overrides(bench.CONFIGS["quant"], ns)  # the sweep has no batch or top-K
