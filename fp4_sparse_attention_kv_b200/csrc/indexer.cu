@@ -446,18 +446,26 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
     int cur_b = -1;
     uint32_t it = 0;
     TileIter ti;
+    // adds this CTA's histogram(s) of sequence b to the global ones and clears them: four
+    // bins per 16-byte access, atomics only for non-zero bins (the scores of a sequence
+    // fall into few bins)
+    auto flush_one = [&](uint32_t* sh, uint32_t* gh) {
+      for (int i4 = gtid; i4 < kHistBins / 4; i4 += kEpiThreads) {
+        uint4* q4 = reinterpret_cast<uint4*>(sh) + i4;
+        const uint4 c = *q4;
+        if ((c.x | c.y | c.z | c.w) == 0u) continue;
+        uint32_t* g = gh + 4 * i4;
+        if (c.x) atomicAdd(g, c.x);
+        if (c.y) atomicAdd(g + 1, c.y);
+        if (c.z) atomicAdd(g + 2, c.z);
+        if (c.w) atomicAdd(g + 3, c.w);
+        *q4 = make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
     auto flush = [&](int b) {
       epi_sync(group);
-      for (int i = gtid; i < kHistBins; i += kEpiThreads) {
-        const uint32_t c = s_hist[i];
-        if (c) atomicAdd(p.hist + int64_t(b) * kHistBins + i, c);
-        s_hist[i] = 0;
-        if (p.bmax != nullptr) {
-          const uint32_t c2 = s_bhist[i];
-          if (c2) atomicAdd(p.bmax_hist + int64_t(b) * kHistBins + i, c2);
-          s_bhist[i] = 0;
-        }
-      }
+      flush_one(s_hist, p.hist + int64_t(b) * kHistBins);
+      if (p.bmax != nullptr) flush_one(s_bhist, p.bmax_hist + int64_t(b) * kHistBins);
       epi_sync(group);
     };
     int len_b = -1;

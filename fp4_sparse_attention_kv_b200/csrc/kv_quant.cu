@@ -80,6 +80,9 @@ __global__ void __launch_bounds__(256) k_kv_quant_fp4(const uint16_t* __restrict
   // the indexer scan that follows on the stream may start its prologue now (it waits for
   // this grid before reading anything)
   griddep_launch_dependents();
+  // launched as a programmatic dependent: the kernel before it on the stream (the previous
+  // step's attention merge, whose attention may still read these rows) is complete past here
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -111,6 +114,7 @@ __global__ void __launch_bounds__(256) k_swa_quant_fp8(const uint16_t* __restric
                                                        const int64_t* __restrict__ dst_row,
                                                        uint8_t* __restrict__ out, int64_t cap_rows) {
   griddep_launch_dependents();
+  griddep_wait();  // (as in k_kv_quant_fp4)
   const int lane = threadIdx.x & 31;
   const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -141,6 +145,23 @@ __global__ void __launch_bounds__(256) k_swa_quant_fp8(const uint16_t* __restric
   }
 }
 
+// A launch that may begin while the kernel before it on the stream finishes (programmatic
+// dependent launch); the kernel orders itself with griddep_wait().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 }  // namespace
 
 cudaError_t launch_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int d, int64_t x_stride,
@@ -151,8 +172,9 @@ cudaError_t launch_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int d, int64
   int64_t blocks = (n_rows + 7) / 8;
   const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
   if (blocks > max_blocks) blocks = max_blocks;
-  k_swa_quant_fp8<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, n_rows, d, x_stride, dst_row, out,
-                                                                          cap_rows);
+  cudaError_t e = launch_pdl(k_swa_quant_fp8, dim3(static_cast<unsigned>(blocks)), dim3(threads), stream, x, n_rows,
+                             d, x_stride, dst_row, out, cap_rows);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -165,8 +187,9 @@ cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_
   int64_t blocks = (n_rows + rows_per_block - 1) / rows_per_block;
   const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
   if (blocks > max_blocks) blocks = max_blocks;
-  k_kv_quant_fp4<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-      x, n_rows, d, x_stride, dst_row, packed, scales, cap_rows);
+  cudaError_t e = launch_pdl(k_kv_quant_fp4, dim3(static_cast<unsigned>(blocks)), dim3(threads), stream, x, n_rows,
+                             d, x_stride, dst_row, packed, scales, cap_rows);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
