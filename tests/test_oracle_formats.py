@@ -171,3 +171,12 @@ def test_packed_row_size_and_890_bytes_per_token():
     # 2.5 cached entries per token, each a 288 B FP4 row plus a 68 B indexer key
     # (64 B of 4-bit codes for 128 dims and one 4 B scale).
     assert O.global_kv_bytes_per_token(2.5, 512, 68) == facts["global_kv_bytes_per_token"]["value"]
+
+
+def test_swa_fp8_golden_codes():
+    """Hand-derived E4M3 codes of the sliding-window KV's FP8 storage (tests/golden)."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "swa_fp8_example.json")))
+    for c in g["cases"]:
+        assert int(O.swa_quant_fp8(np.float64(c["x"]))) == c["code"], c["why"]
