@@ -297,21 +297,17 @@ def sparse_attn_decode(q, packed, scales, idx, seq_len: int, sm_scale: float):
     if sel.size == 0:
         return np.zeros((H, d)), np.full(H, -np.inf)
     v = kv_dequant_fp4(np.asarray(packed)[sel], np.asarray(scales)[sel])  # [J, d]
-    z = sm_scale * (q @ v.T)  # [H, J]
-    m = z.max(axis=1, keepdims=True)
-    e = np.exp(z - m)
-    den = e.sum(axis=1, keepdims=True)
-    out = (e @ v) / den
-    lse = m[:, 0] + np.log(den[:, 0])
-    return out, lse
+    return sparse_attn_decode_rows(q, v, sm_scale)
 
 
 def sparse_attn_decode_rows(q, v_hat, sm_scale: float):
-    """Same as ``sparse_attn_decode`` when the selected rows are already dequantized:
-    v_hat [J, d] fp64 (J >= 1)."""
+    """Softmax attention of every head of q [H, d] over already dequantized rows v_hat
+    [J, d] (J >= 1, fp64): z = sm_scale * q . v_hat_j, m = max_j z, o = sum e^(z-m) v_hat /
+    sum e^(z-m), lse = m + ln sum e^(z-m). ``sparse_attn_decode`` calls this after it has
+    gathered and dequantized the selected rows. Returns (out [H, d], lse [H])."""
     q = np.asarray(q, dtype=np.float64)
     v = np.asarray(v_hat, dtype=np.float64)
-    z = sm_scale * (q @ v.T)
+    z = sm_scale * (q @ v.T)  # [H, J]
     m = z.max(axis=1, keepdims=True)
     e = np.exp(z - m)
     den = e.sum(axis=1, keepdims=True)

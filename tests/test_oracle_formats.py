@@ -32,6 +32,20 @@ def test_e4m3_decode_matches_torch_all_codes():
     assert len(O.E4M3_POS_VALUES) == 127 and np.all(np.diff(O.E4M3_POS_VALUES) > 0)
 
 
+def test_bf16_bits_to_f64_matches_torch_all_patterns():
+    """Every one of the 65,536 bf16 bit patterns decodes to torch's own bfloat16 -> float64
+    value (NaN patterns to NaN), so a wrong shift or width fails here."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):  # the NaN patterns
+        ours = O.bf16_bits_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))  # -0 stays -0
+    assert nan.sum() == 2 * 127  # exponent all ones, mantissa non-zero, either sign
+
+
 def test_e2m1_values_from_bitfields():
     # E2M1: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit; exponent 0 is subnormal.
     vals = []

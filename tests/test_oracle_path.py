@@ -184,6 +184,27 @@ def test_attention_duplicates_count_and_invalid_entries_skip():
     assert np.allclose(out2, O.sparse_attn_decode(q, packed, scales, np.array([3]), 10, 1.0)[0])
 
 
+def test_attention_rows_helper_matches_brute_force_scaled_with_duplicates():
+    """The helper every GPU parity test compares against, pinned on its own: plain-loop
+    softmax attention at sm_scale != 1 over rows with duplicates and large logits (a
+    dropped sm_scale, a missing max shift or a wrong lse term fails here)."""
+    rng = np.random.default_rng(15)
+    packed, scales = _rows(rng, 9, 32)
+    vh = O.kv_dequant_fp4(packed, scales)
+    sel = vh[[4, 1, 4, 8, 0, 4]]
+    q = rng.standard_normal((3, 32)) * 4.0  # logits of tens: the max shift matters
+    for sm in (0.75, 1.0, 2.5):
+        out, lse = O.sparse_attn_decode_rows(q, sel, sm)
+        ref_out, ref_lse = _brute_attn(q, sel, sm)
+        assert np.allclose(out, ref_out, rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+    # and through the gathering entry point, which must agree with the helper exactly
+    out_g, lse_g = O.sparse_attn_decode(q, packed, scales, np.array([4, 1, 4, 8, 0, 4]), 9, 0.75)
+    ref_out, ref_lse = _brute_attn(q, sel, 0.75)
+    assert np.allclose(out_g, ref_out, rtol=1e-12, atol=1e-12)
+    assert np.allclose(lse_g, ref_lse, rtol=1e-12, atol=1e-12)
+
+
 def test_attention_with_no_valid_entry():
     rng = np.random.default_rng(14)
     packed, scales = _rows(rng, 4, 32)
