@@ -52,6 +52,8 @@ SIGNATURES = [
     ("fp4kv_topk_merge", ctypes.c_int, [_P, _P, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32, _I32, _I32, _P,
                                         _P, _P, _P]),
     ("fp4kv_lse_combine", ctypes.c_int, [_P, _P, _I32, _I32, _I32, _I32, _P, _P, _P]),
+    ("fp4kv_noalloc_status", ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _P]),
+    ("fp4kv_selftest_wait_timeout_noalloc", ctypes.c_int, [_I32, _P]),
 ]
 
 KERNEL_KINDS = ("kv_quant_fp4", "index_score", "topk_select", "sparse_attn")
@@ -377,6 +379,24 @@ def indexer_topk_noalloc(q, w, keys, seq_lens, top_k, pool=None, block_size=8, k
                                             top_k, _ptr(out_idx), _ptr(out_score),
                                             _stream(keys.device)))
     return out_idx
+
+
+def noalloc_status(device=None) -> int:
+    """Read and clear the status word of the allocation-free entry point's scratch on the
+    current device (synchronises the device's current stream)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = ctypes.c_uint32(0)
+    st = lib().fp4kv_noalloc_status(ctypes.byref(out), _stream(dev))
+    if st not in (0, 5):
+        _check(st)
+    return int(out.value)
+
+
+def selftest_wait_timeout_noalloc(limit_us: int, device=None):
+    """Test hook: selftest_wait_timeout on the allocation-free entry point's scratch (read
+    the result with noalloc_status)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check(lib().fp4kv_selftest_wait_timeout_noalloc(int(limit_us), _stream(dev)))
 
 
 def topk_merge(cand_score: torch.Tensor, cand_idx: torch.Tensor, part_base, top_k: int,

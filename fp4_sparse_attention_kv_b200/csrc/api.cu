@@ -325,6 +325,10 @@ fp4kv_status fp4kv_topk_merge(const float* cand_score, const int32_t* cand_idx, 
   if (k_part < 1 || int64_t(n_parts) * k_part > 16384)
     return fail(FP4KV_ERR_UNSUPPORTED, "n_parts * k_part = %lld outside [1, 16384]", (long long)n_parts * k_part);
   if (top_k < 1 || top_k > 4096) return fail(FP4KV_ERR_UNSUPPORTED, "top_k=%d outside [1, 4096]", top_k);
+  if (k_part < top_k)
+    return fail(FP4KV_ERR_UNSUPPORTED,
+                "k_part=%d < top_k=%d: each part must keep top_k candidates for the merge to be exact",
+                k_part, top_k);
   for (int r = 0; r < n_parts; ++r)
     if (part_base[r] < 0) return fail(FP4KV_ERR_INVALID_ARG, "part_base[%d] = %d < 0", r, part_base[r]);
   if (!aligned(cand_score, 4) || !aligned(cand_idx, 4) || !aligned(out_idx, 4) || !aligned(out_local, 4) ||
@@ -591,25 +595,54 @@ static __device__ __align__(256) uint8_t g_noalloc_ws[kNoAllocBytes];
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[256] = {};
+// per device ordinal: the context the address was looked up in, and the address
+struct NoallocSlot {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+NoallocSlot g_noalloc_slot[256];
 
-// Device address of g_noalloc_ws on the current device, looked up once per device (with
-// that device current). In host code the array's name is only a host-side stand-in.
+// The driver's cuCtxGetCurrent through the runtime's entry-point query (no link against
+// libcuda). The cached address of the scratch is only valid in the context it was looked
+// up in: after a device reset the primary context is a new one and the lookup is redone.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_noalloc_ws on the current device, looked up with that device current
+// on the first call in each context and cached. In host code the array's name is only a
+// host-side stand-in, never a device address.
 fp4kv_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= 256) return fail(FP4KV_ERR_UNSUPPORTED, "device ordinal %d", dev);
   std::lock_guard<std::mutex> g(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  void* ctx = current_context();
+  if (!slot.ptr || ctx == nullptr || ctx != slot.ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_ws);
     if (e != cudaSuccess || p == nullptr)
       return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
                        "indexer_topk_noalloc: cudaGetSymbolAddress");
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx = current_context();  // the lookup has made the device's context current
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return FP4KV_OK;
 }
 }  // namespace
@@ -640,13 +673,30 @@ fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H
   st = noalloc_scratch(&ws);
   if (st != FP4KV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the status word and the histogram + counters must start at zero
-  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.cnt - L.hist, s);
+  // the histograms and counters must start at zero. The status word at the head is left
+  // as it is: a bounded wait that gave up in an earlier call stays visible until
+  // fp4kv_noalloc_status reads (and clears) it.
+  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.cnt - L.hist, s);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: clearing scratch");
   return run_indexer(kind, q, w, H_I, keys, key_dtype, key_scale, cap, seq_lens, B, pool,
                      pool ? n_pool_blocks : 0, top_k, out_idx, nullptr, out_score, ws, L.total, s);
+}
+
+fp4kv_status fp4kv_noalloc_status(uint32_t* host_status, void* stream) {
+  if (!host_status) return fail(FP4KV_ERR_INVALID_ARG, "null host_status");
+  void* ws = nullptr;
+  fp4kv_status st = noalloc_scratch(&ws);
+  if (st != FP4KV_OK) return st;
+  return fp4kv_workspace_status(ws, host_status, stream);
+}
+
+fp4kv_status fp4kv_selftest_wait_timeout_noalloc(int32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(FP4KV_ERR_INVALID_ARG, "limit_us=%d outside [1, 1000000]", limit_us);
+  void* ws = nullptr;
+  fp4kv_status st = noalloc_scratch(&ws);
+  if (st != FP4KV_OK) return st;
+  return fp4kv_selftest_wait_timeout(limit_us, ws, kNoAllocBytes, stream);
 }
 
 fp4kv_status fp4kv_profile_enable(int32_t on) {

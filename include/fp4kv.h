@@ -222,6 +222,9 @@ fp4kv_status fp4kv_sparse_swa_attn_decode(const uint16_t* q, int32_t B, int32_t 
  * cand_score fp32 / cand_idx int32 [n_parts][B][k_part]: each part's out_score / out_idx
  *            (range-local positions, -1 absent), as an all-gather lays them out;
  * part_base  HOST int32 [n_parts], >= 0;   1 <= n_parts <= 64, n_parts * k_part <= 16384;
+ *            k_part >= top_k (each part keeps top_k candidates, padded with -1 when its
+ *            range is shorter; fewer could drop a global winner, so k_part < top_k is
+ *            rejected with FP4KV_ERR_UNSUPPORTED);
  * out_local  nullable int32 [B][top_k]: the selection as positions local to
  *            [local_lo, local_hi), -1 elsewhere (what this part's attention needs);
  * out_score  nullable fp32 [B][top_k] (-inf for pads). 1 <= top_k <= 4096. */
@@ -259,16 +262,32 @@ fp4kv_status fp4kv_swa_quant_fp8(const uint16_t* x, int64_t n_rows, int32_t d, i
  * return FP4KV_ERR_UNSUPPORTED with an explanatory message. The call allocates nothing: it
  * clears the scratch's counters with cudaMemsetAsync on `stream` and launches the same
  * kernels as fp4kv_indexer_topk. The first call on each device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current) and caches it; make that first
- * call before any stream capture. All calls on a device share the one array, so calls whose
- * kernels overlap on the GPU (different streams, or different host threads) race and give
- * wrong results: serialise them. */
+ * address (cudaGetSymbolAddress, with that device current) and caches it for the device's
+ * current context (a device reset makes a new context, and the next call looks it up again);
+ * make that first call before any stream capture. All calls on a device share the one
+ * array, so calls whose kernels overlap on the GPU (different streams, or different host
+ * threads) race and give wrong results: serialise them. A kernel whose bounded wait gave up
+ * sets bit 0 of the scratch's status word; the word keeps it across later calls until
+ * fp4kv_noalloc_status reads it. */
 fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H_I,
                                         const void* keys, int32_t key_dtype,
                                         const float* key_scale, int64_t cap,
                                         const int32_t* seq_lens, int32_t B, const int32_t* pool,
                                         int32_t n_pool_blocks, int32_t block_size, int32_t top_k,
                                         int32_t* out_idx, float* out_score, void* stream);
+
+/* noalloc_status -- the status word of the scratch that fp4kv_indexer_topk_noalloc uses on
+ * the current device (no counterpart on the pages; the allocation-free counterpart of
+ * fp4kv_workspace_status): copies it into *host_status, waits for `stream`, then clears it.
+ * Returns FP4KV_ERR_DEVICE_FLAG if it was non-zero (bit 0: a kernel's bounded wait gave up,
+ * so the results of the calls since the last read are not to be trusted). Synchronising
+ * diagnostic; allocates nothing. */
+fp4kv_status fp4kv_noalloc_status(uint32_t* host_status, void* stream);
+
+/* selftest_wait_timeout_noalloc -- fp4kv_selftest_wait_timeout on the scratch of
+ * fp4kv_indexer_topk_noalloc (a test hook, no counterpart on the pages): the status bit
+ * lands in the word that fp4kv_noalloc_status reads. */
+fp4kv_status fp4kv_selftest_wait_timeout_noalloc(int32_t limit_us, void* stream);
 
 /* Benchmark support (no counterpart on the pages). While enabled, every kernel the library
  * launches is bracketed by two CUDA events recorded on the launch stream (do not enable

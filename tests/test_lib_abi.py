@@ -117,6 +117,9 @@ def test_host_validation_of_the_window_shard_and_selftest_calls():
     assert st == 2 and "n_parts" in msg
     st, msg = _call("fp4kv_topk_merge", fake, fake, 8, 4096, 1, bases, 8, 0, 0, fake, None, None, None)
     assert st == 2 and "k_part" in msg
+    # each part must keep top_k candidates, or the merge could miss a global winner
+    st, msg = _call("fp4kv_topk_merge", fake, fake, 2, 8, 1, bases, 16, 0, 0, fake, None, None, None)
+    assert st == 2 and "k_part=8 < top_k=16" in msg
     neg = (ctypes.c_int32 * 2)(0, -5)
     st, msg = _call("fp4kv_topk_merge", fake, fake, 2, 8, 1, neg, 8, 0, 0, fake, None, None, None)
     assert st == 1 and "part_base" in msg
@@ -133,6 +136,10 @@ def test_host_validation_of_the_window_shard_and_selftest_calls():
     assert st == 1 and "limit_us" in msg
     st, msg = _call("fp4kv_selftest_wait_timeout", 1000, None, 256, None)
     assert st == 1 and "workspace" in msg
+    st, msg = _call("fp4kv_selftest_wait_timeout_noalloc", 0, None)
+    assert st == 1 and "limit_us" in msg
+    st, msg = _call("fp4kv_noalloc_status", None, None)
+    assert st == 1 and "host_status" in msg
 
 
 def test_shard_ranges_cover_the_context_once():

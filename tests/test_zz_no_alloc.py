@@ -68,3 +68,21 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(fk):
     with pytest.raises(fk.Fp4kvError) as ei:
         fk.indexer_topk_noalloc(q, w, big_keys, lens_t, 64)
     assert ei.value.status == 2 and "maximum" in str(ei.value)
+
+
+def test_noalloc_status_reports_a_bounded_wait_that_gave_up(fk):
+    """A bounded wait that gives up in a kernel running on the allocation-free scratch sets
+    the scratch's status bit; an indexer call afterwards keeps it (it clears only the
+    histograms and counters), fp4kv_noalloc_status reports it once and clears it, and the
+    next call's results are again exact."""
+    torch.cuda.synchronize()
+    assert fk.noalloc_status() == 0
+    fk.selftest_wait_timeout_noalloc(20000)  # 20 ms, then the bit is set
+    q, w, keys, lens_t = _inputs(55, 2, 6000, [6000, 5000])
+    ref = fk.indexer_topk(q, w, keys, lens_t, 128)
+    got = fk.indexer_topk_noalloc(q, w, keys, lens_t, 128)
+    assert fk.noalloc_status() == 1
+    assert fk.noalloc_status() == 0  # reading clears the word
+    assert torch.equal(got, ref)
+    got2 = fk.indexer_topk_noalloc(q, w, keys, lens_t, 128)
+    assert torch.equal(got2, ref) and fk.noalloc_status() == 0
