@@ -10,7 +10,9 @@ pages' own 20-layer schedule (groups of 4 over one shared KV, top-K 512, pool of
 blocks). Prints ONE JSON line (rank 0).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--config decode32|decode32_fp4idx|decode32_swa|long|hier|csa2_decoder|tiny|quant]
+       [--config long|hier|csa2_decoder|csa2_encoder|decode32|decode32_fp4idx|decode32_swa|tiny|quant]
+The default is `long` (batch 4 x 1,048,576 entries): the largest single-GPU decode step and
+one of the two 1M-entry workloads on which the HBM target is stated.
 Under torchrun (N > 1) each rank runs the same per-GPU workload on its own GPU (weak
 scaling; the path has no exchange step, so there is no collective in the data path); the
 step time is the max over ranks.
@@ -45,7 +47,6 @@ SWA_LAYER = 700  # generator stream of the sliding-window rows
 L2_BYTES = 126 * 2 ** 20
 
 CONFIGS = {
-    # the configuration the metric is quoted on (one GPU)
     "decode32": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=True, seed=1,
                      workload="decode batch 32 x 65,536 FP4 entries, 64 heads, FP8 indexer "
                               "keys, top-K 2048"),
@@ -59,6 +60,8 @@ CONFIGS = {
     "decode32_swa": dict(B=32, cap=65536, H=64, H_I=32, K=2048, fp8=True, swa=128, seed=1,
                          workload="decode batch 32 x 65,536 FP4 entries + a 128-token FP8 sliding "
                                   "window, 64 heads, FP8 indexer keys, top-K 2048"),
+    # the default: the largest single-GPU decode step, one of the 1M-entry configurations
+    # the HBM target (indexer top-K + sparse attention at >= 70 % of HBM) is stated on
     "long": dict(B=4, cap=1 << 20, H=64, H_I=32, K=2048, fp8=True, seed=2,
                  workload="long context batch 4 x 1,048,576 FP4 entries, 64 heads, FP8 "
                           "indexer keys, top-K 2048"),
@@ -74,6 +77,16 @@ CONFIGS = {
                          workload="CSA2 decoder schedule batch 8 x 1,048,576 entries, 20 layers "
                                   "in groups of 4 (Full or Reindex, then 3 Reuse) over one shared "
                                   "FP4 KV and indexer key set, pool of 2048 blocks x 8, top-K 512"),
+    # the encoder schedule of the same section: layers 1-2 attend over their sliding window
+    # only; the other 18 run CSA2 at compression m = 2 in 3 groups of 6 (one Full layer that
+    # owns the group's KV and indexer keys, then 5 Reuse layers); a 1M-token context is
+    # 524,288 compressed entries
+    "csa2_encoder": dict(B=8, cap=1 << 19, H=64, H_I=32, K=512, fp8=True, seed=6, swa=128,
+                         swa_layers=2, groups=3, group=6,
+                         workload="CSA2 encoder schedule batch 8 x 524,288 entries (1M tokens at "
+                                  "m = 2), 2 sliding-window-only layers (128-token FP8 window) "
+                                  "then 3 groups of 6 (Full + 5 Reuse), own FP4 KV and FP8 "
+                                  "indexer keys per group, top-K 512"),
     "tiny": dict(B=1, cap=4096, H=16, H_I=32, K=256, fp8=False, seed=0,
                  workload="tiny batch 1 x 4096 entries, 16 heads, bf16 indexer keys, top-K 256"),
     "quant": dict(tokens=131072, layers=20, seed=4,
@@ -386,9 +399,9 @@ class DecodeWorkload(TwoSets):
             self.inputs.append(self.x_swa_new)
             self.in_attrs = self.in_attrs + ("x_swa_new",)
         self.outputs = [self.out, self.lse]
-        # quantize, scan, select (filter + finish), attention (+ the chunk merge when split)
-        # (+ the query's FP4 quantize with an FP4 indexer, + the window row's FP8 write)
-        self.launches_per_step = (5 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
+        # quantize, scan, select, attention (+ the chunk merge when split) (+ the query's FP4
+        # quantize with an FP4 indexer, + the window row's FP8 write)
+        self.launches_per_step = (4 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
                                   + (1 if self.n_win else 0))
         self.attn_rows_per_step = B * (K + self.n_win)
         self.tokens_per_step = B
@@ -417,7 +430,11 @@ class HierWorkload(TwoSets):
     """Hierarchical: 20 layers per step. Layer 1 (Full): hier_pool_select over all entries
     -> top-K + pool; layers 2, 4, .., 20 (Reindex): own indexer query scored inside the pool
     over layer 1's keys; layers 3, 5, .., 19 (Reuse): the previous layer's indices. Every
-    layer writes its new row into its own FP4 KV and attends over it."""
+    layer has its own FP4 KV and attends over it. The new rows of all 20 layers are written
+    by one quantize call at the start of the step: in the pages' causal encoder-decoder every
+    decoder layer's global KV is a projection of the encoder's last hidden state, so all of
+    them exist before the first decoder layer runs (the queries do not: each layer computes
+    its own from its own hidden state, so the layers' scans and attentions stay in order)."""
 
     def __init__(self, cfg, fk, device, rank=0):
         self.cfg, self.fk, self.dev = cfg, fk, device
@@ -425,8 +442,12 @@ class HierWorkload(TwoSets):
                                       cfg["layers"], cfg["npb"])
         seed = cfg["seed"] + 1000 * rank
         self.B, self.cap, self.H, self.H_I, self.K, self.L, self.npb = B, cap, H, H_I, K, L, npb
-        self.packed = [torch.empty((B, cap, D // 2), dtype=torch.uint8, device=device) for _ in range(L)]
-        self.scales = [torch.empty((B, cap, D // 16), dtype=torch.uint8, device=device) for _ in range(L)]
+        # the 20 layers' caches in one allocation (layer-major), so one call writes every
+        # layer's new row
+        self.packed_all = torch.empty((L, B, cap, D // 2), dtype=torch.uint8, device=device)
+        self.scales_all = torch.empty((L, B, cap, D // 16), dtype=torch.uint8, device=device)
+        self.packed = [self.packed_all[l] for l in range(L)]
+        self.scales = [self.scales_all[l] for l in range(L)]
         self.keys = torch.empty((B, cap, DK), dtype=torch.uint8, device=device)
         chunk = 1 << 18
         for b in range(B):
@@ -441,9 +462,10 @@ class HierWorkload(TwoSets):
         qw = [synth.indexer_query(seed, l, B, H_I, fp8=True, device=device) for l in range(L)]
         self.qi = [a for a, _ in qw]
         self.w = [b_ for _, b_ in qw]
-        self.x_new = [synth.kv_rows(seed, l, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
-                      for l in range(L)]
-        self.dst = torch.arange(B, dtype=torch.int64, device=device) * cap + (cap - 1)
+        # new rows [L * B, d] (layer-major) and their rows in the layer-major caches
+        self.x_new = torch.cat([synth.kv_rows(seed, l, 10 ** 6, torch.arange(B, dtype=torch.int64, device=device), D)
+                                for l in range(L)])
+        self.dst = torch.arange(L * B, dtype=torch.int64, device=device) * cap + (cap - 1)
         self.lens = torch.full((B,), cap, dtype=torch.int32, device=device)
         self.idx = [torch.empty((B, K), dtype=torch.int32, device=device) for _ in range(L)]
         self.pool = torch.empty((B, npb), dtype=torch.int32, device=device)
@@ -452,19 +474,19 @@ class HierWorkload(TwoSets):
         self.ws_h = fk.alloc_workspace(fk.workspace_bytes(fk.OP_HIER_POOL_SELECT, B, cap, H_I, K, npb), device)
         self.ws_r = fk.alloc_workspace(fk.workspace_bytes(fk.OP_REINDEX_TOPK, B, cap, H_I, K, npb), device)
         self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
-        self.inputs = self.q + self.qi + self.w + self.x_new
+        self.inputs = self.q + self.qi + self.w + [self.x_new]
         self.outputs = self.out + self.lse
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
-        # per layer a quantize and an attention (+ merge); the Full layer and each Reindex layer
-        # add a scan and the two select kernels
-        self.launches_per_step = L + 3 + (L // 2) * 3 + L * (1 + attn_split(fk, B, cap, H, K))
+        # one quantize; the Full layer and each Reindex layer a scan and a select; per layer an
+        # attention (+ merge)
+        self.launches_per_step = 1 + 2 + (L // 2) * 2 + L * (1 + attn_split(fk, B, cap, H, K))
         self.tokens_per_step = B
 
     def step(self):
         fk, L = self.fk, self.L
+        fk.kv_quant_fp4(self.x_new, self.packed_all.view(-1, D // 2), self.scales_all.view(-1, D // 16),
+                        dst_row=self.dst)
         for l in range(L):
-            fk.kv_quant_fp4(self.x_new[l], self.packed[l].view(-1, D // 2),
-                            self.scales[l].view(-1, D // 16), dst_row=self.dst)
             if l == 0:
                 fk.hier_pool_select(self.qi[0], self.w[0], self.keys, self.lens, self.K, self.npb,
                                     ws=self.ws_h, out_idx=self.idx[0], out_pool=self.pool)
@@ -528,9 +550,8 @@ class Csa2DecoderWorkload(TwoSets):
         self.inputs = self.q + self.qi + self.w + [self.x_new]
         self.outputs = self.out + self.lse
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
-        # one quantize; a scan and the two select kernels per group; an attention (+ merge)
-        # per layer
-        self.launches_per_step = 1 + 3 * n_src + L * (1 + attn_split(fk, B, cap, H, K))
+        # one quantize; a scan and a select per group; an attention (+ merge) per layer
+        self.launches_per_step = 1 + 2 * n_src + L * (1 + attn_split(fk, B, cap, H, K))
         self.tokens_per_step = B
 
     def step(self):
@@ -554,6 +575,88 @@ class Csa2DecoderWorkload(TwoSets):
         return {"index_score": B * self.cap * DK + n_reindex * B * self.npb * 8 * DK,
                 "sparse_attn": L * B * self.K * ROW_BYTES,
                 "kv_quant_fp4": B * (2 * D + ROW_BYTES)}
+
+
+class Csa2EncoderWorkload(TwoSets):
+    """The encoder schedule of the pages' CSA2 section: layers 1-2 attend over their own
+    sliding window only (its KV kept in FP8); the other 18 layers run CSA2 at compression
+    m = 2 in 3 groups of 6. The first layer of a group (Full) writes the group's new KV row,
+    scores every entry with its indexer query over the group's own keys and keeps the top-K;
+    the 5 Reuse layers attend with their own queries over the same KV and indices. Encoder
+    layers run in order: each group's KV and query come from its own layer's hidden state."""
+
+    def __init__(self, cfg, fk, device, rank=0):
+        self.cfg, self.fk, self.dev = cfg, fk, device
+        B, cap, H, H_I, K = cfg["B"], cfg["cap"], cfg["H"], cfg["H_I"], cfg["K"]
+        G, NG, NS, nw = cfg["group"], cfg["groups"], cfg["swa_layers"], cfg["swa"]
+        seed = cfg["seed"] + 1000 * rank
+        self.B, self.cap, self.H, self.H_I, self.K, self.G, self.NG, self.NS, self.n_win = B, cap, H, H_I, K, G, NG, NS, nw
+        self.L = NS + NG * G
+        self.src = [NS + g * G for g in range(NG)]  # the groups' Full (KV source) layers
+        self.packed = [torch.empty((B, cap, D // 2), dtype=torch.uint8, device=device) for _ in range(NG)]
+        self.scales = [torch.empty((B, cap, D // 16), dtype=torch.uint8, device=device) for _ in range(NG)]
+        self.keys = [torch.empty((B, cap, DK), dtype=torch.uint8, device=device) for _ in range(NG)]
+        chunk = 1 << 18
+        for g in range(NG):
+            for b in range(B):
+                for r0 in range(0, cap, chunk):
+                    rows = torch.arange(r0, min(cap, r0 + chunk), dtype=torch.int64, device=device)
+                    fk.kv_quant_fp4(synth.kv_rows(seed, self.src[g], b, rows, D),
+                                    self.packed[g][b, r0:r0 + rows.numel()], self.scales[g][b, r0:r0 + rows.numel()])
+                    self.keys[g][b, r0:r0 + rows.numel()] = synth.indexer_keys(seed, b, rows, DK, True,
+                                                                               source=self.src[g])
+        # the sliding-window-only layers: a ring of the last nw positions' rows (E4M3)
+        pos = torch.arange(cap - nw, cap, dtype=torch.int64, device=device)
+        self.swa = [torch.empty((B, nw, D), dtype=torch.uint8, device=device) for _ in range(NS)]
+        for l in range(NS):
+            for b in range(B):
+                fk.swa_quant_fp8(synth.kv_rows(seed, SWA_LAYER + l, b, pos, D), self.swa[l][b], dst_row=pos % nw)
+        ar = torch.arange(B, dtype=torch.int64, device=device)
+        self.x_swa_new = [synth.kv_rows(seed, SWA_LAYER + l, 10 ** 6, ar, D) for l in range(NS)]
+        self.swa_dst = ar * nw + (cap - 1) % nw
+        self.x_new = [synth.kv_rows(seed, self.src[g], 10 ** 6, ar, D) for g in range(NG)]
+        self.dst = ar * cap + (cap - 1)
+        self.q = [synth.attn_query(seed, l, B, H, D, device=device) for l in range(self.L)]
+        qw = [synth.indexer_query(seed, self.src[g], B, H_I, fp8=True, device=device) for g in range(NG)]
+        self.qi = [a for a, _ in qw]
+        self.w = [b_ for _, b_ in qw]
+        self.lens = torch.full((B,), cap, dtype=torch.int32, device=device)
+        self.idx = [torch.empty((B, K), dtype=torch.int32, device=device) for _ in range(NG)]
+        self.no_idx = torch.full((B, 1), -1, dtype=torch.int32, device=device)  # window-only layers
+        self.out = [torch.empty((B, H, D), dtype=torch.float32, device=device) for _ in range(self.L)]
+        self.lse = [torch.empty((B, H), dtype=torch.float32, device=device) for _ in range(self.L)]
+        self.ws_i = fk.alloc_workspace(fk.workspace_bytes(fk.OP_INDEXER_TOPK, B, cap, H_I, K), device)
+        self.ws_a = fk.alloc_workspace(fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K), device)
+        self.inputs = self.q + self.qi + self.w + self.x_new + self.x_swa_new
+        self.outputs = self.out + self.lse
+        self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new", "x_swa_new"), ("out", "lse")
+        # per window-only layer a window write and an attention; per group a quantize, a
+        # scan, the two select kernels and G attentions
+        self.launches_per_step = 2 * NS + NG * (4 + G)
+        self.attn_rows_per_step = NG * G * B * K + NS * B * nw
+        self.tokens_per_step = B
+
+    def step(self):
+        fk = self.fk
+        for l in range(self.NS):
+            fk.swa_quant_fp8(self.x_swa_new[l], self.swa[l].view(-1, D), dst_row=self.swa_dst)
+            fk.sparse_attn_decode(self.q[l], self.packed[0], self.scales[0], self.lens, self.no_idx, 1.0,
+                                  ws=self.ws_a, out=self.out[l], lse=self.lse[l], swa=self.swa[l])
+        for g in range(self.NG):
+            fk.kv_quant_fp4(self.x_new[g], self.packed[g].view(-1, D // 2), self.scales[g].view(-1, D // 16),
+                            dst_row=self.dst)
+            fk.indexer_topk(self.qi[g], self.w[g], self.keys[g], self.lens, self.K, ws=self.ws_i,
+                            out_idx=self.idx[g])
+            for j in range(self.G):
+                l = self.src[g] + j
+                fk.sparse_attn_decode(self.q[l], self.packed[g], self.scales[g], self.lens, self.idx[g], 1.0,
+                                      ws=self.ws_a, out=self.out[l], lse=self.lse[l])
+
+    def algorithmic_bytes(self):
+        B, NG, G, NS = self.B, self.NG, self.G, self.NS
+        return {"index_score": NG * B * self.cap * DK,
+                "sparse_attn": NG * G * B * self.K * ROW_BYTES + NS * B * self.n_win * D,
+                "kv_quant_fp4": NG * B * (2 * D + ROW_BYTES) + NS * B * (2 * D + D)}
 
 
 class QuantWorkload(TwoSets):
@@ -684,40 +787,146 @@ def e2e_steps(wl, steps, warmup):
 # CPU oracle baseline (the oracle as it stands, on a bounded sample)
 # ----------------------------------------------------------------------------------------
 
-def oracle_sample_decode(cfg, seq: int, layer_seed=None):
-    """The whole decode step for ONE sequence with the oracle (host inputs from synth)."""
+def _bits(x):
+    """bf16 tensor -> its uint16 bit patterns (numpy), the oracle's input form."""
+    return x.view(torch.int16).numpy().astype(np.uint16)
+
+
+def oracle_prepare_decode(cfg, seq: int):
+    """Inputs of the whole decode step for ONE sequence, drawn from synth as the GPU workload
+    draws them (untimed), and the oracle's run over them (timed)."""
     from oracle import fp4kv_oracle as O
     seed = cfg["seed"]
     cap, H, H_I, K, fp8 = cfg["cap"], cfg["H"], cfg["H_I"], cfg["K"], cfg["fp8"]
     rows = torch.arange(cap, dtype=torch.int64)
     keys = synth.indexer_keys(seed, seq, rows, DK, fp8)
     qi, w = synth.indexer_query(seed, 0, seq + 1, H_I, fp8=fp8)
-    kf = O.fp8_e4m3_to_f64(keys.numpy()) if fp8 else O.bf16_bits_to_f64(keys.view(torch.int16).numpy().astype(np.uint16))
-    qf = O.fp8_e4m3_to_f64(qi[seq].numpy()) if fp8 else O.bf16_bits_to_f64(qi[seq].view(torch.int16).numpy().astype(np.uint16))
-    if cfg.get("idx") == "fp4":
-        kf, qf = O.indexer_fp4_values(kf), O.indexer_fp4_values(qf)
-    x_new = synth.kv_rows(seed, 0, 10 ** 6, torch.tensor([seq]), D)
-    O.kv_quant_fp4(O.bf16_bits_to_f64(x_new.view(torch.int16).numpy().astype(np.uint16)))
-    idx, _ = O.indexer_topk(qf, w[seq].double().numpy(), kf, cap, K)
-    sel = idx[idx >= 0]
-    xr = synth.kv_rows(seed, 0, seq, torch.as_tensor(sel), D)
-    pk, sc = O.kv_quant_fp4(O.bf16_bits_to_f64(xr.view(torch.int16).numpy().astype(np.uint16)))
-    q = synth.attn_query(seed, 0, seq + 1, H, D)[seq]
-    qf64 = O.bf16_bits_to_f64(q.view(torch.int16).numpy().astype(np.uint16))
+    keys_in = keys.numpy() if fp8 else _bits(keys)
+    qi_in = qi[seq].numpy() if fp8 else _bits(qi[seq])
+    w_in = w[seq].double().numpy()
+    x_new = _bits(synth.kv_rows(seed, 0, 10 ** 6, torch.tensor([seq]), D))
+    q = _bits(synth.attn_query(seed, 0, seq + 1, H, D)[seq])
     nw = cfg.get("swa", 0)
-    if nw:
-        xw = synth.kv_rows(seed, SWA_LAYER, seq, torch.arange(cap - nw, cap, dtype=torch.int64), D)
-        vw = O.e4m3_decode(O.swa_quant_fp8(O.bf16_bits_to_f64(xw.view(torch.int16).numpy().astype(np.uint16))))
-        O.sparse_swa_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), vw, 1.0)
-    else:
-        O.sparse_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), 1.0)
+    xw = _bits(synth.kv_rows(seed, SWA_LAYER, seq, torch.arange(cap - nw, cap, dtype=torch.int64), D)) if nw else None
+
+    def rows_of(sel):  # the selected rows' bf16 values (the cache content), drawn on demand
+        return _bits(synth.kv_rows(seed, 0, seq, torch.as_tensor(sel), D))
+
+    def run():
+        dec = O.fp8_e4m3_to_f64 if fp8 else O.bf16_bits_to_f64
+        kf, qf = dec(keys_in), dec(qi_in)
+        if cfg.get("idx") == "fp4":
+            kf, qf = O.indexer_fp4_values(kf), O.indexer_fp4_values(qf)
+        O.kv_quant_fp4(O.bf16_bits_to_f64(x_new))
+        idx, _ = O.indexer_topk(qf, w_in, kf, cap, K)
+        pk, sc = O.kv_quant_fp4(O.bf16_bits_to_f64(rows_of(idx[idx >= 0])))
+        qf64 = O.bf16_bits_to_f64(q)
+        if nw:
+            vw = O.e4m3_decode(O.swa_quant_fp8(O.bf16_bits_to_f64(xw)))
+            O.sparse_swa_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), vw, 1.0)
+        else:
+            O.sparse_attn_decode_rows(qf64, O.kv_dequant_fp4(pk, sc), 1.0)
+    return run
 
 
-def oracle_sample_quant(cfg, rows=2048):
+def oracle_prepare_layers(cfg, seq: int):
+    """The whole 20-layer step (hier or csa2_decoder) for ONE sequence: inputs drawn from
+    synth (untimed) and the oracle's run (timed): the Full layer's scan with top-K and
+    pool, the Reindex layers inside the pool, every layer's new-row write and attention."""
     from oracle import fp4kv_oracle as O
-    x = synth.kv_rows(cfg["seed"], 0, 0, torch.arange(rows, dtype=torch.int64), D, heavy_frac=0.001)
-    O.kv_quant_fp4(O.bf16_bits_to_f64(x.view(torch.int16).numpy().astype(np.uint16)))
-    return rows
+    seed, cap, H, H_I, K, L, npb = (cfg["seed"], cfg["cap"], cfg["H"], cfg["H_I"], cfg["K"],
+                                     cfg["layers"], cfg["npb"])
+    G = cfg.get("group")  # csa2_decoder: groups of G over one shared KV
+    keys = synth.indexer_keys(seed, seq, torch.arange(cap, dtype=torch.int64), DK, True).numpy()
+    writes = [l for l in range(L) if G is None or l == 0]  # csa2: only the Full layer writes
+    x_new = {l: _bits(synth.kv_rows(seed, l, 10 ** 6, torch.tensor([seq]), D)) for l in writes}
+    scans = [l for l in range(L) if l == 0 or (G is None and l % 2 == 1) or (G is not None and l % G == 0)]
+    qw = {}
+    for l in scans:
+        src = l if G is None else (l // G) * G
+        qi, w = synth.indexer_query(seed, src, seq + 1, H_I, fp8=True)
+        qw[l] = (qi[seq].numpy(), w[seq].double().numpy())
+    q = {l: _bits(synth.attn_query(seed, l, seq + 1, H, D)[seq]) for l in range(L)}
+
+    def rows_of(l, sel):
+        return _bits(synth.kv_rows(seed, l if G is None else 0, seq, torch.as_tensor(sel), D))
+
+    def run():
+        kf = O.fp8_e4m3_to_f64(keys)
+        idx_of, pool = {}, None
+        for l in range(L):
+            if l in x_new:
+                O.kv_quant_fp4(O.bf16_bits_to_f64(x_new[l]))
+            if l in qw:
+                qf = O.fp8_e4m3_to_f64(qw[l][0])
+                if l == 0:
+                    idx_of[l], pool, _ = O.hier_pool_select(qf, qw[l][1], kf, cap, K, 8, npb)
+                else:
+                    idx_of[l], _, _ = O.reindex_topk(qf, qw[l][1], kf, cap, pool, 8, K)
+            else:
+                idx_of[l] = idx_of[l - 1]
+            pk, sc = O.kv_quant_fp4(O.bf16_bits_to_f64(rows_of(l, idx_of[l][idx_of[l] >= 0])))
+            O.sparse_attn_decode_rows(O.bf16_bits_to_f64(q[l]), O.kv_dequant_fp4(pk, sc), 1.0)
+    return run
+
+
+def oracle_prepare_encoder(cfg, seq: int):
+    """The whole csa2_encoder step for ONE sequence: inputs drawn from synth (untimed) and
+    the oracle's run (timed): the window-only layers' writes and attentions, then per group
+    the new row, the scan with top-K over the group's keys and the group's attentions."""
+    from oracle import fp4kv_oracle as O
+    seed, cap, H, H_I, K = cfg["seed"], cfg["cap"], cfg["H"], cfg["H_I"], cfg["K"]
+    G, NG, NS, nw = cfg["group"], cfg["groups"], cfg["swa_layers"], cfg["swa"]
+    src = [NS + g * G for g in range(NG)]
+    rows = torch.arange(cap, dtype=torch.int64)
+    keys = [synth.indexer_keys(seed, seq, rows, DK, True, source=src[g]).numpy() for g in range(NG)]
+    qw = []
+    for g in range(NG):
+        qi, w = synth.indexer_query(seed, src[g], seq + 1, H_I, fp8=True)
+        qw.append((qi[seq].numpy(), w[seq].double().numpy()))
+    q = [_bits(synth.attn_query(seed, l, seq + 1, H, D)[seq]) for l in range(NS + NG * G)]
+    x_new = [_bits(synth.kv_rows(seed, src[g], 10 ** 6, torch.tensor([seq]), D)) for g in range(NG)]
+    win = []
+    for l in range(NS):
+        wr = _bits(synth.kv_rows(seed, SWA_LAYER + l, seq, torch.arange(cap - nw, cap, dtype=torch.int64), D))
+        wr[-1] = _bits(synth.kv_rows(seed, SWA_LAYER + l, 10 ** 6, torch.tensor([seq]), D))[0]  # this step's row
+        win.append(wr)
+
+    def run():
+        for l in range(NS):
+            vw = O.e4m3_decode(O.swa_quant_fp8(O.bf16_bits_to_f64(win[l])))
+            O.sparse_attn_decode_rows(O.bf16_bits_to_f64(q[l]), vw, 1.0)
+        for g in range(NG):
+            O.kv_quant_fp4(O.bf16_bits_to_f64(x_new[g]))
+            kf = O.fp8_e4m3_to_f64(keys[g])
+            idx, _ = O.indexer_topk(O.fp8_e4m3_to_f64(qw[g][0]), qw[g][1], kf, cap, K)
+            sel = idx[idx >= 0]
+            xr = _bits(synth.kv_rows(seed, src[g], seq, torch.as_tensor(sel), D))
+            xr[sel == cap - 1] = x_new[g][0]
+            vh = O.kv_dequant_fp4(*O.kv_quant_fp4(O.bf16_bits_to_f64(xr)))
+            for j in range(G):
+                O.sparse_attn_decode_rows(O.bf16_bits_to_f64(q[src[g] + j]), vh, 1.0)
+    return run
+
+
+def oracle_prepare_quant(cfg, rows=2048):
+    from oracle import fp4kv_oracle as O
+    x = _bits(synth.kv_rows(cfg["seed"], 0, 0, torch.arange(rows, dtype=torch.int64), D, heavy_frac=0.001))
+    return lambda: O.kv_quant_fp4(O.bf16_bits_to_f64(x))
+
+
+def oracle_sample(cfg_name, cfg, i: int):
+    """One bounded sample of the workload for the oracle: (run, work). Building the inputs
+    happens here, outside any timing; run() is the oracle's work on them. work is in the
+    metric's unit: GB read + written for the quant sweep, else tokens (one sequence's whole
+    step)."""
+    if cfg_name == "quant":
+        return oracle_prepare_quant(cfg), 2048 * (2 * D + ROW_BYTES) / 1e9
+    if cfg_name == "csa2_encoder":
+        return oracle_prepare_encoder(cfg, i % cfg["B"]), 1.0
+    if "layers" in cfg:
+        return oracle_prepare_layers(cfg, i % cfg["B"]), 1.0
+    return oracle_prepare_decode(cfg, i % cfg["B"]), 1.0
 
 
 def oracle_threads():
@@ -729,29 +938,44 @@ def oracle_threads():
         return 1
 
 
-def cpu_baseline(cfg_name, cfg, budget_s=12.0):
-    """Oracle throughput on a bounded sample of the workload, in the metric's unit."""
-    t0 = time.perf_counter()
-    if cfg_name == "quant":
-        rows = 0
-        while time.perf_counter() - t0 < budget_s:
-            rows += oracle_sample_quant(cfg)
-        el = time.perf_counter() - t0
-        gbs = rows * (2 * D + ROW_BYTES) / el / 1e9
-        return {"value": gbs, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
-                "sample": f"{rows} rows of the quant sweep in {el:.1f} s"}
-    # layered configurations: one sequence's Full layer (scan + top-K + attention) stands for
-    # the step's dominant work; the 19 pool-bounded layers are not sampled
-    seqs = 0
-    while time.perf_counter() - t0 < budget_s or seqs == 0:
-        oracle_sample_decode(cfg, seqs % cfg["B"])
-        seqs += 1
-    el = time.perf_counter() - t0
-    layers = cfg.get("layers", 1)
-    return {"value": seqs / el / layers, "unit": "tokens/s",
-            "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{seqs} of {cfg['B']} sequences (whole decode step per sequence"
-                      f"{f', layer 1 only, scaled by 1/{layers}' if layers > 1 else ''}) in {el:.1f} s"}
+def _oracle_rate(cfg_name, cfg, budget_s, threads=None):
+    """(work per second, samples, seconds, threads used) of the oracle on whole samples,
+    taken until budget_s seconds of oracle time have passed (at least one sample); only
+    run() is timed, the inputs are built outside."""
+    from contextlib import nullcontext
+    try:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=threads, user_api="blas") if threads else nullcontext()
+    except Exception:
+        ctx = nullcontext()
+    with ctx:
+        used = oracle_threads()
+        el, work, n = 0.0, 0.0, 0
+        while n == 0 or el < budget_s:
+            run, w = oracle_sample(cfg_name, cfg, n)
+            t0 = time.perf_counter()
+            run()
+            el += time.perf_counter() - t0
+            work += w
+            n += 1
+    return work / el, n, el, used
+
+
+def cpu_baseline(cfg_name, cfg, budget_s=10.0):
+    """Oracle throughput on a bounded sample of the workload, in the metric's unit: once
+    single-threaded and once with the BLAS pool at its default size (the oracle's only
+    parallelism is numpy's BLAS), with the host's core count."""
+    unit = "GB/s" if cfg_name == "quant" else "tokens/s"
+    what = ("rows of the quant sweep, 2048 per sample" if cfg_name == "quant" else
+            "sequences, the whole step of one sequence per sample" +
+            (f" ({cfg['layers']} layers)" if "layers" in cfg else "") +
+            (" (20 layers)" if cfg_name == "csa2_encoder" else ""))
+    v1, n1, el1, _ = _oracle_rate(cfg_name, cfg, budget_s, threads=1)
+    vt, nt, elt, used = _oracle_rate(cfg_name, cfg, budget_s)
+    return {"value": vt, "unit": unit, "cores": used, "nproc": os.cpu_count(), "kind": "oracle",
+            "sample": f"{nt} {what} in {elt:.1f} s, BLAS on {used} threads",
+            "single_thread": {"value": v1, "unit": unit, "cores": 1,
+                              "sample": f"{n1} {what} in {el1:.1f} s"}}
 
 
 # ----------------------------------------------------------------------------------------
@@ -761,31 +985,30 @@ def run_reference(args, cfg_name, cfg):
     if rank != 0:
         return 0
     unit = "GB/s" if cfg_name == "quant" else "tokens/s"
-    per = []
-    for _ in range(args.warmup):
-        (oracle_sample_quant(cfg) if cfg_name == "quant" else oracle_sample_decode(cfg, 0))
-    t0 = time.perf_counter()
-    work = 0
+    # the oracle is plain CPU code: one untimed sample stands in for the warm-up steps
+    oracle_sample(cfg_name, cfg, 0)[0]()
+    el, work = 0.0, 0.0
     for i in range(args.steps):
-        if cfg_name == "quant":
-            work += oracle_sample_quant(cfg) * (2 * D + ROW_BYTES) / 1e9
-        else:
-            oracle_sample_decode(cfg, i % cfg["B"])
-            work += 1
-    el = time.perf_counter() - t0
+        run, w = oracle_sample(cfg_name, cfg, i)  # inputs built outside the timing
+        t0 = time.perf_counter()
+        run()
+        el += time.perf_counter() - t0
+        work += w
     value = work / el
-    if "layers" in cfg:
-        value /= cfg["layers"]
     cores = oracle_threads()
-    sample = ("2048 rows per step" if cfg_name == "quant" else
-              "one sequence of the batch per step (whole decode step for that sequence)")
+    sample = ("2048 rows of the sweep per step" if cfg_name == "quant" else
+              "one sequence of the batch per step (its whole step" +
+              (f", all {cfg['layers']} layers" if "layers" in cfg else "") + ")")
     line = {"metric": METRIC, "impl": "reference", "value": value, "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg["workload"], "sample": sample},
-            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "config": {"workload": cfg["workload"], "name": cfg_name, "sample": sample,
+                       "timing": "oracle compute only, summed over the steps; inputs drawn "
+                                 "from the generator outside the timing; one untimed warm-up "
+                                 "sample"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "nproc": os.cpu_count(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -801,7 +1024,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="decode32", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="long", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each step eagerly instead of "
@@ -834,6 +1057,8 @@ def main(argv=None):
         wl = HierWorkload(cfg, fk, device, rank)
     elif cfg_name == "csa2_decoder":
         wl = Csa2DecoderWorkload(cfg, fk, device, rank)
+    elif cfg_name == "csa2_encoder":
+        wl = Csa2EncoderWorkload(cfg, fk, device, rank)
     else:
         wl = DecodeWorkload(cfg, fk, device, rank)
     streamed = sum(wl.algorithmic_bytes().values())
@@ -896,6 +1121,17 @@ def main(argv=None):
     roof.update({"traffic": traffic_record(dom, cfg_name),
                  "algorithmic_bytes_per_launch": bytes_per_launch, "ms_per_launch": per_launch_ms})
     step_bytes = sum(v for k, v in alg.items())
+    # the HBM target's own quantity: the algorithmic bytes of indexer_topk + sparse_attn_decode
+    # (indexer keys, FP4 rows and scales) per step over the device time of the whole step
+    # (quantize-on-write included: the chained kernels are timed together)
+    target = None
+    if cfg_name != "quant":
+        tb = alg["index_score"] + alg["sparse_attn"]
+        tg = tb * world / (step_ms * 1e-3) / 1e9
+        target = {"kernels": "indexer_topk + sparse_attn_decode", "bound": "hbm",
+                  "algorithmic_bytes_per_step": tb, "ms_per_step": step_ms, "achieved": tg,
+                  "peak": peak, "unit": "GB/s", "frac": tg / peak, "peak_kind": peak_kind,
+                  "time": "device time of the whole step (CUDA events, max over ranks)"}
     kernels = {k: {"launches_per_step": n / args.steps, "ms_per_step": t / args.steps,
                    "algorithmic_bytes_per_step": alg.get(k), "gbs": (alg[k] / (t / args.steps * 1e-3) / 1e9) if k in alg and t > 0 else None}
                for k, (n, t) in prof.items() if n}
@@ -917,6 +1153,7 @@ def main(argv=None):
                        "tokens_per_step": tokens},
             "hbm_gbs_step": step_bytes * world / (step_ms * 1e-3) / 1e9,
             "roofline": roof,
+            "hbm_target": target,
             "kernels": kernels,
             "gpu_launches": wl.launches_per_step * args.steps,
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,

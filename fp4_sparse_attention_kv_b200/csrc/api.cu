@@ -101,7 +101,7 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Workspace layouts
 // ---------------------------------------------------------------------------------------
 struct IndexerLayout {
-  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist2 = 0, counters = 0, cnt = 0, list = 0;
+  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist2 = 0, counters = 0, zero_end = 0, cnt = 0, list = 0;
   size_t total = 0;
   int64_t score_stride = 0, bmax_stride = 0;
   int n_probs = 0;
@@ -133,15 +133,17 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
     L.k[1] = npb;
     L.vstride[1] = L.bmax_stride;
   }
-  // hist, hist2 and counters are contiguous: the region that must start at zero
+  // hist, hist2 and counters are contiguous: the region that must start at zero (the select
+  // leaves it so)
   L.hist = off;
   off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
   L.hist2 = off;
   off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
   L.counters = off;
   off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kSelCounters);
+  L.zero_end = off;
   L.cnt = off;
-  off += up(sizeof(uint32_t) * L.n_probs * 2 * B * fp4kv::kMaxSlices);
+  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kMaxSlices * fp4kv::kSelRegions);
   L.list = off;
   for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(uint64_t) * B * L.vstride[i]);
   L.total = off;
@@ -149,22 +151,16 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
 }
 
 struct AttnLayout {
-  size_t part_ml = 0, part_o = 0, total = 0;
-  int n_chunks = 1, n_hg = 1;
+  size_t total = 0;
+  int n_chunks = 1;
 };
 
+// The attention's workspace is the status word only: its chunk CTAs combine their partials
+// in distributed shared memory.
 AttnLayout attn_layout(int64_t B, int64_t H, int64_t top_k, int sms) {
   AttnLayout L;
-  L.n_hg = static_cast<int>((H + 63) / 64);
   L.n_chunks = fp4kv::attn_chunks(static_cast<int>(B), static_cast<int>(H), static_cast<int>(top_k), sms);
-  size_t off = kAlign;
-  if (L.n_chunks > 1) {
-    L.part_ml = off;
-    off += up(sizeof(float) * B * L.n_hg * L.n_chunks * 64 * 2);
-    L.part_o = off;
-    off += up(sizeof(float) * B * L.n_hg * L.n_chunks * 64 * 512);
-  }
-  L.total = off;
+  L.total = kAlign;
   return L;
 }
 
@@ -454,8 +450,7 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
     P.hist = p.hist + int64_t(i) * B * fp4kv::kHistBins;
     P.hist2 = reinterpret_cast<uint32_t*>(base + L.hist2) + int64_t(i) * B * fp4kv::kHistBins;
     P.counters = reinterpret_cast<uint32_t*>(base + L.counters) + int64_t(i) * B * fp4kv::kSelCounters;
-    P.cnt1 = reinterpret_cast<uint32_t*>(base + L.cnt) + int64_t(2 * i) * B * fp4kv::kMaxSlices;
-    P.cnt2 = P.cnt1 + int64_t(B) * fp4kv::kMaxSlices;
+    P.cnt = reinterpret_cast<uint32_t*>(base + L.cnt) + int64_t(i) * B * fp4kv::kMaxSlices * fp4kv::kSelRegions;
     P.list = reinterpret_cast<uint64_t*>(base + list_off);
     list_off += up(sizeof(uint64_t) * B * L.vstride[i]);
     P.out_idx = (i == 0) ? out_idx : out_pool;
@@ -546,8 +541,6 @@ static fp4kv_status run_attn(const uint16_t* q, int32_t B, int32_t H, int32_t d,
   p.out = out;
   p.lse = lse;
   p.n_chunks = L.n_chunks;
-  p.part_ml = L.n_chunks > 1 ? reinterpret_cast<float*>(base + L.part_ml) : nullptr;
-  p.part_o = L.n_chunks > 1 ? reinterpret_cast<float*>(base + L.part_o) : nullptr;
   p.status = reinterpret_cast<uint32_t*>(base);
   cudaError_t e;
   {
@@ -676,7 +669,7 @@ fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H
   // the histograms and counters must start at zero. The status word at the head is left
   // as it is: a bounded wait that gave up in an earlier call stays visible until
   // fp4kv_noalloc_status reads (and clears) it.
-  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.cnt - L.hist, s);
+  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.zero_end - L.hist, s);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: clearing scratch");
   return run_indexer(kind, q, w, H_I, keys, key_dtype, key_scale, cap, seq_lens, B, pool,
                      pool ? n_pool_blocks : 0, top_k, out_idx, nullptr, out_score, ws, L.total, s);

@@ -35,7 +35,12 @@
 //    (MN-major B operand). Cross-lane reductions happen only when a reference moves and
 //    once at the end, when O^T is staged in shared memory and leaves in one bulk store.
 //  Per-chunk barriers let the next tile's dequantization overlap the current tile's P.V.
-//  Chunks of the index list go to different CTAs; k_attn_combine merges their partials.
+//  * Chunks of the index list go to different CTAs, and the chunk CTAs of one (sequence,
+//    head group) form one thread-block cluster. At the end they exchange their per-head
+//    reference m and row sum l through distributed shared memory, each stages its O scaled
+//    by its log-sum-exp weight 2^(m_c - M) / L, and CTA r sums its share of the output
+//    dims over the cluster and writes them: no partials pass through global memory and no
+//    second kernel runs.
 //  * With a sliding window (the pages' SWA branch, its KV kept in FP8), the last chunk's CTA
 //    runs one more tile: the window's E4M3 rows (exact in fp16), in the same softmax as the
 //    selected rows, so the window and the sparse selection share one normalisation.
@@ -66,6 +71,7 @@ constexpr int kMmaWarp = kSoftWarps + kGatherWarps;
 constexpr int kAttnThreads = 32 * (kMmaWarp + 1);  // 416
 constexpr int kSoftThreads = 32 * kSoftWarps;
 constexpr uint32_t kFlagMisaligned = 2u;
+constexpr int kMaxCluster = 16;   // chunk CTAs of one (sequence, head group)
 
 constexpr uint32_t kQChunkBytes = kHeadsPerCta * 128;  // 64 heads x 64 dims x 2 B
 constexpr uint32_t kVChunkBytes = kTile * 128;         // 128 entries x 64 dims x 2 B
@@ -324,10 +330,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   float* sL = reinterpret_cast<float*>(smem + kOffL);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
   volatile uint32_t* s_abort = s_tmem + 1;
+  volatile uint32_t* s_fail = s_tmem + 2;  // a softmax wait gave up: this CTA's partial is void
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int n_hg = gridDim.y, n_chunks = gridDim.x;
+  const int n_chunks = gridDim.x;
   const int hbase = hg * kHeadsPerCta;
   const int nh = min(kHeadsPerCta, p.H - hbase);
   int64_t len = p.seq_lens[b];
@@ -436,6 +443,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         }
         tc_fence_after();
         const uint32_t ds = tmem + kColS + 64u * u;
+        // (loops kept rolled: their first pass runs from a cold instruction cache)
+#pragma unroll 1
         for (int jc = 0; jc < kChunks && ok; ++jc) {
           if (!mbar_wait_timed(&bars[B_VREADY + jc], t & 1)) {
             ok = false;
@@ -460,10 +469,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         }
         tc_fence_after();
         const bool acc0 = t > 0;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           const uint32_t d = tmem + 64u * c;
-#pragma unroll
+#pragma unroll 2
           for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
             const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
             const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
@@ -676,13 +685,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
                                                    : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1));
       }
     }
-    // ---- output: wait for the last P.V, reduce the row sums, stage O, one bulk store ----
+    // ---- wait for the last P.V and reduce the row sums over the CTA ----
     if (!fail && n_tiles > 0) {
       const bool f = !softmax_wait(&bars[B_PFREE], (n_tiles - 1) & 1);
       fail = softmax_any(f);
     }
     if (fail) {
       if (tid == 0) fail_wait(p, s_abort);
+      if (q4 == 0) sL[h0 + lane] = 0.0f;  // this CTA's partial is dropped
     } else {
       tc_fence_after();
       const float lw = butterfly32<false>(lsum);  // lane l: head h0 + l over this warp's rows
@@ -692,58 +702,96 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         const int h = h0 + lane;
         sL[h] = sRed[h] + sRed[64 + h] + sRed[128 + h] + sRed[192 + h];
       }
-      softmax_sync();
-      const bool split = n_chunks > 1;
-      if (q4 == 0) {  // per-head factor: 1 for a partial, 1 / (2^6 L) for a final row, 0 if empty
-        const int h = h0 + lane;
-        const float L = sL[h];
-        sA[h] = L > 0.0f ? (split ? 1.0f : 1.0f / (kPScale * L)) : 0.0f;
+    }
+    if (tid == 0) *s_fail = fail ? 1u : 0u;
+  }
+
+  // ---- combine the chunk CTAs of this (sequence, head group): one cluster ----
+  // Every thread of every CTA of the cluster passes the cluster barriers below.
+  __syncthreads();
+  cluster_sync_all();  // (A) every CTA's per-head reference m and row sum l are visible
+  const uint32_t C = cluster_nctas(), rank = cluster_ctarank();
+  if (tid < kHeadsPerCta) {
+    // per head: M = max_c m_c over the CTAs with rows, Lt = sum_c 2^(m_c - M) l_c; this CTA's
+    // weight 2^(m_r - M) / (2^6 Lt) (O holds p * 2^6); lse = M ln 2 + ln Lt
+    const int h = tid;
+    float lc[kMaxCluster], mc[kMaxCluster];
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {  // (all remote loads first, then their use)
+      lc[c] = 0.0f;
+      mc[c] = -INFINITY;
+      if (c < static_cast<int>(C)) {
+        lc[c] = dsmem_ld_f32(dsmem_map(&sL[h], static_cast<uint32_t>(c)));
+        mc[c] = dsmem_ld_f32(dsmem_map(&sM[h], static_cast<uint32_t>(c)));
       }
-      softmax_sync();
-      // O^T -> staging [64 heads][512 dims] fp32 in the V_hat region: one 32-column TMEM load
-      // (this thread's heads) per dim tile
-      float* stage = reinterpret_cast<float*>(smem + kOffV);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c)
+      if (lc[c] > 0.0f) M = fmaxf(M, mc[c]);
+    float Lt = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c)
+      if (lc[c] > 0.0f) Lt += exp2f(mc[c] - M) * lc[c];
+    const float lo = sL[h];
+    sA[h] = (lo > 0.0f && Lt > 0.0f) ? exp2f(sM[h] - M) / (kPScale * Lt) : 0.0f;
+    if (rank == 0 && p.lse != nullptr && h < nh)
+      p.lse[int64_t(b) * p.H + hbase + h] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
+  }
+  __syncthreads();
+  // this CTA's O^T, scaled by its weight, as [64 heads][512 dims] fp32 in the V_hat region
+  // (free: the last P.V has completed): one 32-column TMEM load per dim tile
+  float* stage = reinterpret_cast<float*>(smem + kOffV);
+  if (warp < kSoftWarps) {
+    const int q4 = warp & 3, h0 = 32 * (warp >> 2), e = 32 * q4 + lane;
+    const uint32_t lane_addr = uint32_t(32 * q4) << 16;
+    const bool have = n_tiles > 0 && *s_fail == 0u;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        if (n_tiles > 0) {
-          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
-          tmem_ld_wait();
-        } else {
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      if (have) {
+        tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = 0u;
-        }
+        for (int k = 0; k < 32; ++k) r[k] = 0u;
+      }
 #pragma unroll
-        for (int k = 0; k < 32; ++k) stage[(h0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[h0 + k];
-      }
-      fence_proxy_async_smem();
-      softmax_sync();
-      const int64_t part = (int64_t(b) * n_hg + hg) * n_chunks + chunk;
-      float* dst = split ? p.part_o + part * kHeadsPerCta * kD : p.out + (int64_t(b) * p.H + hbase) * kD;
-      const uint32_t bytes = uint32_t(split ? kHeadsPerCta : nh) * kD * 4u;
-      if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
-        if (tid == 0) {
-          bulk_s2g(dst, stage, bytes);
-          bulk_commit();
-        }
-      } else {  // the output is only 8-byte aligned: copy with the softmax threads
-        const float2* s2 = reinterpret_cast<const float2*>(stage);
-        float2* d2 = reinterpret_cast<float2*>(dst);
-        for (uint32_t i = tid; i < bytes / 8; i += kSoftThreads) d2[i] = s2[i];
-      }
-      if (q4 == 0) {
-        const int h = h0 + lane;
-        const float L = sL[h];
-        if (split) {
-          p.part_ml[(part * kHeadsPerCta + h) * 2] = sM[h];
-          p.part_ml[(part * kHeadsPerCta + h) * 2 + 1] = L;
-        } else if (p.lse != nullptr && h < nh) {
-          p.lse[int64_t(b) * p.H + hbase + h] = L > 0.0f ? sM[h] * kLn2 + logf(L) : -INFINITY;
-        }
-      }
-      if (tid == 0) bulk_wait_read_all();  // the staging buffer stays valid until read
+      for (int k = 0; k < 32; ++k) stage[(h0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[h0 + k];
     }
   }
+  __syncthreads();
+  cluster_sync_all();  // (B) every CTA's scaled O is staged
+  {
+    // CTA `rank` sums dims [rank * 512 / C, +512 / C) of all 64 heads over the cluster's CTAs
+    // and writes them: 16-byte units, consecutive threads on consecutive dims of a head
+    const int slice4 = kD / 4 / static_cast<int>(C);  // float4 units per head in the slice
+    const int d0 = static_cast<int>(rank) * slice4 * 4;
+    const bool al16 = (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
+    for (int u = tid; u < nh * slice4; u += kAttnThreads) {
+      const int h = u / slice4, d = d0 + 4 * (u % slice4);
+      // all the CTAs' values are loaded before they are added (independent remote loads)
+      float4 v[kMaxCluster];
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c)
+        if (c < static_cast<int>(C)) v[c] = dsmem_ld_f32x4(dsmem_map(stage + h * kD + d, static_cast<uint32_t>(c)));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kMaxCluster; ++c) {
+        if (c < static_cast<int>(C)) {
+          acc.x += v[c].x; acc.y += v[c].y; acc.z += v[c].z; acc.w += v[c].w;
+        }
+      }
+      float* dst = p.out + (int64_t(b) * p.H + hbase + h) * kD + d;
+      if (al16) {
+        *reinterpret_cast<float4*>(dst) = acc;
+      } else {  // the output is only 8-byte aligned
+        reinterpret_cast<float2*>(dst)[0] = make_float2(acc.x, acc.y);
+        reinterpret_cast<float2*>(dst)[1] = make_float2(acc.z, acc.w);
+      }
+    }
+  }
+  cluster_sync_all();  // (C) no CTA leaves while another still reads its shared memory
 
   tc_fence_before();
   __syncthreads();
@@ -753,81 +801,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   }
 }
 
-// Merge of the chunk partials (log-sum-exp combine). Grid (64 heads, head groups, B), 128
-// threads: every thread accumulates 4 of the 512 dims over the chunks; the first chunks'
-// rows are loaded while the weights 2^(m_c - M) are computed into shared memory.
-constexpr int kMaxChunks = 256;
-__global__ void __launch_bounds__(128) k_attn_combine(const AttnParams p, int n_hg) {
-  __shared__ float s_w[kMaxChunks];
-  __shared__ float s_red[2][4];
-  griddep_wait();  // the attention grid's partials are complete and visible
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int hh = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int nh = min(kHeadsPerCta, p.H - hg * kHeadsPerCta);
-  if (hh >= nh) return;
-  const int n_chunks = p.n_chunks;
-  const int64_t base = (int64_t(b) * n_hg + hg) * n_chunks;
-  const float4* src = reinterpret_cast<const float4*>(p.part_o + (base * kHeadsPerCta + hh) * kD) + tid;
-  const int64_t cstride = int64_t(kHeadsPerCta) * kD / 4;  // float4s between chunks
-  // the first chunks' partial rows are loaded before the weights are known (independent)
-  constexpr int kPre = 8;
-  float4 v[kPre];
-#pragma unroll
-  for (int u = 0; u < kPre; ++u) v[u] = u < n_chunks ? __ldcg(src + u * cstride) : make_float4(0.f, 0.f, 0.f, 0.f);
-  float mloc = -INFINITY;
-  for (int c = tid; c < n_chunks; c += 128) {
-    const float mc = __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2]);
-    const float lc = __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1]);
-    s_w[c] = lc > 0.0f ? mc : -INFINITY;
-    if (lc > 0.0f) mloc = fmaxf(mloc, mc);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-  if (lane == 0) s_red[0][warp] = mloc;
-  __syncthreads();
-  const float M = fmaxf(fmaxf(s_red[0][0], s_red[0][1]), fmaxf(s_red[0][2], s_red[0][3]));
-  float lsum = 0.0f;
-  for (int c = tid; c < n_chunks; c += 128) {
-    const float mc = s_w[c];
-    const float w = mc == -INFINITY ? 0.0f : exp2f(mc - M);
-    s_w[c] = w;
-    lsum += w * __ldcg(&p.part_ml[((base + c) * kHeadsPerCta + hh) * 2 + 1]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if (lane == 0) s_red[1][warp] = lsum;
-  __syncthreads();
-  const float Lt = s_red[1][0] + s_red[1][1] + s_red[1][2] + s_red[1][3];
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int u = 0; u < kPre; ++u) {
-    if (u >= n_chunks) break;
-    const float w = s_w[u];
-    acc.x += w * v[u].x; acc.y += w * v[u].y; acc.z += w * v[u].z; acc.w += w * v[u].w;
-  }
-  for (int c = kPre; c < n_chunks; ++c) {
-    const float4 x = __ldcg(src + c * cstride);
-    const float w = s_w[c];
-    acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
-  }
-  const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
-  float4* dst = reinterpret_cast<float4*>(p.out + (int64_t(b) * p.H + hg * kHeadsPerCta + hh) * kD) + tid;
-  *dst = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (p.lse != nullptr && tid == 0)
-    p.lse[int64_t(b) * p.H + hg * kHeadsPerCta + hh] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
-}
-
 }  // namespace
 
+// Chunks of the index list per (sequence, head group), one CTA each, forming one cluster: a
+// power of two up to 16 (at most one chunk per 128-entry tile), the grid within about one
+// CTA per SM.
 int attn_chunks(int B, int H, int top_k, int num_sms) {
   const int n_hg = (H + kHeadsPerCta - 1) / kHeadsPerCta;
-  int c = num_sms / (B * n_hg);
-  const int max_c = top_k / kTile;
-  if (c > max_c) c = max_c;
-  if (c > kMaxChunks) c = kMaxChunks;
-  if (c < 1) c = 1;
+  const int tiles = (top_k + kTile - 1) / kTile;
+  int c = 1;
+  while (c < kMaxCluster && 2 * c <= tiles && int64_t(B) * n_hg * 2 * c <= num_sms) c *= 2;
   return c;
 }
+
+namespace {
+// per device and cluster size 2^i: how many clusters of the attention can be resident at
+// once (0: not asked yet, -1: none)
+int g_attn_max_clusters[64][5] = {};
+
+int max_active_clusters(int chunks) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int li = 0;
+  while ((1 << li) < chunks) ++li;
+  int& known = g_attn_max_clusters[dev & 63][li];
+  if (known == 0) {
+    known = -1;
+    for (auto kf : {k_sparse_attn_tc<false>, k_sparse_attn_tc<true>}) {
+      if (chunks > 8 && cudaFuncSetAttribute(kf, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return known;
+      if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemAttn)) !=
+          cudaSuccess)
+        return known;
+    }
+    cudaLaunchConfig_t q = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = static_cast<unsigned>(chunks);
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.gridDim = dim3(chunks, 1, 1);
+    q.blockDim = dim3(kAttnThreads);
+    q.dynamicSmemBytes = kSmemAttn;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_sparse_attn_tc<false>, &q) == cudaSuccess && n > 0) known = n;
+    (void)cudaGetLastError();
+  }
+  return known;
+}
+}  // namespace
 
 cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream) {
   (void)num_sms;
@@ -837,27 +861,36 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t st
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAttn));
   if (e != cudaSuccess) return e;
-  // Both kernels are programmatic dependents of the kernel before them on the stream: their
-  // CTAs may be scheduled while that kernel finishes (an SM it has left idle can run the
-  // attention prologue: barriers, TMEM, Q conversion) and wait in griddep_wait() before
-  // reading what it produced. A predecessor that never signals early simply completes first.
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int chunks = p.n_chunks;
+  if (chunks < 1 || chunks > kMaxCluster || (chunks & (chunks - 1)) != 0) return cudaErrorInvalidValue;
+  // fewer chunks per cluster until every (sequence, head group) cluster can be resident at
+  // once (a cluster needs all its CTAs, one per SM here, inside one GPC)
+  const int64_t want = int64_t(p.B) * n_hg;
+  while (chunks > 1) {
+    const int n = max_active_clusters(chunks);
+    if (n >= want || (n > 0 && chunks <= 4)) break;
+    chunks >>= 1;
+  }
+  AttnParams pc = p;
+  pc.n_chunks = chunks;
+  // A programmatic dependent of the kernel before it on the stream: its CTAs may be scheduled
+  // while that kernel finishes (an SM it has left idle can run the prologue: barriers, TMEM,
+  // Q conversion) and wait in griddep_wait() before reading what it produced.
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(chunks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_chunks, n_hg, p.B);
+  cfg.gridDim = dim3(chunks, n_hg, p.B);
   cfg.blockDim = dim3(kAttnThreads);
   cfg.dynamicSmemBytes = kSmemAttn;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, p);
-  if (e != cudaSuccess) return e;
-  if (p.n_chunks == 1) return cudaSuccess;
-  cfg.gridDim = dim3(kHeadsPerCta, n_hg, p.B);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, k_attn_combine, p, n_hg);
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, kern, pc);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -44,10 +44,12 @@ struct IndexScoreParams {
 cudaError_t launch_index_score(const IndexScoreParams& p, int num_sms, cudaStream_t stream);
 
 // ----------------------------------------------------------------------------------------
-// Exact top-K select over per-segment fp32 values, given the first-level histogram.
+// Exact top-K select over per-segment fp32 values, given the first-level histogram: a filter
+// kernel over every SM, then one finishing CTA per (problem, sequence).
 // ----------------------------------------------------------------------------------------
-constexpr int kMaxSlices = 512;   // CTAs per sequence in the top-K select kernels
-constexpr int kSelCounters = 4;   // per sequence: n_sure, digit 1 + 1, ticket, spare
+constexpr int kMaxSlices = 512;   // filter CTAs per sequence
+constexpr int kSelRegions = 8;    // kept-entry regions per filter CTA (one per warp)
+constexpr int kSelCounters = 4;   // per sequence: n_sure, digit 1 + 1, spare, spare
 struct SelectProblem {
   const float* values;      // [B][vstride], vstride a multiple of 8
   int64_t vstride;
@@ -60,16 +62,14 @@ struct SelectProblem {
   uint32_t* hist;           // [B][4096] digit-1 histogram (from the scoring kernel)
   uint32_t* hist2;          // [B][4096] digit-2 histogram
   uint32_t* counters;       // [B][kSelCounters]
-  uint32_t* cnt1;           // [B][kMaxSlices] kept entries per slice after filter
-  uint32_t* cnt2;           // [B][kMaxSlices] ... after finish
-  uint64_t* list;           // [B][vstride] (order key << 32) | value index, per-slice regions
+  uint32_t* cnt;            // [B][slices * kSelRegions] kept entries per region
+  uint64_t* list;           // [B][vstride] (order key << 32) | value index, per-region lists
   int32_t* out_idx;         // [B][k]
   float* out_score;         // nullable [B][k]
   int slices;
 };
 // hist, hist2 and counters must be zero on entry; the kernels leave them zero.
-cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B,
-                               cudaStream_t stream);
+cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, cudaStream_t stream);
 int select_slices(int64_t n_values, int B, int num_sms);
 
 // ----------------------------------------------------------------------------------------
@@ -91,10 +91,9 @@ struct AttnParams {
   float sm_scale;
   float* out;               // [B][H][d]
   float* lse;               // nullable [B][H]
-  // split over chunks of the top_k list; partials merged by a combine kernel
-  int n_chunks;             // chunks of the index list, plus the window's chunk when swa != nullptr
-  float* part_o;            // [B][n_hg][n_chunks][64][d]
-  float* part_ml;           // [B][n_hg][n_chunks][64][2]
+  // chunks of the top_k list, one CTA each; the chunk CTAs of a (sequence, head group) form
+  // one cluster and combine their partials in distributed shared memory (1 .. 16)
+  int n_chunks;
   uint32_t* status;
 };
 cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream);
@@ -109,6 +108,7 @@ cudaError_t launch_topk_merge(const float* cand_score, const int32_t* cand_idx, 
                               int32_t* out_local, float* out_score, cudaStream_t stream);
 cudaError_t launch_lse_combine(const float* part_out, const float* part_lse, int n_parts, int64_t n_bh, int d,
                                float* out, float* lse, cudaStream_t stream);
+// chunk CTAs (= cluster size) of the attention for these sizes
 int attn_chunks(int B, int H, int top_k, int num_sms);
 
 }  // namespace fp4kv

@@ -20,8 +20,9 @@
 //  * cvt.rn.satfinite.e2m1x2.f32 rounds to nearest-even on the code and saturates at 6.
 //  * The sign bit of x is OR-ed in separately, so -0 and negative values rounding to zero
 //    keep the sign (code 0x8).
-// Memory: one warp per row, one 16-channel group per lane: 32 B read, 8 B + 1 B written per
-// lane; a warp reads 1 KiB and writes 256 B + 32 B contiguous.
+// Memory: at d = 512 (with 16-byte aligned codes) half a warp per row, two groups per lane,
+// four rows' loads in flight per warp; otherwise one warp per row, one 16-channel group per
+// lane (32 B read, 8 B + 1 B written per lane).
 #include "fp4kv_common.cuh"
 #include "fp4kv_sm100.cuh"
 #include "fp4kv_launch.h"
@@ -106,6 +107,50 @@ __global__ void __launch_bounds__(256) k_kv_quant_fp4(const uint16_t* __restrict
   }
 }
 
+// d = 512, the path of the bulk writes: half a warp per row and two 16-channel groups per
+// lane (64 B read, one 16-byte packed store and one 2-byte scale store per lane), and the
+// loads of kRows rows (kRows / 2 row pairs, 128 B per lane) issued before any is quantized, so
+// that enough bytes are in flight to stream at the HBM rate.
+constexpr int kRows512 = 4;
+__global__ void __launch_bounds__(256) k_kv_quant_fp4_d512(const uint16_t* __restrict__ x, int64_t n_rows,
+                                                           int64_t x_stride, const int64_t* __restrict__ dst_row,
+                                                           uint8_t* __restrict__ packed,
+                                                           uint8_t* __restrict__ scales, int64_t cap_rows) {
+  griddep_launch_dependents();
+  griddep_wait();  // (as in k_kv_quant_fp4)
+  constexpr int kD = 512, kGroups = kD / kGroup;
+  const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
+  const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r0 = warp * kRows512; r0 < n_rows; r0 += nwarps * kRows512) {
+    uint4 v[kRows512 / 2][4];
+    int64_t row[kRows512 / 2];
+#pragma unroll
+    for (int k = 0; k < kRows512 / 2; ++k) {
+      row[k] = r0 + 2 * k + half;
+      if (row[k] < n_rows) {
+        const uint16_t* xr = x + row[k] * x_stride + 2 * kGroup * hl;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[k][j] = ld_stream_v4(xr + 8 * j);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kRows512 / 2; ++k) {
+      if (row[k] >= n_rows) continue;
+      const int64_t dst = dst_row ? dst_row[row[k]] : row[k];
+      if (dst < 0 || dst >= cap_rows) continue;
+      const uint32_t wa[8] = {v[k][0].x, v[k][0].y, v[k][0].z, v[k][0].w, v[k][1].x, v[k][1].y, v[k][1].z, v[k][1].w};
+      const uint32_t wb[8] = {v[k][2].x, v[k][2].y, v[k][2].z, v[k][2].w, v[k][3].x, v[k][3].y, v[k][3].z, v[k][3].w};
+      uint2 pa, pb;
+      uint32_t sa, sb;
+      quant_group(wa, pa, sa);
+      quant_group(wb, pb, sb);
+      *reinterpret_cast<uint4*>(packed + dst * (kD / 2) + 16 * hl) = make_uint4(pa.x, pa.y, pb.x, pb.y);
+      *reinterpret_cast<uint16_t*>(scales + dst * kGroups + 2 * hl) = static_cast<uint16_t>(sa | (sb << 8));
+    }
+  }
+}
+
 // SWA KV write: bf16 rows -> E4M3 codes (round to nearest even, saturating at +-448), one
 // byte per channel ([PyTorchKR] FP4 KV section: the quantization-sensitive SWA KV stays
 // FP8). One warp per row, 16 channels per lane and step: 32 B read, 16 B written per lane.
@@ -183,9 +228,25 @@ cudaError_t launch_kv_quant_fp4(const uint16_t* x, int64_t n_rows, int d, int64_
                                 int64_t cap_rows, int num_sms, cudaStream_t stream) {
   if (n_rows == 0) return cudaSuccess;
   const int threads = 256;
+  const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
+  // (x is 16-byte aligned and its stride a multiple of 8 elements, so its rows are too)
+  if (d == 512 && (reinterpret_cast<uintptr_t>(packed) & 15u) == 0 && (reinterpret_cast<uintptr_t>(scales) & 1u) == 0) {
+    // one resident wave: the grid-stride loop then ends on every SM at about the same time
+    static int per_sm = 0;
+    if (per_sm == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_kv_quant_fp4_d512, threads, 0) != cudaSuccess ||
+         per_sm < 1))
+      per_sm = 2;
+    const int64_t rows_per_block = (threads / 32) * kRows512;
+    int64_t blocks = (n_rows + rows_per_block - 1) / rows_per_block;
+    if (blocks > int64_t(num_sms) * per_sm) blocks = int64_t(num_sms) * per_sm;
+    cudaError_t e = launch_pdl(k_kv_quant_fp4_d512, dim3(static_cast<unsigned>(blocks)), dim3(threads), stream, x,
+                               n_rows, x_stride, dst_row, packed, scales, cap_rows);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   const int64_t rows_per_block = threads / 32;
   int64_t blocks = (n_rows + rows_per_block - 1) / rows_per_block;
-  const int64_t max_blocks = static_cast<int64_t>(num_sms) * 8;
   if (blocks > max_blocks) blocks = max_blocks;
   cudaError_t e = launch_pdl(k_kv_quant_fp4, dim3(static_cast<unsigned>(blocks)), dim3(threads), stream, x, n_rows,
                              d, x_stride, dst_row, packed, scales, cap_rows);

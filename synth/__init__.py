@@ -128,10 +128,12 @@ def attn_query(seed: int, layer: int, B: int, H: int, d: int, device="cpu") -> t
 
 
 def indexer_keys(seed: int, seq: int, rows: torch.Tensor, dk: int = 128,
-                 fp8: bool = True) -> torch.Tensor:
+                 fp8: bool = True, source: int = 0) -> torch.Tensor:
     """Indexer keys [len(rows), dk]: bf16 N(0,1), cast to FP8 E4M3 when fp8 (returned as
-    uint8 codes), else bf16."""
-    h = hash_rows_cols(_key(seed, S_KEYS, seq), rows, dk)
+    uint8 codes), else bf16. `source` selects the key set of one KV source layer (0: the
+    stream every single-source workload uses)."""
+    key = _key(seed, S_KEYS, seq) if source == 0 else _key(seed, S_KEYS, seq, source)
+    h = hash_rows_cols(key, rows, dk)
     k = normal_bf16(h)
     if fp8:
         return k.to(torch.float8_e4m3fn).view(torch.uint8)

@@ -80,3 +80,42 @@ def test_size_overrides_apply_and_are_reported():
     assert "overrides" not in bench.CONFIGS["decode32"]  # the table itself is unchanged
     with pytest.raises(SystemExit):
         bench.apply_overrides(bench.CONFIGS["quant"], ns)  # the sweep has no batch or top-K
+
+
+@pytest.mark.timeout(300)
+def test_cpu_baseline_reports_single_and_threaded_runs():
+    """The oracle baseline is timed single-threaded and with the BLAS pool, and names the
+    host's core count and the threads it used (inputs are built outside the timing)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cb = bench.cpu_baseline("tiny", bench.CONFIGS["tiny"], budget_s=0.5)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0
+    assert cb["nproc"] == os.cpu_count() and cb["cores"] >= 1
+    st = cb["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0 and "sequences" in st["sample"]
+
+
+def test_layered_oracle_sample_runs_every_layer_on_a_small_case():
+    """The 20-layer oracle sample (hier schedule) runs on a reduced size: it calls the
+    Full layer's pool select once, a Reindex per even layer and one attention per layer."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle import fp4kv_oracle as O
+    cfg = dict(bench.CONFIGS["hier"], cap=4096, K=64, npb=32, layers=6)
+    calls = {"hier": 0, "reindex": 0, "attn": 0}
+    orig = (O.hier_pool_select, O.reindex_topk, O.sparse_attn_decode_rows)
+
+    def count(name, f):
+        def g(*a, **k):
+            calls[name] += 1
+            return f(*a, **k)
+        return g
+    try:
+        O.hier_pool_select = count("hier", orig[0])
+        O.reindex_topk = count("reindex", orig[1])
+        O.sparse_attn_decode_rows = count("attn", orig[2])
+        run, work = bench.oracle_sample("hier", cfg, 1)
+        run()
+    finally:
+        O.hier_pool_select, O.reindex_topk, O.sparse_attn_decode_rows = orig
+    assert work == 1.0 and calls == {"hier": 1, "reindex": 3, "attn": 6}

@@ -89,12 +89,14 @@ def test_hierarchical_step_at_full_size(fk):
     idx1 = wl.idx[1][b].cpu().numpy()
     P.check_topk(idx1, sc2, pos, K, "Reindex top-K")
     # attention of layers 1, 2 (over their own indices) and 3 (Reuse: layer 2's indices)
-    for layer, sel in ((0, wl.idx[0][b]), (1, wl.idx[1][b]), (2, wl.idx[1][b])):
-        new_row = P.to_f64(wl.x_new[layer][b].cpu())
+    # (the step wrote every layer's new row with one call: x_new is [layers * B, d], layer-major)
+    for layer, sel in ((0, wl.idx[0][b]), (1, wl.idx[1][b]), (2, wl.idx[1][b]), (19, wl.idx[19][b])):
+        x_layer = wl.x_new[layer * wl.B:(layer + 1) * wl.B]
+        new_row = P.to_f64(x_layer[b].cpu())
         _attn_check(seed, layer, b, wl.q[layer][b], sel.cpu().numpy(), cap, new_row,
                     wl.out[layer][b].cpu().numpy(), wl.lse[layer][b].cpu().numpy(),
                     f"hier layer {layer + 1} attention")
-        _new_row_check(wl, b, wl.packed[layer], wl.scales[layer], wl.x_new[layer], f"hier layer {layer + 1} new row")
+        _new_row_check(wl, b, wl.packed[layer], wl.scales[layer], x_layer, f"hier layer {layer + 1} new row")
 
 
 @pytest.mark.timeout(900)
@@ -160,3 +162,34 @@ def test_decode_step_with_sliding_window_at_full_size(fk):
         P.check_attn(out[b], lse[b], ro, rl, f"attention + window b={b}")
         slot = (cap - 1) % nw
         assert np.array_equal(wl.swa[b, slot].cpu().numpy(), O.swa_quant_fp8(wrows[-1])), "window write"
+
+
+@pytest.mark.timeout(1200)
+def test_csa2_encoder_step_at_full_size(fk):
+    """The pages' encoder schedule: window-only layers 1-2, then 3 groups of 6 (Full + 5
+    Reuse) over each group's own 524,288-entry FP4 KV and FP8 keys, top-K 512."""
+    cfg = bench.CONFIGS["csa2_encoder"]
+    wl = bench.Csa2EncoderWorkload(cfg, fk, torch.device("cuda"))
+    wl.step()
+    torch.cuda.synchronize()
+    seed, cap, K, nw = cfg["seed"], wl.cap, wl.K, wl.n_win
+    for b in (0, wl.B - 1):
+        # the window-only layers: one softmax over the window's E4M3 rows (this step's row
+        # in slot (cap - 1) % nw)
+        for l in range(wl.NS):
+            wrows = P.kv_rows_host(seed, bench.SWA_LAYER + l, b, np.arange(cap - nw, cap), D)
+            wrows[-1] = P.to_f64(wl.x_swa_new[l][b].cpu())
+            v_win = O.e4m3_decode(O.swa_quant_fp8(wrows))
+            ro, rl = O.sparse_attn_decode_rows(P.to_f64(wl.q[l][b].cpu()), v_win, 1.0)
+            P.check_attn(wl.out[l][b].cpu().numpy(), wl.lse[l][b].cpu().numpy(), ro, rl,
+                         f"encoder window-only layer {l + 1} b={b}")
+        for g in (0, wl.NG - 1):
+            src = wl.src[g]
+            sc = P.oracle_scores_seq(wl.qi[g][b], wl.w[g][b], wl.keys[g][b], cap)
+            idx = wl.idx[g][b].cpu().numpy()
+            P.check_topk(idx, sc, np.arange(cap), K, f"encoder group {g + 1} top-K b={b}")
+            new_row = P.to_f64(wl.x_new[g][b].cpu())
+            for l in (src, src + wl.G - 1):  # the group's Full layer and its last Reuse layer
+                _attn_check(seed, src, b, wl.q[l][b], idx, cap, new_row, wl.out[l][b].cpu().numpy(),
+                            wl.lse[l][b].cpu().numpy(), f"encoder layer {l + 1} attention b={b}")
+            _new_row_check(wl, b, wl.packed[g], wl.scales[g], wl.x_new[g], f"encoder group {g + 1} new row")

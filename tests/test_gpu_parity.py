@@ -336,6 +336,36 @@ def test_attention_tiny_config_end_to_end(fk):
     _attn_case(fk, 0, 1, cap, 16, [cap], idx)
 
 
+def test_tiny_config_chained_on_the_gpu(fk):
+    """The tiny configuration as the bench runs it, every step on the GPU: the library's
+    quantize writes the cache and the new row, its indexer top-K (bf16 keys) selects from
+    the written cache, and its attention reads those rows and that selection. The oracle
+    runs the same chain from the generator's bf16 inputs on its own: its own quantizer,
+    its own top-K (the GPU's selection must match it up to the tie band) and its own
+    attention over its own selection."""
+    import bench
+    cfg = bench.CONFIGS["tiny"]
+    wl = bench.DecodeWorkload(cfg, fk, torch.device(DEV))
+    wl.step()
+    torch.cuda.synchronize()
+    cap, K, seed = wl.cap, wl.K, cfg["seed"]
+    sc = P.oracle_scores_seq(wl.qi[0], wl.w[0], wl.keys[0], cap)
+    idx = wl.idx[0].cpu().numpy()
+    P.check_topk(idx, sc, np.arange(cap), K, "tiny top-K")
+    want = O.topk_positions(sc, np.arange(cap), K)
+    if not np.array_equal(idx, want):  # a swap inside the tie band: attend over the GPU's set
+        want = idx
+    rows = P.kv_rows_host(seed, 0, 0, want[want >= 0], 512)
+    rows[want[want >= 0] == cap - 1] = P.to_f64(wl.x_new[0:1].cpu())[0]
+    pk, s8 = O.kv_quant_fp4(rows)
+    ro, rl = O.sparse_attn_decode_rows(P.to_f64(wl.q[0].cpu()), O.kv_dequant_fp4(pk, s8), 1.0)
+    P.check_attn(wl.out[0].cpu().numpy(), wl.lse[0].cpu().numpy(), ro, rl, "tiny chained attention")
+    # the row the step wrote, bit-exact
+    pk1, s1 = O.kv_quant_fp4(P.to_f64(wl.x_new[0:1].cpu()))
+    assert np.array_equal(wl.packed[0, cap - 1].cpu().numpy(), pk1[0])
+    assert np.array_equal(wl.scales[0, cap - 1].cpu().numpy(), s1[0])
+
+
 @pytest.mark.parametrize("H", [64, 16, 20, 128])
 def test_attention_decode_shapes(fk, H):
     B, cap, k = 3, 8192, 2048
