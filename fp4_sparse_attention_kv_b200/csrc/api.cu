@@ -101,7 +101,7 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Workspace layouts
 // ---------------------------------------------------------------------------------------
 struct IndexerLayout {
-  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist2 = 0, counters = 0, zero_end = 0, cnt = 0, list = 0;
+  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist_end = 0, list = 0;
   size_t total = 0;
   int64_t score_stride = 0, bmax_stride = 0;
   int n_probs = 0;
@@ -133,17 +133,10 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
     L.k[1] = npb;
     L.vstride[1] = L.bmax_stride;
   }
-  // hist, hist2 and counters are contiguous: the region that must start at zero (the select
-  // leaves it so)
+  // the first-digit histograms: the region that must start at zero (the select leaves it so)
   L.hist = off;
   off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
-  L.hist2 = off;
-  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kHistBins);
-  L.counters = off;
-  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kSelCounters);
-  L.zero_end = off;
-  L.cnt = off;
-  off += up(sizeof(uint32_t) * L.n_probs * B * fp4kv::kMaxSlices * fp4kv::kSelRegions);
+  L.hist_end = off;
   L.list = off;
   for (int i = 0; i < L.n_probs; ++i) off += up(sizeof(uint64_t) * B * L.vstride[i]);
   L.total = off;
@@ -151,16 +144,22 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
 }
 
 struct AttnLayout {
-  size_t total = 0;
-  int n_chunks = 1;
+  size_t part_ml = 0, part_o = 0, total = 0;
+  int n_chunks = 1, n_hg = 1;
 };
 
-// The attention's workspace is the status word only: its chunk CTAs combine their partials
-// in distributed shared memory.
+// The chunk partials the attention's CTAs exchange (sized for the largest chunk count the
+// launch may use for these sizes; it never uses more).
 AttnLayout attn_layout(int64_t B, int64_t H, int64_t top_k, int sms) {
   AttnLayout L;
+  L.n_hg = static_cast<int>((H + 63) / 64);
   L.n_chunks = fp4kv::attn_chunks(static_cast<int>(B), static_cast<int>(H), static_cast<int>(top_k), sms);
-  L.total = kAlign;
+  size_t off = kAlign;
+  L.part_ml = off;
+  off += up(sizeof(float) * B * L.n_hg * L.n_chunks * 64 * 2);
+  L.part_o = off;
+  off += up(sizeof(float) * B * L.n_hg * L.n_chunks * 64 * 512);
+  L.total = off;
   return L;
 }
 
@@ -448,19 +447,15 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
     P.npb = n_pool_blocks;
     P.k = static_cast<int>(L.k[i]);
     P.hist = p.hist + int64_t(i) * B * fp4kv::kHistBins;
-    P.hist2 = reinterpret_cast<uint32_t*>(base + L.hist2) + int64_t(i) * B * fp4kv::kHistBins;
-    P.counters = reinterpret_cast<uint32_t*>(base + L.counters) + int64_t(i) * B * fp4kv::kSelCounters;
-    P.cnt = reinterpret_cast<uint32_t*>(base + L.cnt) + int64_t(i) * B * fp4kv::kMaxSlices * fp4kv::kSelRegions;
     P.list = reinterpret_cast<uint64_t*>(base + list_off);
     list_off += up(sizeof(uint64_t) * B * L.vstride[i]);
     P.out_idx = (i == 0) ? out_idx : out_pool;
     P.out_score = (i == 0) ? out_score : nullptr;
-    const int64_t nvals = (kind == 1) ? int64_t(n_pool_blocks) * 8 : (i == 0 ? cap : (cap + 7) / 8);
-    P.slices = fp4kv::select_slices(nvals, B, sms);
+    P.status = p.status;
   }
   {
     prof::Scope ps(2, stream);
-    e = fp4kv::launch_topk_select(probs, L.n_probs, B, stream);
+    e = fp4kv::launch_topk_select(probs, L.n_probs, B, sms, stream);
   }
   if (e != cudaSuccess) return cuda_fail(e, "top-k select");
   return ok();
@@ -541,6 +536,8 @@ static fp4kv_status run_attn(const uint16_t* q, int32_t B, int32_t H, int32_t d,
   p.out = out;
   p.lse = lse;
   p.n_chunks = L.n_chunks;
+  p.part_ml = reinterpret_cast<float*>(base + L.part_ml);
+  p.part_o = reinterpret_cast<float*>(base + L.part_o);
   p.status = reinterpret_cast<uint32_t*>(base);
   cudaError_t e;
   {
@@ -666,10 +663,10 @@ fp4kv_status fp4kv_indexer_topk_noalloc(const void* q, const float* w, int32_t H
   st = noalloc_scratch(&ws);
   if (st != FP4KV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the histograms and counters must start at zero. The status word at the head is left
+  // the histograms must start at zero. The status word at the head is left
   // as it is: a bounded wait that gave up in an earlier call stays visible until
   // fp4kv_noalloc_status reads (and clears) it.
-  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.zero_end - L.hist, s);
+  cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + L.hist, 0, L.hist_end - L.hist, s);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc: clearing scratch");
   return run_indexer(kind, q, w, H_I, keys, key_dtype, key_scale, cap, seq_lens, B, pool,
                      pool ? n_pool_blocks : 0, top_k, out_idx, nullptr, out_score, ws, L.total, s);

@@ -36,11 +36,10 @@
 //    once at the end, when O^T is staged in shared memory and leaves in one bulk store.
 //  Per-chunk barriers let the next tile's dequantization overlap the current tile's P.V.
 //  * Chunks of the index list go to different CTAs, and the chunk CTAs of one (sequence,
-//    head group) form one thread-block cluster. At the end they exchange their per-head
-//    reference m and row sum l through distributed shared memory, each stages its O scaled
-//    by its log-sum-exp weight 2^(m_c - M) / L, and CTA r sums its share of the output
-//    dims over the cluster and writes them: no partials pass through global memory and no
-//    second kernel runs.
+//    head group) form one thread-block cluster. At the end each writes its partial (O and
+//    the per-head reference m and row sum l) to the workspace, where it stays in L2; after
+//    one cluster barrier CTA r sums its share of the output dims over the chunks with the
+//    log-sum-exp weights and writes them, so no second kernel runs.
 //  * With a sliding window (the pages' SWA branch, its KV kept in FP8), the last chunk's CTA
 //    runs one more tile: the window's E4M3 rows (exact in fp16), in the same softmax as the
 //    selected rows, so the window and the sparse selection share one normalisation.
@@ -309,6 +308,52 @@ FP4KV_DEV bool load_dequant_win(uint8_t* smem, uint64_t* bars, const uint8_t* wi
     }
   }
   return ok;
+}
+
+// CTA `rank` of a cluster of C chunk CTAs: sums 16-byte units (head, 4 dims) of its dim slice
+// [rank * 512 / C, +512 / C) over the C chunk partials with the per-(chunk, head) weights sW
+// and writes them. Each thread keeps 16 loads in flight: 16 / C units over the C chunks.
+template <int C>
+FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint32_t rank, int64_t part0,
+                             const float* sW) {
+  constexpr int kSlice4 = kD / 4 / C;  // 16-byte units per head in the slice
+  constexpr int kPer = 16 / C;         // units per thread and batch
+  const int tid = threadIdx.x;
+  const int n_units = nh * kSlice4;
+  const int d0 = static_cast<int>(rank) * kSlice4 * 4;
+  const bool al16 = (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
+  const float4* part4 = reinterpret_cast<const float4*>(p.part_o + part0 * (kHeadsPerCta * kD));
+  for (int u0 = tid; u0 < n_units; u0 += kAttnThreads * kPer) {
+    float4 v[kPer][C];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int u = u0 + j * kAttnThreads;
+      const int h = u / kSlice4, d = d0 + 4 * (u % kSlice4);
+#pragma unroll
+      for (int c = 0; c < C; ++c)
+        v[j][c] = u < n_units ? __ldcg(part4 + (int64_t(c) * kHeadsPerCta * kD + h * kD + d) / 4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int u = u0 + j * kAttnThreads;
+      if (u >= n_units) continue;
+      const int h = u / kSlice4, d = d0 + 4 * (u % kSlice4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const float w = sW[c * kHeadsPerCta + h];
+        acc.x += w * v[j][c].x; acc.y += w * v[j][c].y; acc.z += w * v[j][c].z; acc.w += w * v[j][c].w;
+      }
+      float* dst = p.out + (int64_t(b) * p.H + hbase + h) * kD + d;
+      if (al16) {
+        *reinterpret_cast<float4*>(dst) = acc;
+      } else {  // the output is only 8-byte aligned
+        reinterpret_cast<float2*>(dst)[0] = make_float2(acc.x, acc.y);
+        reinterpret_cast<float2*>(dst)[1] = make_float2(acc.z, acc.w);
+      }
+    }
+  }
 }
 
 // kWin: with the sliding-window tile (a separate instantiation, so that the plain sparse
@@ -707,22 +752,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   }
 
   // ---- combine the chunk CTAs of this (sequence, head group): one cluster ----
-  // Every thread of every CTA of the cluster passes the cluster barriers below.
+  // Each CTA writes its partial -- O^T as [64 heads][512 dims] fp32, unscaled, straight from
+  // TMEM, and (m, l) per head -- to the workspace (it stays in L2). One cluster barrier
+  // makes every chunk's partial visible to the others; then CTA `rank` sums dims
+  // [rank * 512 / C, +512 / C) of every head over the chunks with the log-sum-exp weights
+  // 2^(m_c - M) / (2^6 L) (O holds p * 2^6) and writes them.
   __syncthreads();
-  cluster_sync_all();  // (A) every CTA's per-head reference m and row sum l are visible
   const uint32_t C = cluster_nctas(), rank = cluster_ctarank();
-  if (tid < kHeadsPerCta) {
-    // per head: M = max_c m_c over the CTAs with rows, Lt = sum_c 2^(m_c - M) l_c; this CTA's
-    // weight 2^(m_r - M) / (2^6 Lt) (O holds p * 2^6); lse = M ln 2 + ln Lt
-    const int h = tid;
-    float lc[kMaxCluster], mc[kMaxCluster];
+  const int64_t part0 = (int64_t(b) * gridDim.y + hg) * C;  // this (sequence, head group)'s first chunk
+  {
+    float* po = p.part_o + (part0 + rank) * (kHeadsPerCta * kD);
+    if (warp < kSoftWarps) {
+      const int q4 = warp & 3, h0 = 32 * (warp >> 2), e = 32 * q4 + lane;
+      const uint32_t lane_addr = uint32_t(32 * q4) << 16;
+      const bool have = n_tiles > 0 && *s_fail == 0u;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (have) {
+          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c) {  // (all remote loads first, then their use)
-      lc[c] = 0.0f;
+          for (int k = 0; k < 32; ++k) r[k] = 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < 32; ++k) __stcg(po + (h0 + k) * kD + 128 * c + e, __uint_as_float(r[k]));
+      }
+    }
+    if (tid < kHeadsPerCta) {
+      const float l = sL[tid];
+      float* pml = p.part_ml + ((part0 + rank) * kHeadsPerCta + tid) * 2;
+      __stcg(pml, l > 0.0f ? sM[tid] : -INFINITY);
+      __stcg(pml + 1, l);
+    }
+  }
+  cluster_sync_all();  // every chunk CTA's partial is in the workspace and visible
+  float* sW = reinterpret_cast<float*>(smem + kOffV);  // [C][64] weights (V_hat is free now)
+  if (tid < kHeadsPerCta) {
+    const int h = tid;
+    float mc[kMaxCluster], lc[kMaxCluster];
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {  // (all loads first, then their use)
       mc[c] = -INFINITY;
+      lc[c] = 0.0f;
       if (c < static_cast<int>(C)) {
-        lc[c] = dsmem_ld_f32(dsmem_map(&sL[h], static_cast<uint32_t>(c)));
-        mc[c] = dsmem_ld_f32(dsmem_map(&sM[h], static_cast<uint32_t>(c)));
+        const float* pml = p.part_ml + ((part0 + c) * kHeadsPerCta + h) * 2;
+        mc[c] = __ldcg(pml);
+        lc[c] = __ldcg(pml + 1);
       }
     }
     float M = -INFINITY;
@@ -733,65 +810,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
     for (int c = 0; c < kMaxCluster; ++c)
       if (lc[c] > 0.0f) Lt += exp2f(mc[c] - M) * lc[c];
-    const float lo = sL[h];
-    sA[h] = (lo > 0.0f && Lt > 0.0f) ? exp2f(sM[h] - M) / (kPScale * Lt) : 0.0f;
+    const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c)
+      if (c < static_cast<int>(C)) sW[c * kHeadsPerCta + h] = lc[c] > 0.0f ? exp2f(mc[c] - M) * inv : 0.0f;
     if (rank == 0 && p.lse != nullptr && h < nh)
       p.lse[int64_t(b) * p.H + hbase + h] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
   }
   __syncthreads();
-  // this CTA's O^T, scaled by its weight, as [64 heads][512 dims] fp32 in the V_hat region
-  // (free: the last P.V has completed): one 32-column TMEM load per dim tile
-  float* stage = reinterpret_cast<float*>(smem + kOffV);
-  if (warp < kSoftWarps) {
-    const int q4 = warp & 3, h0 = 32 * (warp >> 2), e = 32 * q4 + lane;
-    const uint32_t lane_addr = uint32_t(32 * q4) << 16;
-    const bool have = n_tiles > 0 && *s_fail == 0u;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
-      if (have) {
-        tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int k = 0; k < 32; ++k) r[k] = 0u;
-      }
-#pragma unroll
-      for (int k = 0; k < 32; ++k) stage[(h0 + k) * kD + 128 * c + e] = __uint_as_float(r[k]) * sA[h0 + k];
-    }
+  switch (C) {  // (only the instance that runs is ever fetched)
+    case 1: combine_slice<1>(p, b, hbase, nh, rank, part0, sW); break;
+    case 2: combine_slice<2>(p, b, hbase, nh, rank, part0, sW); break;
+    case 4: combine_slice<4>(p, b, hbase, nh, rank, part0, sW); break;
+    case 8: combine_slice<8>(p, b, hbase, nh, rank, part0, sW); break;
+    default: combine_slice<16>(p, b, hbase, nh, rank, part0, sW); break;
   }
-  __syncthreads();
-  cluster_sync_all();  // (B) every CTA's scaled O is staged
-  {
-    // CTA `rank` sums dims [rank * 512 / C, +512 / C) of all 64 heads over the cluster's CTAs
-    // and writes them: 16-byte units, consecutive threads on consecutive dims of a head
-    const int slice4 = kD / 4 / static_cast<int>(C);  // float4 units per head in the slice
-    const int d0 = static_cast<int>(rank) * slice4 * 4;
-    const bool al16 = (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
-    for (int u = tid; u < nh * slice4; u += kAttnThreads) {
-      const int h = u / slice4, d = d0 + 4 * (u % slice4);
-      // all the CTAs' values are loaded before they are added (independent remote loads)
-      float4 v[kMaxCluster];
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c)
-        if (c < static_cast<int>(C)) v[c] = dsmem_ld_f32x4(dsmem_map(stage + h * kD + d, static_cast<uint32_t>(c)));
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < kMaxCluster; ++c) {
-        if (c < static_cast<int>(C)) {
-          acc.x += v[c].x; acc.y += v[c].y; acc.z += v[c].z; acc.w += v[c].w;
-        }
-      }
-      float* dst = p.out + (int64_t(b) * p.H + hbase + h) * kD + d;
-      if (al16) {
-        *reinterpret_cast<float4*>(dst) = acc;
-      } else {  // the output is only 8-byte aligned
-        reinterpret_cast<float2*>(dst)[0] = make_float2(acc.x, acc.y);
-        reinterpret_cast<float2*>(dst)[1] = make_float2(acc.z, acc.w);
-      }
-    }
-  }
-  cluster_sync_all();  // (C) no CTA leaves while another still reads its shared memory
 
   tc_fence_before();
   __syncthreads();

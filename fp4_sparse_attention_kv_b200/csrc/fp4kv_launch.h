@@ -44,12 +44,9 @@ struct IndexScoreParams {
 cudaError_t launch_index_score(const IndexScoreParams& p, int num_sms, cudaStream_t stream);
 
 // ----------------------------------------------------------------------------------------
-// Exact top-K select over per-segment fp32 values, given the first-level histogram: a filter
-// kernel over every SM, then one finishing CTA per (problem, sequence).
+// Exact top-K select over per-segment fp32 values, given the first-level histogram: one
+// kernel, one thread-block cluster per (problem, sequence).
 // ----------------------------------------------------------------------------------------
-constexpr int kMaxSlices = 512;   // filter CTAs per sequence
-constexpr int kSelRegions = 8;    // kept-entry regions per filter CTA (one per warp)
-constexpr int kSelCounters = 4;   // per sequence: n_sure, digit 1 + 1, spare, spare
 struct SelectProblem {
   const float* values;      // [B][vstride], vstride a multiple of 8
   int64_t vstride;
@@ -59,18 +56,14 @@ struct SelectProblem {
   const int32_t* pool;      // mode 2
   int npb;
   int k;
-  uint32_t* hist;           // [B][4096] digit-1 histogram (from the scoring kernel)
-  uint32_t* hist2;          // [B][4096] digit-2 histogram
-  uint32_t* counters;       // [B][kSelCounters]
-  uint32_t* cnt;            // [B][slices * kSelRegions] kept entries per region
-  uint64_t* list;           // [B][vstride] (order key << 32) | value index, per-region lists
+  uint32_t* hist;           // [B][4096] digit-1 histogram (from the scoring kernel); the
+                            // select reads it and leaves it zeroed
+  uint64_t* list;           // [B][vstride] overflow of the kept-entry lists
   int32_t* out_idx;         // [B][k]
   float* out_score;         // nullable [B][k]
-  int slices;
+  uint32_t* status;         // workspace status word (bit 0: a bounded wait gave up)
 };
-// hist, hist2 and counters must be zero on entry; the kernels leave them zero.
-cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, cudaStream_t stream);
-int select_slices(int64_t n_values, int B, int num_sms);
+cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, int num_sms, cudaStream_t stream);
 
 // ----------------------------------------------------------------------------------------
 // Sparse attention decode
@@ -91,9 +84,11 @@ struct AttnParams {
   float sm_scale;
   float* out;               // [B][H][d]
   float* lse;               // nullable [B][H]
-  // chunks of the top_k list, one CTA each; the chunk CTAs of a (sequence, head group) form
-  // one cluster and combine their partials in distributed shared memory (1 .. 16)
+  // chunks of the top_k list, one CTA each (1 .. 16); the chunk CTAs of a (sequence, head
+  // group) form one cluster and combine their partials after one cluster barrier
   int n_chunks;
+  float* part_o;            // [B][n_hg][n_chunks][64][d] fp32 partial outputs
+  float* part_ml;           // [B][n_hg][n_chunks][64][2] per-head reference and row sum
   uint32_t* status;
 };
 cudaError_t launch_sparse_attn(const AttnParams& p, int num_sms, cudaStream_t stream);

@@ -227,8 +227,8 @@ FP4KV_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch
 FP4KV_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------------
-// Thread-block clusters: rank and size, barrier, distributed shared memory (documented PTX:
-// %cluster_ctarank / %cluster_nctarank, barrier.cluster, mapa, ld/st.shared::cluster)
+// Thread-block clusters: rank, size and barrier (documented PTX: %cluster_ctarank,
+// %cluster_nctarank, barrier.cluster)
 // ---------------------------------------------------------------------------------------
 FP4KV_DEV uint32_t cluster_ctarank() {
   uint32_t r;
@@ -244,32 +244,5 @@ FP4KV_DEV uint32_t cluster_nctas() {
 // visible to reads after it, cluster-wide.
 FP4KV_DEV void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Address of `p` (this CTA's shared memory) in the shared memory of CTA `rank` of the cluster.
-FP4KV_DEV uint32_t dsmem_map(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-// Loads from distributed shared memory (volatile, with a memory clobber: never moved across
-// a cluster barrier; issue several in a row before using any, so that they overlap).
-FP4KV_DEV uint32_t dsmem_ld_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-FP4KV_DEV float dsmem_ld_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-FP4KV_DEV float4 dsmem_ld_f32x4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-  return v;
-}
-FP4KV_DEV void dsmem_st_u64(uint32_t addr, uint64_t v) {
-  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
 }  // namespace fp4kv

@@ -112,26 +112,8 @@ FP4KV_DEV void regroup_scales(const uint8_t* raw, int blk_stride, uint8_t* block
   __syncwarp();
 }
 
-// Warp-collective histogram update: the lanes with `valid` add one to bin `bin`; lanes that
-// share a bin are counted by one atomic (a sequence's scores fall into few of the 4096 bins,
-// so per-lane atomics would serialise on the same shared-memory words).
-FP4KV_DEV void hist_add_warp(uint32_t* hist, bool valid, uint32_t bin, int lane) {
-  const uint32_t key = valid ? bin : 0xffffffffu;
-  const uint32_t peers = __match_any_sync(0xffffffffu, key);
-  if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
-}
-
 // named barrier of one epilogue warpgroup (ids 1 and 2)
 FP4KV_DEV void epi_sync(int group) { asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(kEpiThreads)); }
-// the same barrier, ORing a predicate over the warpgroup: a decision all its warps share
-FP4KV_DEV bool epi_any(int group, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, %2, %3, pi;\n"
-      " selp.u32 %0, 1, 0, po;\n}"
-      : "=r"(r) : "r"(v ? 1u : 0u), "r"(1 + group), "n"(kEpiThreads) : "memory");
-  return r != 0;
-}
 
 struct Tiles {
   int64_t begin, end, per_seq;
@@ -504,14 +486,18 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
 #pragma unroll
         for (int h = 0; h < N; ++h) wv[h] = h < p.H_I ? p.w[int64_t(cur_b) * p.H_I + h] : 0.0f;
       }
-      const bool got = mbar_wait_warp(&tfull[acc], aph);
-      if (!got && lane == 0) {
-        atomicOr(p.status, kFlagWaitTimeout);
-        *s_abort = 1;
+      // Once a wait has given up (here or in another role) the warp stops waiting and working
+      // but keeps walking the same tiles, so every warp of the warpgroup reaches the same
+      // histogram flushes (named barriers) and none is left waiting at one alone.
+      bool live = __shfl_sync(0xffffffffu, *s_abort, 0) == 0u;
+      if (live) {
+        live = mbar_wait_warp(&tfull[acc], aph);
+        if (!live && lane == 0) {
+          atomicOr(p.status, kFlagWaitTimeout);
+          *s_abort = 1;
+        }
       }
-      // leave together: every warp of the warpgroup takes the same decision, so none is left
-      // waiting alone at the warpgroup's barrier
-      if (epi_any(group, !got || *s_abort != 0)) break;
+      if (!live) continue;
       tc_fence_after();
       uint32_t r[N];
 #pragma unroll
@@ -536,8 +522,8 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
         if (valid) {
           if (p.key_scale != nullptr) s *= p.key_scale[seq_base + pos];
           srow[pos] = s;
+          if (p.hist != nullptr) atomicAdd(&s_hist[order_key(s) >> (32 - kHistBits)], 1u);
         }
-        if (p.hist != nullptr) hist_add_warp(s_hist, valid, order_key(s) >> (32 - kHistBits), lane);
         if (p.bmax != nullptr) {
           float m = valid ? s : -INFINITY;
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
@@ -558,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
           if (valid && p.key_scale != nullptr) s *= p.key_scale[seq_base + pos];
           srow[slot * kPoolBlock + (row % kPoolBlock)] = valid ? s : -INFINITY;
         }
-        if (p.hist != nullptr) hist_add_warp(s_hist, valid, order_key(s) >> (32 - kHistBits), lane);
+        if (valid && p.hist != nullptr) atomicAdd(&s_hist[order_key(s) >> (32 - kHistBits)], 1u);
       }
     }
     if (cur_b >= 0 && p.hist != nullptr) flush(cur_b);

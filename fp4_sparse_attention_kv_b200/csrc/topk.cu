@@ -7,22 +7,26 @@
 // 인덱서로 인덱싱 비용을 컨텍스트 길이에서 분리하기": the blocks with the highest block max).
 //
 // Values are mapped to order-preserving 32-bit keys. The scoring kernel has already built a
-// histogram of the top 12 key bits (digit 1) of every sequence. Two kernels follow:
-//  filter  (every SM busy: S slices per sequence, 8 warps per slice, each warp one contiguous
-//          sub-slice read with fully coalesced 16-byte loads, two batches in flight) finds the
-//          digit-1 value b1 of the K-th largest key, keeps the keys with digit 1 >= b1 of its
-//          sub-slice in position order (a ballot prefix inside the warp, no block barrier) in
-//          the sub-slice's own region of the list array, and histograms the next 12 bits
-//          (digit 2) of the keys with digit 1 == b1;
-//  finish  (a programmatic dependent; one CTA per sequence) finds the digit-2 value b2 of the
-//          K-th key, stages the few thousand kept entries in shared memory (regions in
-//          position order), resolves the (b1, b2) bin exactly only when it is taken in part
-//          (the last 8 key bits, then the lowest positions among equal keys), and writes the
-//          selection with one ordered compaction: positions come out ascending without a
-//          sort (the pool mode, whose positions need not grow with the value index, sorts
-//          its at most 4096 selected pairs). It also zeroes the histograms and counters,
-//          leaving the workspace ready for the next call.
-// No CTA ever waits on another CTA.
+// histogram of the top 12 key bits (digit 1) of every sequence. One kernel follows, with one
+// thread-block cluster of C CTAs per (problem, sequence); CTA r owns slice r of the values,
+// warp w of it sub-slice w (slices and sub-slices in position order):
+//  1. every CTA finds the digit-1 value b1 of the K-th largest key from the histogram, as two
+//     float thresholds: "digit 1 >= b1" is v >= f_lo, "digit 1 > b1" is v >= f_hi;
+//  2. each warp streams its sub-slice through a ring of shared-memory buffers filled by bulk
+//     asynchronous copies (the copy engine keeps every buffer's bytes in flight), keeps the
+//     values >= f_lo in position order (a warp prefix, no block barrier) in its own list, and
+//     the CTA histograms the next 12 key bits (digit 2) of the keys with digit 1 == b1;
+//  3. the CTAs add up the digit-2 histograms through distributed shared memory (CTA r sums
+//     segment r of the bins in place) and every CTA finds the digit-2 value b2 of the K-th key;
+//  4. only when the (b1, b2) bin is taken in part: the last 8 key bits, then the lowest
+//     positions among the keys equal to the K-th key, are resolved the same way;
+//  5. every CTA counts what it takes, reads the counts of the CTAs before it and writes its
+//     positions at that offset: ascending without a sort. A Reindex pool whose blocks are not
+//     in ascending order gathers its at most 4096 selected pairs in CTA 0, which sorts them.
+// The CTAs also clear the scoring kernel's histogram for the next call. Cluster barriers are
+// the only synchronisation between CTAs; every mbarrier wait is bounded in time.
+// Kernels that live a few microseconds run mostly from a cold instruction cache, so the loop
+// bodies here are kept short.
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
 #include "fp4kv_sm100.cuh"
@@ -30,21 +34,40 @@
 namespace fp4kv {
 namespace {
 
-constexpr int kFThreads = 256;               // filter CTA
-constexpr int kFWarps = kFThreads / 32;      // sub-slices per slice
-constexpr int kGroups = 8;                   // 16-byte loads per lane and batch
-constexpr int kWarpBatch = 32 * 4 * kGroups; // 1024 values
-constexpr int kNThreads = 1024;              // finish CTA
-constexpr int kNWarps = kNThreads / 32;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 1024;              // values per ring buffer (4 KiB)
+constexpr int kMaxDepth = 4;              // ring buffers per warp
+constexpr int kWarpCap = 512;             // kept entries per warp held in shared memory
+constexpr int kMaxCluster = 16;
 constexpr int kMaxSel = 4096;
 constexpr int kMaxProblems = 2;
-constexpr int kStage = 12288;                // kept entries the finish CTA stages in shared memory
-static_assert(kFWarps == kSelRegions, "one kept-entry region per filter warp");
-static_assert(kMaxSlices * kFWarps <= 4 * kNThreads, "region counts: four per finishing thread");
 
 struct SelectArgs {
   SelectProblem p[kMaxProblems];
+  int depth;  // ring buffers per warp
 };
+
+struct SelSmem {
+  uint32_t h2[kHistBins];               // digit-2 histogram; segment r is summed in place
+  uint64_t list[kWarps][kWarpCap];      // kept entries: (order key << 32) | value index
+  uint64_t bar[kWarps][kMaxDepth];      // ring mbarriers
+  uint32_t h8[256];                     // last 8 key bits of the (b1, b2) bin
+  uint32_t hp[2][256];                  // position digits among the keys equal to the K-th
+  uint32_t hsum[256];                   // a 256-bin histogram summed over the cluster
+  uint32_t wcnt[kWarps];                // kept entries per warp
+  uint32_t wsel[kWarps];                // selected entries per warp
+  uint32_t w[kWarps];                   // block scans
+  uint32_t res[4];
+  uint32_t sure;                        // keys of this CTA with digit 1 > b1
+  uint32_t seg_total;                   // sum of this CTA's summed digit-2 segment
+  uint32_t sel_total;                   // entries this CTA selects
+  uint32_t bc[4];                       // block broadcasts
+};
+// the ring follows; after the filter phase CTA 0 reuses it for the pool mode's sorted pairs
+constexpr size_t kSmemFixed = (sizeof(SelSmem) + 127) / 128 * 128;
+size_t select_smem(int depth) { return kSmemFixed + size_t(kWarps) * depth * kChunk * sizeof(float); }
+static_assert(kWarps * kChunk * sizeof(float) >= kMaxSel * sizeof(uint64_t), "pairs fit a depth-1 ring");
 
 FP4KV_DEV int64_t n_values(const SelectProblem& P, int b) {
   int64_t len = P.seq_lens[b];
@@ -55,19 +78,6 @@ FP4KV_DEV int64_t n_values(const SelectProblem& P, int b) {
     return nb < P.vstride ? nb : P.vstride;
   }
   return int64_t(P.npb) * 8;
-}
-
-// Slice s of n values over `slices` CTAs, sub-slice w of it: [lo, hi), multiples of 128
-// values (whole 16-byte lane groups of a warp) except at n.
-struct Region {
-  int64_t lo, hi;
-};
-FP4KV_DEV Region region_of(int64_t n, int slices, int s, int w) {
-  const int64_t per_s = ((n + slices - 1) / slices + kWarpBatch - 1) / kWarpBatch * kWarpBatch;
-  const int64_t slo = min(n, per_s * s), shi = min(n, slo + per_s);
-  const int64_t per_w = ((shi - slo + kFWarps - 1) / kFWarps + 127) / 128 * 128;
-  const int64_t lo = min(shi, slo + per_w * w);
-  return {lo, min(shi, lo + per_w)};
 }
 
 FP4KV_DEV int64_t position_of(const SelectProblem& P, int b, int64_t i) {
@@ -81,6 +91,33 @@ FP4KV_DEV int32_t ent_idx(uint64_t c) { return static_cast<int32_t>(c & 0xffffff
 FP4KV_DEV int digit1(uint32_t key) { return static_cast<int>(key >> 20); }
 FP4KV_DEV int digit2(uint32_t key) { return static_cast<int>((key >> 8) & 0xfffu); }
 
+// distributed shared memory (the cluster's CTAs): the address of `p` in CTA `rank`, and loads
+// and stores there (volatile with a memory clobber: never moved across a cluster barrier)
+FP4KV_DEV uint32_t dsmem_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+FP4KV_DEV uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+FP4KV_DEV void dsmem_st64(uint32_t addr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+// sum over the cluster's CTAs of the u32 at `p` (each CTA's copy); the loads are all issued
+// before any is added
+FP4KV_DEV uint32_t cluster_sum(const uint32_t* p, uint32_t C) {
+  uint32_t v[kMaxCluster];
+#pragma unroll
+  for (uint32_t q = 0; q < kMaxCluster; ++q) v[q] = q < C ? dsmem_ld(dsmem_map(p, q)) : 0u;
+  uint32_t s = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxCluster; ++q) s += v[q];
+  return s;
+}
+
 FP4KV_DEV uint32_t warp_incl_scan(uint32_t x) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -91,54 +128,51 @@ FP4KV_DEV uint32_t warp_incl_scan(uint32_t x) {
   return x;
 }
 
-// Block-wide exclusive prefix sum over the kT threads; *total gets the block sum. s_w: kT / 32
-// words. Every thread calls it (barriers inside).
-template <int kT>
+// Block-wide exclusive prefix sum; *total gets the block sum. Every thread calls it.
 FP4KV_DEV uint32_t block_excl_scan(uint32_t v, uint32_t* s_w, uint32_t* total) {
-  constexpr int kW = kT / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const uint32_t x = warp_incl_scan(v);
   if (lane == 31) s_w[w] = x;
   __syncthreads();
-  if (w == 0) {
-    uint32_t t = lane < kW ? s_w[lane] : 0u;
-    t = warp_incl_scan(t);
-    if (lane < kW) s_w[lane] = t;
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) {
+    const uint32_t t = s_w[i];
+    before += i < w ? t : 0u;
+    all += t;
   }
   __syncthreads();
-  const uint32_t excl = x - v + (w > 0 ? s_w[w - 1] : 0u);
-  *total = s_w[kW - 1];
-  __syncthreads();
-  return excl;
+  *total = all;
+  return x - v + before;
 }
 
-// Block-wide (kT threads): thread t owns kPer bins counted from the top, h[nbins - kPer (t+1)
-// .. nbins - kPer t), given in vals[] highest first. Finds the bin d at which the count from
-// the top reaches r (r >= 1): d, the count above it and its own count. If the total is below
-// r: d = -1, above = total, cnt = 0. Every thread calls it.
-template <int kT, int kPer>
-FP4KV_DEV void block_find_desc(const uint32_t (&vals)[kPer], int nbins, uint32_t r, int* d_out,
+// Block-wide: thread t owns `per` bins counted from the top, h[nbins - per (t + 1) .. nbins -
+// per t), given in vals[] highest first. Finds the bin d at which the count from the top
+// reaches r (r >= 1): d, the count above it and its own count. If the total is below r:
+// d = -1, above = total, cnt = 0. Every thread calls it.
+template <int kPer>
+FP4KV_DEV void block_find_desc(const uint32_t (&vals)[kPer], int per, int nbins, uint32_t r, int* d_out,
                                uint32_t* above_out, uint32_t* cnt_out, uint32_t* s_w, uint32_t* s_res) {
   const int tid = threadIdx.x;
-  const int hi = nbins - kPer * tid;
+  const int hi = nbins - per * tid;
   uint32_t sum = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i)
-    if (hi - 1 - i >= 0) sum += vals[i];
+    if (i < per && hi - 1 - i >= 0) sum += vals[i];
   if (tid == 0) {
     s_res[0] = 0xffffffffu;
     s_res[1] = 0;
     s_res[2] = 0;
   }
   uint32_t total;
-  const uint32_t excl = block_excl_scan<kT>(sum, s_w, &total);  // (its barriers order s_res)
+  const uint32_t excl = block_excl_scan(sum, s_w, &total);  // (its barriers order s_res)
   if (total < r) {
     if (tid == 0) s_res[1] = total;
   } else if (excl < r && excl + sum >= r) {
     uint32_t acc = excl;
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      if (hi - 1 - i >= 0) {
+      if (i < per && hi - 1 - i >= 0) {
         if (acc + vals[i] >= r) {
           s_res[0] = static_cast<uint32_t>(hi - 1 - i);
           s_res[1] = acc;
@@ -156,19 +190,17 @@ FP4KV_DEV void block_find_desc(const uint32_t (&vals)[kPer], int nbins, uint32_t
   __syncthreads();
 }
 
-// Block-wide ascending bitonic sort of N = kNThreads * E keys held in shared memory.
-// Each thread keeps E consecutive keys in registers: strides below E are exchanged inside
-// the thread, strides up to 16 E through warp shuffles, and only the widest strides through
-// shared memory (one barrier pair each).
-template <typename T, int E>
-__device__ void block_sort(T* s) {
-  constexpr int N = kNThreads * E;
+// Block-wide ascending bitonic sort of kMaxSel keys held in shared memory (16 per thread).
+// Strides below 16 are exchanged inside a thread, strides up to 256 through warp shuffles,
+// and only the widest ones through shared memory (one barrier pair each).
+__device__ void block_sort_pairs(uint64_t* s) {
+  constexpr int E = kMaxSel / kThreads;
   const int tid = threadIdx.x;
-  T v[E];
+  uint64_t v[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) v[e] = s[tid * E + e];
 #pragma unroll
-  for (int size = 2; size <= N; size <<= 1) {
+  for (int size = 2; size <= kMaxSel; size <<= 1) {
 #pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       if (stride >= 32 * E) {
@@ -179,7 +211,7 @@ __device__ void block_sort(T* s) {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int i = tid * E + e;
-          const T p = s[i ^ stride];
+          const uint64_t p = s[i ^ stride];
           const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
           v[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
         }
@@ -187,16 +219,16 @@ __device__ void block_sort(T* s) {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int i = tid * E + e;
-          const T p = __shfl_xor_sync(0xffffffffu, v[e], stride / E);
+          const uint64_t p = __shfl_xor_sync(0xffffffffu, v[e], stride / E);
           const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
           v[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
         }
       } else {
-        T nv[E];
+        uint64_t nv[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int i = tid * E + e;
-          const T p = v[e ^ stride];
+          const uint64_t p = v[e ^ stride];
           const bool keep_min = ((i & stride) == 0) == ((i & size) == 0);
           nv[e] = keep_min ? (v[e] < p ? v[e] : p) : (v[e] < p ? p : v[e]);
         }
@@ -211,286 +243,257 @@ __device__ void block_sort(T* s) {
   __syncthreads();
 }
 
-FP4KV_DEV float4 ld_vals4(const float* p, bool ok) {
-  return ok ? __ldcg(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+// The float whose order key is bin << 20, as a threshold: for finite v (or -inf),
+// order_key(v) >= bin << 20 exactly when v >= thresh(bin). Keys below the key of -inf map to
+// -inf; keys at or above the key of +inf to NaN (no finite value reaches them).
+FP4KV_DEV float thresh(int bin) {
+  if (bin <= 0) return -INFINITY;
+  const uint64_t t = uint64_t(bin) << 20;
+  if (t <= 0x007FFFFFull) return -INFINITY;
+  if (t >= 0xFF800000ull) return __int_as_float(0x7FC00000);
+  return key_to_float(static_cast<uint32_t>(t));
 }
 
-// --------------------------------------------------------------------------------------
-// filter
-// --------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kFThreads) k_select_filter(const SelectArgs args) {
-  // the finishing kernel is a programmatic dependent: it may be scheduled from now on
+__global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args) {
+  // the attention (or the next kernel) may be scheduled from now on
   griddep_launch_dependents();
-  __shared__ __align__(16) uint32_t s_h2[kHistBins];  // digit-2 histogram of this slice
-  __shared__ uint32_t s_w[kFThreads / 32];
-  __shared__ uint32_t s_res[4];
-  __shared__ uint32_t s_sure;
+  extern __shared__ __align__(128) uint8_t sel_raw[];
+  SelSmem& S = *reinterpret_cast<SelSmem*>(sel_raw);
+  float* ring = reinterpret_cast<float*>(sel_raw + kSmemFixed);           // [warp][depth][kChunk]
+  uint64_t* s_pairs = reinterpret_cast<uint64_t*>(sel_raw + kSmemFixed);  // pool pairs (after the filter)
   const SelectProblem& P = args.p[blockIdx.z];
-  const int b = blockIdx.y, s = blockIdx.x;
-  if (s >= P.slices) return;
+  const int D = args.depth;
+  const int b = blockIdx.y;
+  const uint32_t C = cluster_nctas(), r = cluster_ctarank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kHistBins; i += kFThreads) s_h2[i] = 0;
-  if (tid == 0) s_sure = 0;
+
+  for (int i = tid; i < kHistBins; i += kThreads) S.h2[i] = 0;
+  S.h8[tid] = 0;  // (kThreads == 256 bins)
+  if (tid == 0) S.sure = 0;
+  if (lane < D) mbar_init(&S.bar[warp][lane], 1);
+  fence_mbar_init();
+  __syncwarp();
   griddep_wait();  // the scores and the digit-1 histogram are complete past here
 
   const int64_t n = n_values(P, b);
   const uint32_t k = static_cast<uint32_t>(P.k);
   const float* vals = P.values + int64_t(b) * P.vstride;
-  uint64_t* list = P.list + int64_t(b) * P.vstride;
+  uint64_t* glist = P.list + int64_t(b) * P.vstride;
+  uint32_t* hist1 = P.hist + int64_t(b) * kHistBins;
+  // slices in position order, multiples of 128 values (whole 16-byte lane groups)
+  const int64_t per_cta = ((n + C - 1) / C + 127) / 128 * 128;
+  const int64_t lo = min(n, per_cta * r), hi = min(n, lo + per_cta);
+  const int64_t per_w = ((hi - lo + kWarps - 1) / kWarps + 127) / 128 * 128;
+  const int64_t wlo = min(hi, lo + per_w * warp), whi = min(hi, wlo + per_w);
+  const int n_chunks = static_cast<int>((whi - wlo + kChunk - 1) / kChunk);
+  float* wring = ring + size_t(warp) * D * kChunk;
+  // chunk c of the sub-slice into buffer c % D: [c0, c1) rounded up to whole 16-byte units
+  // (at most 3 values past c1, inside the row: vstride is a multiple of 8 and >= n)
+  auto issue = [&](int c) {
+    const int64_t c0 = wlo + int64_t(c) * kChunk, c1 = min(whi, c0 + kChunk);
+    const uint32_t bytes = static_cast<uint32_t>(((c1 - c0 + 3) / 4) * 16);
+    uint64_t* bar = &S.bar[warp][c % D];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s(wring + (c % D) * kChunk, vals + c0, bytes, bar);
+  };
+  if (lane == 0)
+    for (int c = 0; c < D && c < n_chunks; ++c) issue(c);
 
-  // digit 1 of the K-th largest key (b1 = -1: fewer than K values, all are kept)
+  // ---- 1. digit 1 of the K-th largest key (b1 = -1: fewer than K values, all are kept) ----
   int b1;
   {
-    static_assert(kHistBins == kFThreads * 16, "16 bins per thread");
-    const uint32_t* h1 = P.hist + int64_t(b) * kHistBins;
+    static_assert(kHistBins == kThreads * 16, "16 bins per thread");
     const int lo16 = kHistBins - 16 * (tid + 1);
     uint32_t h[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(h1 + lo16 + 4 * (3 - q)));
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(hist1 + lo16 + 4 * (3 - q)));
       h[4 * q] = v.w;
       h[4 * q + 1] = v.z;
       h[4 * q + 2] = v.y;
       h[4 * q + 3] = v.x;
     }
     uint32_t above1, cnt1;
-    block_find_desc<kFThreads, 16>(h, kHistBins, k, &b1, &above1, &cnt1, s_w, s_res);
+    block_find_desc<16>(h, 16, kHistBins, k, &b1, &above1, &cnt1, S.w, S.res);
   }
+  const float f_lo = b1 < 0 ? -INFINITY : thresh(b1);
+  const float f_hi = b1 < 0 ? -INFINITY : thresh(b1 + 1);
 
-  // this warp's sub-slice: keys with digit 1 >= b1, in position order, into list[lo ..)
-  const Region R = region_of(n, P.slices, s, warp);
+  // ---- 2. keep digit 1 >= b1 per warp, in position order; digit-2 histogram of b1 ----
   uint32_t run = 0, sure = 0;
-  float4 cur[kGroups], nxt[kGroups];
-#pragma unroll
-  for (int g = 0; g < kGroups; ++g) {
-    const int64_t i = R.lo + 128 * g + 4 * lane;
-    cur[g] = ld_vals4(vals + i, i < R.hi);
-  }
-  for (int64_t base = R.lo; base < R.hi; base += kWarpBatch) {
-#pragma unroll
-    for (int g = 0; g < kGroups; ++g) {  // the next batch is loaded while this one is kept
-      const int64_t i = base + kWarpBatch + 128 * g + 4 * lane;
-      nxt[g] = ld_vals4(vals + i, i < R.hi);
+  int c_fail = -1;
+#pragma unroll 1
+  for (int c = 0; c < n_chunks; ++c) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_timed(&S.bar[warp][c % D], (c / D) & 1));
+    if (!ok) {
+      c_fail = c;
+      break;
     }
-#pragma unroll
-    for (int g = 0; g < kGroups; ++g) {
-      const int64_t i0 = base + 128 * g + 4 * lane;
-      const float v[4] = {cur[g].x, cur[g].y, cur[g].z, cur[g].w};
-      uint32_t keep = 0, key[4];
+    const float* buf = wring + (c % D) * kChunk;
+    const int64_t base = wlo + int64_t(c) * kChunk;
+    const int n_here = static_cast<int>(min(int64_t(kChunk), whi - base));
+#pragma unroll 2
+    for (int g = 0; g < kChunk / 128; ++g) {
+      if (128 * g >= n_here) break;
+      const int o0 = 128 * g + 4 * lane;
+      const float4 q = *reinterpret_cast<const float4*>(buf + o0);
+      const float v[4] = {q.x, q.y, q.z, q.w};
+      uint32_t keep = 0;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        key[u] = order_key(v[u]);
-        const bool valid = i0 + u < R.hi && (P.mode != 2 || v[u] != -INFINITY);
-        const int d = digit1(key[u]);
-        if (valid && d > b1) {
-          keep |= 1u << u;
-          ++sure;
-        } else if (valid && d == b1) {
-          keep |= 1u << u;
-          atomicAdd(&s_h2[digit2(key[u])], 1u);
-        }
+        const bool in = o0 + u < n_here && v[u] != -INFINITY;  // (-inf: an empty pool slot)
+        keep |= (in && v[u] >= f_lo) ? (1u << u) : 0u;
+        sure += (in && v[u] >= f_hi) ? 1u : 0u;
       }
-      const uint32_t c = __popc(keep);
-      const uint32_t incl = warp_incl_scan(c);
-      if (__any_sync(0xffffffffu, keep != 0)) {
-        // (run + the kept count never exceeds the sub-slice length: the region holds them)
-        uint64_t* dst = list + R.lo + run + (incl - c);
+      if (__ballot_sync(0xffffffffu, keep != 0) == 0u) continue;  // (most groups keep nothing)
+      const uint32_t cnt = __popc(keep);
+      const uint32_t incl = warp_incl_scan(cnt);
+      uint32_t o = run + incl - cnt;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if ((keep >> u) & 1u)
-            *dst++ = (static_cast<uint64_t>(key[u]) << 32) | static_cast<uint32_t>(i0 + u);
+      for (int u = 0; u < 4; ++u) {
+        if (!((keep >> u) & 1u)) continue;
+        const uint32_t key = order_key(v[u]);
+        if (digit1(key) == b1) atomicAdd(&S.h2[digit2(key)], 1u);
+        const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(base + o0 + u);
+        if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
+        else glist[wlo + o] = e;  // (a warp keeps at most its sub-slice: the region holds them)
+        ++o;
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
-#pragma unroll
-    for (int g = 0; g < kGroups; ++g) cur[g] = nxt[g];
+    __syncwarp();  // every lane has read the buffer before lane 0 refills it
+    if (lane == 0 && c + D < n_chunks) {
+      fence_proxy_async_smem();
+      issue(c + D);
+    }
+  }
+  if (c_fail >= 0 && lane == 0) {
+    atomicOr(P.status, kFlagWaitTimeout);
+    // copies still in flight into this warp's ring land (bounded) before the CTA moves on
+    for (int c = c_fail; c < n_chunks && c < c_fail + D; ++c)
+      (void)mbar_wait_timed(&S.bar[warp][c % D], (c / D) & 1);
   }
   sure = __reduce_add_sync(0xffffffffu, sure);
-  uint32_t* ctr = P.counters + int64_t(b) * kSelCounters;
   if (lane == 0) {
-    P.cnt[(int64_t(b) * P.slices + s) * kFWarps + warp] = run;
-    if (sure) atomicAdd(&s_sure, sure);
+    S.wcnt[warp] = run;
+    if (sure) atomicAdd(&S.sure, sure);
   }
   __syncthreads();
-  if (tid == 0) {
-    if (s_sure) atomicAdd(&ctr[0], s_sure);
-    if (s == 0) ctr[1] = static_cast<uint32_t>(b1 + 1);
-  }
-  // merge this slice's digit-2 histogram into the sequence's
-  uint32_t* h2 = P.hist2 + int64_t(b) * kHistBins;
-  for (int i4 = tid; i4 < kHistBins / 4; i4 += kFThreads) {
-    const uint4 c = reinterpret_cast<const uint4*>(s_h2)[i4];
-    if ((c.x | c.y | c.z | c.w) == 0u) continue;
-    if (c.x) atomicAdd(&h2[4 * i4], c.x);
-    if (c.y) atomicAdd(&h2[4 * i4 + 1], c.y);
-    if (c.z) atomicAdd(&h2[4 * i4 + 2], c.z);
-    if (c.w) atomicAdd(&h2[4 * i4 + 3], c.w);
-  }
-}
+  cluster_sync_all();  // (1) digit-2 histograms and sure counts of every CTA are visible
 
-// --------------------------------------------------------------------------------------
-// finish
-// --------------------------------------------------------------------------------------
-struct FinSmem {
-  uint64_t stage[kStage];            // kept entries, regions concatenated in position order
-  uint64_t sel[kMaxSel];             // the pool mode's selected (position, index) pairs
-  uint32_t roff[kNThreads * 4 + 1];  // region offsets in the concatenation
-  uint32_t h8[256];
-  uint32_t w[kNWarps];
-  uint32_t res[4];
-};
-constexpr size_t kFinSmem = sizeof(FinSmem);
-
-// Entry j of the concatenated kept lists: staged, or read straight from its region.
-FP4KV_DEV uint64_t kept_entry(const FinSmem& S, bool staged, const uint64_t* list, int64_t n, int slices,
-                              int n_regions, uint32_t j) {
-  if (staged) return S.stage[j];
-  int lo = 0, hi = n_regions - 1;  // last region with roff <= j
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (S.roff[mid] <= j) lo = mid;
-    else hi = mid - 1;
+  // every CTA has read the digit-1 histogram: clear this CTA's share for the next call
+  {
+    const int seg1 = kHistBins / static_cast<int>(C);
+    for (int i = static_cast<int>(r) * seg1 + tid; i < static_cast<int>(r + 1) * seg1; i += kThreads) hist1[i] = 0;
   }
-  const Region R = region_of(n, slices, lo / kFWarps, lo % kFWarps);
-  return __ldcg(reinterpret_cast<const unsigned long long*>(list) + R.lo + (j - S.roff[lo]));
-}
-
-__global__ void __launch_bounds__(kNThreads) k_select_finish(const SelectArgs args) {
-  // the attention that follows may be scheduled from now on
-  griddep_launch_dependents();
-  griddep_wait();  // the filter grid has completed and its writes are visible
-  extern __shared__ __align__(16) uint8_t fin_raw[];
-  FinSmem& S = *reinterpret_cast<FinSmem*>(fin_raw);
-  const SelectProblem& P = args.p[blockIdx.z];
-  const int b = blockIdx.y;
-  const int tid = threadIdx.x;
-  const int64_t n = n_values(P, b);
-  const uint32_t k = static_cast<uint32_t>(P.k);
-  uint32_t* ctr = P.counters + int64_t(b) * kSelCounters;
-  uint32_t* h1 = P.hist + int64_t(b) * kHistBins;
-  uint32_t* h2 = P.hist2 + int64_t(b) * kHistBins;
-  const uint64_t* list = P.list + int64_t(b) * P.vstride;
-  const int b1 = static_cast<int>(__ldcg(&ctr[1])) - 1;
-  const uint32_t n_sure = __ldcg(&ctr[0]);
   const bool have_b1 = b1 >= 0;
+  const int seg = kHistBins / static_cast<int>(C);
+  if (tid == 0) S.bc[0] = cluster_sum(&S.sure, C);
+  if (have_b1) {  // sum segment r of the digit-2 histograms in place
+    uint32_t tsum = 0;
+    for (int bin = static_cast<int>(r) * seg + tid; bin < static_cast<int>(r + 1) * seg; bin += kThreads) {
+      const uint32_t sv = cluster_sum(&S.h2[bin], C);
+      S.h2[bin] = sv;
+      tsum += sv;
+    }
+    tsum = __reduce_add_sync(0xffffffffu, tsum);
+    if (lane == 0) S.w[warp] = tsum;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = 0;
+      for (int i = 0; i < kWarps; ++i) t += S.w[i];
+      S.seg_total = t;
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // (2) summed segments and their totals are visible
+  const uint32_t n_sure = S.bc[0];
 
-  // ---- digit 2 of the K-th key ----
+  // ---- 3. digit 2 of the K-th key ----
   int b2 = -1;
   uint32_t r3 = 0, cnt_b2 = 0;
-  {
-    static_assert(kHistBins == kNThreads * 4, "4 bins per thread");
-    const int lo4 = kHistBins - 4 * (tid + 1);
-    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(h2 + lo4));
-    const uint32_t h[4] = {v.w, v.z, v.y, v.x};
-    const uint32_t r2 = have_b1 && k > n_sure ? k - n_sure : 1u;
+  if (have_b1) {
+    const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
+    if (tid == 0) {
+      uint32_t cum = 0;
+      int qs = 0;
+      for (int q = static_cast<int>(C) - 1; q >= 0; --q) {
+        const uint32_t t = dsmem_ld(dsmem_map(&S.seg_total, static_cast<uint32_t>(q)));
+        if (cum + t >= r2) {
+          qs = q;
+          break;
+        }
+        cum += t;
+      }
+      S.bc[1] = static_cast<uint32_t>(qs);
+      S.bc[2] = cum;
+    }
+    __syncthreads();
+    const uint32_t qs = S.bc[1], cum = S.bc[2];
+    // the bins of segment qs (summed in CTA qs): thread t owns `per` of them from the top
+    const int per = seg >= kThreads ? seg / kThreads : 1;
+    const int top = static_cast<int>(qs) * seg + seg - per * tid;
+    uint32_t hv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      hv[i] = (i < per && per * tid + i < seg) ? dsmem_ld(dsmem_map(&S.h2[top - 1 - i], qs)) : 0u;
     int d;
     uint32_t above, cnt;
-    block_find_desc<kNThreads, 4>(h, kHistBins, r2, &d, &above, &cnt, S.w, S.res);
-    if (have_b1) {
-      b2 = d;
-      r3 = r2 - above;
-      cnt_b2 = cnt;
-    }
+    block_find_desc<16>(hv, per, seg, r2 - cum, &d, &above, &cnt, S.w, S.res);
+    b2 = static_cast<int>(qs) * seg + d;  // (the segment holds the crossing)
+    r3 = r2 - cum - above;                // keys to take from the (b1, b2) bin
+    cnt_b2 = cnt;
   }
-  // the histograms have been read (the digit-1 one by the whole filter grid): clear them
-  for (int i = tid; i < kHistBins; i += kNThreads) {
-    h1[i] = 0;
-    h2[i] = 0;
-  }
-
-  // ---- region offsets (regions in position order) and staging ----
-  const int n_regions = P.slices * kFWarps;
-  uint32_t total_kept;
-  {
-    uint32_t c[4], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rg = 4 * tid + i;
-      c[i] = rg < n_regions ? __ldcg(P.cnt + int64_t(b) * n_regions + rg) : 0u;
-      sum += c[i];
-    }
-    uint32_t excl = block_excl_scan<kNThreads>(sum, S.w, &total_kept);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rg = 4 * tid + i;
-      if (rg < n_regions) S.roff[rg] = excl;
-      excl += c[i];
-    }
-    if (tid == 0) S.roff[n_regions] = total_kept;
-    __syncthreads();
-  }
-  const bool staged = total_kept <= static_cast<uint32_t>(kStage);
-  if (staged) {
-    // entry j of the concatenation: its region by binary search over the offsets; eight
-    // entries' loads per thread are in flight before any is stored
-    constexpr int kBatch = 8;
-    for (uint32_t jb = tid; jb < total_kept; jb += kNThreads * kBatch) {
-      uint64_t v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const uint32_t j = jb + u * kNThreads;
-        v[u] = 0;
-        if (j < total_kept) {
-          int lo = 0, hi = n_regions - 1;  // last region with roff <= j
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (S.roff[mid] <= j) lo = mid;
-            else hi = mid - 1;
-          }
-          const Region R = region_of(n, P.slices, lo / kFWarps, lo % kFWarps);
-          v[u] = __ldcg(reinterpret_cast<const unsigned long long*>(list) + R.lo + (j - S.roff[lo]));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const uint32_t j = jb + u * kNThreads;
-        if (j < total_kept) S.stage[j] = v[u];
-      }
-    }
-    __syncthreads();
-  }
-  auto entry = [&](uint32_t j) -> uint64_t { return kept_entry(S, staged, list, n, P.slices, n_regions, j); };
-
-  // ---- the (b1, b2) bin, when only r3 of its cnt_b2 keys are taken ----
-  const bool tie = have_b1 && b2 >= 0 && r3 < cnt_b2;
+  const bool tie = have_b1 && r3 < cnt_b2;  // the (b1, b2) bin is taken in part
   const uint32_t pre24 = tie ? (static_cast<uint32_t>(b1) << 12) | static_cast<uint32_t>(b2) : 0u;
+  const uint32_t wcnt = S.wcnt[warp];
+  auto entry = [&](uint32_t j) -> uint64_t {
+    return j < static_cast<uint32_t>(kWarpCap) ? S.list[warp][j]
+                                               : __ldcg(reinterpret_cast<const unsigned long long*>(glist) + wlo + j);
+  };
+
+  // ---- 4. the (b1, b2) bin: the last 8 key bits, then the lowest positions ----
   uint32_t ustar = 0;
   int64_t pos_star = INT64_MAX;
   if (tie) {
-    if (tid < 256) S.h8[tid] = 0;
-    __syncthreads();
-    for (uint32_t j = tid; j < total_kept; j += kNThreads) {
+    for (uint32_t j = lane; j < wcnt; j += 32) {
       const uint32_t key = ent_key(entry(j));
       if ((key >> 8) == pre24) atomicAdd(&S.h8[key & 255u], 1u);
     }
     __syncthreads();
-    uint32_t hv[1] = {tid < 256 ? S.h8[255 - tid] : 0u};
+    cluster_sync_all();  // (3) last-8-bit histograms visible
+    S.hsum[tid] = cluster_sum(&S.h8[tid], C);
+    __syncthreads();
+    uint32_t hv[1] = {S.hsum[255 - tid]};
     int d3;
     uint32_t above3, cnt3;
-    block_find_desc<kNThreads, 1>(hv, 256, r3, &d3, &above3, &cnt3, S.w, S.res);
+    block_find_desc<1>(hv, 1, 256, r3, &d3, &above3, &cnt3, S.w, S.res);
     ustar = (pre24 << 8) | static_cast<uint32_t>(d3);
     uint32_t rr = r3 - above3;  // keys equal to ustar to take, lowest positions first
     if (rr < cnt3) {
-      // 8-bit passes over the 32-bit positions, from the top
       uint64_t pprefix = 0;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        if (tid < 256) S.h8[tid] = 0;
+      for (int pass = 0; pass < 4; ++pass) {  // 8-bit passes over the positions, from the top
+        const int shift = 24 - 8 * pass;
+        uint32_t* hp = S.hp[pass & 1];
+        hp[tid] = 0;
         __syncthreads();
-        for (uint32_t j = tid; j < total_kept; j += kNThreads) {
+        for (uint32_t j = lane; j < wcnt; j += 32) {
           const uint64_t e = entry(j);
           if (ent_key(e) != ustar) continue;
           const uint64_t pos = static_cast<uint64_t>(position_of(P, b, ent_idx(e)));
-          if ((pos >> (shift + 8)) == pprefix) atomicAdd(&S.h8[(pos >> shift) & 255], 1u);
+          if ((pos >> (shift + 8)) == pprefix) atomicAdd(&hp[(pos >> shift) & 255], 1u);
         }
         __syncthreads();
-        // lowest digit first: thread t holds bin t, as the (255 - t)-th bin from the top
-        uint32_t hp[1] = {tid < 256 ? S.h8[tid] : 0u};
+        cluster_sync_all();  // (4 + pass) position-digit histograms visible
+        S.hsum[tid] = cluster_sum(&hp[tid], C);
+        __syncthreads();
+        // lowest digit first: thread t holds bin t as the (255 - t)-th bin from the top
+        uint32_t hq[1] = {S.hsum[tid]};
         int dv;
         uint32_t below, cntd;
-        block_find_desc<kNThreads, 1>(hp, 256, rr, &dv, &below, &cntd, S.w, S.res);
-        const int dd = dv < 0 ? 255 : 255 - dv;
+        block_find_desc<1>(hq, 1, 256, rr, &dv, &below, &cntd, S.w, S.res);
         rr -= below;
-        pprefix = (pprefix << 8) | static_cast<uint64_t>(dd);
+        pprefix = (pprefix << 8) | static_cast<uint64_t>(dv < 0 ? 255 : 255 - dv);
       }
       pos_star = static_cast<int64_t>(pprefix);
     }
@@ -506,88 +509,192 @@ __global__ void __launch_bounds__(kNThreads) k_select_finish(const SelectArgs ar
     return key > ustar || (key == ustar && position_of(P, b, ent_idx(e)) <= pos_star);
   };
 
-  // ---- ordered compaction: thread t owns one contiguous run of the concatenation ----
+  // ---- 5. count, place and write the selection ----
+  // A Reindex pool whose valid blocks are strictly ascending in slot order keeps positions
+  // ascending in slot order: then no sort is needed. Thread t checks slots [16 t, 16 t + 16)
+  // and that its first valid block exceeds every valid block before it.
+  bool in_order = true;
+  if (P.mode == 2) {
+    const int32_t* pl = P.pool + int64_t(b) * P.npb;
+    int32_t mx = -1, first = -1;
+    bool ok = true;
+    for (int i = tid * 16; i < P.npb && i < tid * 16 + 16; ++i) {
+      const int32_t j = pl[i];
+      if (j < 0) continue;
+      if (first < 0) first = j;
+      ok = ok && j > mx;
+      mx = j;
+    }
+    int32_t run_max = mx;  // inclusive running max over the threads of the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, run_max, o);
+      if (lane >= o) run_max = max(run_max, y);
+    }
+    int32_t prev = __shfl_up_sync(0xffffffffu, run_max, 1);
+    if (lane == 0) prev = -1;
+    if (lane == 31) S.w[warp] = static_cast<uint32_t>(run_max + 1);
+    __syncthreads();
+    for (int i = 0; i < warp; ++i) prev = max(prev, static_cast<int32_t>(S.w[i]) - 1);
+    ok = ok && (first < 0 || first > prev);
+    in_order = __syncthreads_and(ok) != 0;
+  }
+  {
+    uint32_t m = 0;
+    for (uint32_t j = lane; j < wcnt; j += 32) m += selected(entry(j)) ? 1u : 0u;
+    m = __reduce_add_sync(0xffffffffu, m);
+    if (lane == 0) S.wsel[warp] = m;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < kWarps; ++w) t += S.wsel[w];
+    S.sel_total = t;
+  }
+  __syncthreads();
+  cluster_sync_all();  // (5) per-CTA selection counts visible
+  if (tid < 32) {
+    uint32_t before = 0, all = 0;
+    if (static_cast<uint32_t>(lane) < C) {
+      const uint32_t c = dsmem_ld(dsmem_map(&S.sel_total, static_cast<uint32_t>(lane)));
+      all = c;
+      before = static_cast<uint32_t>(lane) < r ? c : 0u;
+    }
+    before = __reduce_add_sync(0xffffffffu, before);
+    all = __reduce_add_sync(0xffffffffu, all);
+    if (lane == 0) {
+      S.bc[1] = before;
+      S.bc[2] = all;
+    }
+  }
+  __syncthreads();
+  uint32_t off = S.bc[1];
+  const uint32_t total_sel = S.bc[2];
+  for (int w = 0; w < warp; ++w) off += S.wsel[w];
   int32_t* oi = P.out_idx + int64_t(b) * P.k;
   float* os = P.out_score ? P.out_score + int64_t(b) * P.k : nullptr;
-  const uint32_t per = (total_kept + kNThreads - 1) / kNThreads;
-  const uint32_t j0 = min(total_kept, per * tid), j1 = min(total_kept, j0 + per);
-  uint32_t m_own = 0;
-  for (uint32_t j = j0; j < j1; ++j) m_own += selected(entry(j)) ? 1u : 0u;
-  uint32_t m_all;
-  uint32_t o = block_excl_scan<kNThreads>(m_own, S.w, &m_all);
-  for (uint32_t j = j0; j < j1 && o < k; ++j) {
-    const uint64_t e = entry(j);
-    if (!selected(e)) continue;
-    const int32_t i = ent_idx(e);
-    if (P.mode != 2) {
-      oi[o] = i;
-      if (os) os[o] = key_to_float(ent_key(e));
-    } else {
-      S.sel[o] = (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i);
+  for (uint32_t j0 = 0; j0 < wcnt; j0 += 32) {
+    const uint32_t j = j0 + lane;
+    const uint64_t e = j < wcnt ? entry(j) : 0ull;
+    const bool t = j < wcnt && selected(e);
+    const uint32_t bal = __ballot_sync(0xffffffffu, t);
+    const uint32_t o = off + __popc(bal & ((1u << lane) - 1u));
+    if (t && o < k) {
+      const int32_t i = ent_idx(e);
+      if (in_order) {
+        oi[o] = static_cast<int32_t>(position_of(P, b, i));
+        if (os) os[o] = key_to_float(ent_key(e));
+      } else {  // (position, value index) into CTA 0's pair buffer
+        dsmem_st64(dsmem_map(s_pairs + o, 0),
+                   (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i));
+      }
     }
-    ++o;
+    off += __popc(bal);
   }
-  const uint32_t m = m_all < k ? m_all : k;
-  if (P.mode == 2) {
-    // pool slots: positions need not grow with the value index, sort (position, index)
-    __syncthreads();
-    for (uint32_t i = m + tid; i < static_cast<uint32_t>(kMaxSel); i += kNThreads) S.sel[i] = ~0ull;
-    __syncthreads();
-    block_sort<uint64_t, kMaxSel / kNThreads>(S.sel);
-    const float* vals = P.values + int64_t(b) * P.vstride;
-    for (uint32_t j = tid; j < m; j += kNThreads) {
-      oi[j] = static_cast<int32_t>(S.sel[j] >> 32);
-      if (os) os[j] = vals[static_cast<uint32_t>(S.sel[j] & 0xffffffffu)];
+  const uint32_t m = total_sel < k ? total_sel : k;
+  if (in_order) {
+    for (uint32_t j = m + r * kThreads + tid; j < k; j += C * kThreads) {
+      oi[j] = -1;
+      if (os) os[j] = -INFINITY;
     }
   }
-  for (uint32_t j = m + tid; j < k; j += kNThreads) {
-    oi[j] = -1;
-    if (os) os[j] = -INFINITY;
+  __syncthreads();
+  cluster_sync_all();  // (6) remote reads done, pool pairs delivered: CTAs may leave
+  if (!in_order && r == 0) {
+    for (uint32_t i = m + tid; i < static_cast<uint32_t>(kMaxSel); i += kThreads) s_pairs[i] = ~0ull;
+    __syncthreads();
+    block_sort_pairs(s_pairs);
+    for (uint32_t j = tid; j < k; j += kThreads) {
+      if (j < m) {
+        oi[j] = static_cast<int32_t>(s_pairs[j] >> 32);
+        if (os) os[j] = vals[static_cast<uint32_t>(s_pairs[j] & 0xffffffffu)];
+      } else {
+        oi[j] = -1;
+        if (os) os[j] = -INFINITY;
+      }
+    }
   }
-  if (tid < kSelCounters) ctr[tid] = 0;  // (every thread read them above, before the barriers)
+}
+
+// per device, cluster size 2^i and ring depth: clusters that can be resident at once
+// (0: not asked yet, -1: none)
+int g_sel_clusters[64][5][kMaxDepth + 1] = {};
+
+int sel_max_clusters(int cluster, int depth) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  int li = 0;
+  while ((1 << li) < cluster) ++li;
+  int& known = g_sel_clusters[dev & 63][li][depth];
+  if (known == 0) {
+    known = -1;
+    if (cluster > 8 && cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return known;
+    cudaLaunchConfig_t q = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.gridDim = dim3(cluster, 1, 1);
+    q.blockDim = dim3(kThreads);
+    q.dynamicSmemBytes = select_smem(depth);
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, k_topk_select, &q) == cudaSuccess && nc > 0) known = nc;
+    (void)cudaGetLastError();
+  }
+  return known;
 }
 
 }  // namespace
 
-int select_slices(int64_t n_values, int B, int num_sms) {
-  // about two filter CTAs per SM (what their registers allow) over the whole grid, at least
-  // 4096 values each
-  int64_t s = (2 * int64_t(num_sms)) / B;
-  const int64_t cap = (n_values + 4095) / 4096;
-  if (s > cap) s = cap;
-  if (s > kMaxSlices) s = kMaxSlices;
-  if (s < 1) s = 1;
-  return static_cast<int>(s);
-}
-
-cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, cudaStream_t stream) {
+cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, int num_sms, cudaStream_t stream) {
   if (n_probs < 1 || n_probs > kMaxProblems || B == 0) return cudaSuccess;
   SelectArgs args{};
-  int gx = 1;
+  int64_t n_max = 0;
   for (int i = 0; i < n_probs; ++i) {
     args.p[i] = probs[i];
-    if (probs[i].slices > gx) gx = probs[i].slices;
+    const int64_t nv = probs[i].mode == 2 ? int64_t(probs[i].npb) * 8 : probs[i].vstride;
+    if (nv > n_max) n_max = nv;
   }
-  cudaError_t e = cudaFuncSetAttribute(k_select_finish, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kFinSmem));
+  cudaError_t e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(select_smem(kMaxDepth)));
   if (e != cudaSuccess) return e;
-  // both kernels are programmatic dependents of the kernel before them on the stream
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // CTAs per sequence: a power of two up to 16, at least 4096 values each, the whole grid
+  // within about one CTA per SM, and every cluster resident at once
+  int cluster = 1;
+  while (cluster < kMaxCluster && n_max / (2 * cluster) >= 4096 &&
+         int64_t(B) * n_probs * 2 * cluster <= num_sms)
+    cluster *= 2;
+  auto depth_for = [&](int c) {
+    const int64_t per_warp = (n_max + int64_t(c) * kWarps - 1) / (int64_t(c) * kWarps);
+    const int64_t chunks = (per_warp + kChunk - 1) / kChunk;
+    return static_cast<int>(chunks < 1 ? 1 : (chunks > kMaxDepth ? kMaxDepth : chunks));
+  };
+  while (cluster > 1) {
+    const int nc = sel_max_clusters(cluster, depth_for(cluster));
+    if (nc >= B * n_probs) break;
+    cluster >>= 1;
+  }
+  args.depth = depth_for(cluster);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  // a programmatic dependent of the scoring kernel before it on the stream
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(gx, B, n_probs);
-  cfg.blockDim = dim3(kFThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = dim3(cluster, B, n_probs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = select_smem(args.depth);
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k_select_filter, args);
-  if (e != cudaSuccess) return e;
-  cfg.gridDim = dim3(1, B, n_probs);
-  cfg.blockDim = dim3(kNThreads);
-  cfg.dynamicSmemBytes = kFinSmem;
-  e = cudaLaunchKernelEx(&cfg, k_select_finish, args);
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, k_topk_select, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
