@@ -264,12 +264,6 @@ def traffic_record(kernel: str, workload: str):
     return None
 
 
-def attn_split(fk, B, cap, H, K) -> int:
-    """1 when sparse_attn_decode splits the index list into chunks (a second, combine
-    kernel then runs), else 0; the split needs workspace beyond the 256-byte header."""
-    return 1 if fk.workspace_bytes(fk.OP_SPARSE_ATTN, B, cap, H, K) > 256 else 0
-
-
 class TwoSets:
     """Per-step inputs and outputs in two buffer sets, so that the end-to-end run can copy one
     step's data while another step computes. `in_attrs` / `out_attrs` name the attributes
@@ -399,10 +393,9 @@ class DecodeWorkload(TwoSets):
             self.inputs.append(self.x_swa_new)
             self.in_attrs = self.in_attrs + ("x_swa_new",)
         self.outputs = [self.out, self.lse]
-        # quantize, scan, select, attention (+ the chunk merge when split) (+ the query's FP4
-        # quantize with an FP4 indexer, + the window row's FP8 write)
-        self.launches_per_step = (4 + attn_split(fk, B, cap, H, K) + (1 if self.fp4_idx else 0)
-                                  + (1 if self.n_win else 0))
+        # quantize, scan, select, attention (its chunk CTAs combine in-kernel) (+ the query's
+        # FP4 quantize with an FP4 indexer, + the window row's FP8 write)
+        self.launches_per_step = 4 + (1 if self.fp4_idx else 0) + (1 if self.n_win else 0)
         self.attn_rows_per_step = B * (K + self.n_win)
         self.tokens_per_step = B
 
@@ -477,9 +470,9 @@ class HierWorkload(TwoSets):
         self.inputs = self.q + self.qi + self.w + [self.x_new]
         self.outputs = self.out + self.lse
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
-        # one quantize; the Full layer and each Reindex layer a scan and a select; per layer an
-        # attention (+ merge)
-        self.launches_per_step = 1 + 2 + (L // 2) * 2 + L * (1 + attn_split(fk, B, cap, H, K))
+        # one quantize; the Full layer and each Reindex layer a scan and a select (the Full
+        # layer's pool and position selects share one launch); per layer an attention
+        self.launches_per_step = 1 + 2 + (L // 2) * 2 + L
         self.tokens_per_step = B
 
     def step(self):
@@ -550,8 +543,8 @@ class Csa2DecoderWorkload(TwoSets):
         self.inputs = self.q + self.qi + self.w + [self.x_new]
         self.outputs = self.out + self.lse
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new"), ("out", "lse")
-        # one quantize; a scan and a select per group; an attention (+ merge) per layer
-        self.launches_per_step = 1 + 2 * n_src + L * (1 + attn_split(fk, B, cap, H, K))
+        # one quantize; a scan and a select per group; an attention per layer
+        self.launches_per_step = 1 + 2 * n_src + L
         self.tokens_per_step = B
 
     def step(self):
@@ -631,8 +624,8 @@ class Csa2EncoderWorkload(TwoSets):
         self.outputs = self.out + self.lse
         self.in_attrs, self.out_attrs = ("q", "qi", "w", "x_new", "x_swa_new"), ("out", "lse")
         # per window-only layer a window write and an attention; per group a quantize, a
-        # scan, the two select kernels and G attentions
-        self.launches_per_step = 2 * NS + NG * (4 + G)
+        # scan, a select and G attentions
+        self.launches_per_step = 2 * NS + NG * (3 + G)
         self.attn_rows_per_step = NG * G * B * K + NS * B * nw
         self.tokens_per_step = B
 
@@ -1136,6 +1129,13 @@ def main(argv=None):
                    "algorithmic_bytes_per_step": alg.get(k), "gbs": (alg[k] / (t / args.steps * 1e-3) / 1e9) if k in alg and t > 0 else None}
                for k, (n, t) in prof.items() if n}
 
+    # launches per step as the library recorded them in the profiled pass (the graph replays
+    # the same sequence); the workload's own count is the cross-check
+    recorded = sum(n for n, _ in prof.values()) / args.steps
+    if recorded and abs(recorded - wl.launches_per_step) > 1e-9:
+        print(f"bench: {recorded:g} library launches per step recorded, {wl.launches_per_step} expected",
+              file=sys.stderr)
+    launches = recorded if recorded else wl.launches_per_step
     result = None
     if rank == 0:
         clocks = sampler.summary()
@@ -1155,7 +1155,7 @@ def main(argv=None):
             "roofline": roof,
             "hbm_target": target,
             "kernels": kernels,
-            "gpu_launches": wl.launches_per_step * args.steps,
+            "gpu_launches": int(round(launches * args.steps)),
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks,

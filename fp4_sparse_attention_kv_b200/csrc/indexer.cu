@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
   if (warp == 0) {
     // ------------------------------- TMA producer ----------------------------------
     if (lane == 0) {
+      const uint64_t stream_pol = l2_evict_first();
       uint32_t it = 0, nq = 0;  // tiles issued, query blocks issued
       int cur_b = -1, q_b = -1;
       int64_t len = 0;
@@ -260,17 +261,19 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
         uint8_t* dst = ring + size_t(stage) * Cfg::kStageBytes;
         const int32_t row_base = static_cast<int32_t>(int64_t(ti.b) * p.cap);
         if (!pool_mode) {
+          // a Full scan reads every key once: evict-first keeps the scores it writes (which
+          // the select reads next) in L2 while the keys stream through
           mbar_arrive_expect_tx(&full[stage], Cfg::kKeyBytes + (Cfg::kFp4 ? Cfg::kSfTileBytes : 0));
           const int32_t y = row_base + static_cast<int32_t>(unit);
           if constexpr (Cfg::kFp4) {
             // scale plane viewed as [rows / 2][16 bytes]: y is even (cap even, unit % 128 == 0)
-            tma_load_2d(dst, &tm_keys, 0, y, &full[stage]);
-            tma_load_2d(dst + Cfg::kKeyBytes, &tm_ksf, 0, y >> 1, &full[stage]);
+            tma_load_2d_hint(dst, &tm_keys, 0, y, &full[stage], stream_pol);
+            tma_load_2d_hint(dst + Cfg::kKeyBytes, &tm_ksf, 0, y >> 1, &full[stage], stream_pol);
           } else if constexpr (FP8) {
-            tma_load_2d(dst, &tm_keys, 0, y, &full[stage]);
+            tma_load_2d_hint(dst, &tm_keys, 0, y, &full[stage], stream_pol);
           } else {
-            tma_load_2d(dst, &tm_keys, 0, y, &full[stage]);
-            tma_load_2d(dst + Cfg::kKeyBytes / 2, &tm_keys, 64, y, &full[stage]);
+            tma_load_2d_hint(dst, &tm_keys, 0, y, &full[stage], stream_pol);
+            tma_load_2d_hint(dst + Cfg::kKeyBytes / 2, &tm_keys, 64, y, &full[stage], stream_pol);
           }
         } else {
           const int32_t* pl = p.pool + int64_t(ti.b) * p.npb;

@@ -27,6 +27,8 @@
 // the only synchronisation between CTAs; every mbarrier wait is bounded in time.
 // Kernels that live a few microseconds run mostly from a cold instruction cache, so the loop
 // bodies here are kept short.
+#include <cfloat>
+
 #include "fp4kv_common.cuh"
 #include "fp4kv_launch.h"
 #include "fp4kv_sm100.cuh"
@@ -34,11 +36,11 @@
 namespace fp4kv {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kChunk = 1024;              // values per ring buffer (4 KiB)
-constexpr int kMaxDepth = 4;              // ring buffers per warp
-constexpr int kWarpCap = 512;             // kept entries per warp held in shared memory
+constexpr int kMaxDepth = 2;              // ring buffers per warp
+constexpr int kWarpCap = 256;             // kept entries per warp held in shared memory
 constexpr int kMaxCluster = 16;
 constexpr int kMaxSel = 4096;
 constexpr int kMaxProblems = 2;
@@ -190,8 +192,8 @@ FP4KV_DEV void block_find_desc(const uint32_t (&vals)[kPer], int per, int nbins,
   __syncthreads();
 }
 
-// Block-wide ascending bitonic sort of kMaxSel keys held in shared memory (16 per thread).
-// Strides below 16 are exchanged inside a thread, strides up to 256 through warp shuffles,
+// Block-wide ascending bitonic sort of kMaxSel keys held in shared memory (8 per thread).
+// Strides below 8 are exchanged inside a thread, strides up to 128 through warp shuffles,
 // and only the widest ones through shared memory (one barrier pair each).
 __device__ void block_sort_pairs(uint64_t* s) {
   constexpr int E = kMaxSel / kThreads;
@@ -254,7 +256,7 @@ FP4KV_DEV float thresh(int bin) {
   return key_to_float(static_cast<uint32_t>(t));
 }
 
-__global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args) {
+__global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs args) {
   // the attention (or the next kernel) may be scheduled from now on
   griddep_launch_dependents();
   extern __shared__ __align__(128) uint8_t sel_raw[];
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   for (int i = tid; i < kHistBins; i += kThreads) S.h2[i] = 0;
-  S.h8[tid] = 0;  // (kThreads == 256 bins)
+  if (tid < 256) S.h8[tid] = 0;
   if (tid == 0) S.sure = 0;
   if (lane < D) mbar_init(&S.bar[warp][lane], 1);
   fence_mbar_init();
@@ -302,24 +304,20 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
   // ---- 1. digit 1 of the K-th largest key (b1 = -1: fewer than K values, all are kept) ----
   int b1;
   {
-    static_assert(kHistBins == kThreads * 16, "16 bins per thread");
-    const int lo16 = kHistBins - 16 * (tid + 1);
-    uint32_t h[16];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(hist1 + lo16 + 4 * (3 - q)));
-      h[4 * q] = v.w;
-      h[4 * q + 1] = v.z;
-      h[4 * q + 2] = v.y;
-      h[4 * q + 3] = v.x;
-    }
+    static_assert(kHistBins == kThreads * 8, "8 bins per thread");
+    const int lo8 = kHistBins - 8 * (tid + 1);
+    const uint4 va = __ldcg(reinterpret_cast<const uint4*>(hist1 + lo8));
+    const uint4 vb = __ldcg(reinterpret_cast<const uint4*>(hist1 + lo8 + 4));
+    const uint32_t h[8] = {vb.w, vb.z, vb.y, vb.x, va.w, va.z, va.y, va.x};  // highest bin first
     uint32_t above1, cnt1;
-    block_find_desc<16>(h, 16, kHistBins, k, &b1, &above1, &cnt1, S.w, S.res);
+    block_find_desc<8>(h, 8, kHistBins, k, &b1, &above1, &cnt1, S.w, S.res);
   }
   const float f_lo = b1 < 0 ? -INFINITY : thresh(b1);
   const float f_hi = b1 < 0 ? -INFINITY : thresh(b1 + 1);
 
   // ---- 2. keep digit 1 >= b1 per warp, in position order; digit-2 histogram of b1 ----
+  // v >= f_keep is v >= f_lo without -inf (an empty pool slot) and NaN
+  const float f_keep = f_lo == -INFINITY ? -FLT_MAX : f_lo;
   uint32_t run = 0, sure = 0;
   int c_fail = -1;
 #pragma unroll 1
@@ -332,39 +330,73 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
     const float* buf = wring + (c % D) * kChunk;
     const int64_t base = wlo + int64_t(c) * kChunk;
     const int n_here = static_cast<int>(min(int64_t(kChunk), whi - base));
-#pragma unroll 2
+    // the lane's 32 values of the chunk: group g (128 values), element u at 128 g + 4 lane + u
+    float4 q[kChunk / 128];
+#pragma unroll
+    for (int g = 0; g < kChunk / 128; ++g) q[g] = *reinterpret_cast<const float4*>(buf + 128 * g + 4 * lane);
+    uint32_t mask = 0;  // bit 4 g + u: value (g, u) is kept
+#pragma unroll
     for (int g = 0; g < kChunk / 128; ++g) {
-      if (128 * g >= n_here) break;
-      const int o0 = 128 * g + 4 * lane;
-      const float4 q = *reinterpret_cast<const float4*>(buf + o0);
-      const float v[4] = {q.x, q.y, q.z, q.w};
-      uint32_t keep = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool in = o0 + u < n_here && v[u] != -INFINITY;  // (-inf: an empty pool slot)
-        keep |= (in && v[u] >= f_lo) ? (1u << u) : 0u;
-        sure += (in && v[u] >= f_hi) ? 1u : 0u;
-      }
-      if (__ballot_sync(0xffffffffu, keep != 0) == 0u) continue;  // (most groups keep nothing)
-      const uint32_t cnt = __popc(keep);
-      const uint32_t incl = warp_incl_scan(cnt);
-      uint32_t o = run + incl - cnt;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (!((keep >> u) & 1u)) continue;
-        const uint32_t key = order_key(v[u]);
-        if (digit1(key) == b1) atomicAdd(&S.h2[digit2(key)], 1u);
-        const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(base + o0 + u);
-        if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
-        else glist[wlo + o] = e;  // (a warp keeps at most its sub-slice: the region holds them)
-        ++o;
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
+      mask |= (q[g].x >= f_keep ? 1u : 0u) << (4 * g);
+      mask |= (q[g].y >= f_keep ? 2u : 0u) << (4 * g);
+      mask |= (q[g].z >= f_keep ? 4u : 0u) << (4 * g);
+      mask |= (q[g].w >= f_keep ? 8u : 0u) << (4 * g);
     }
-    __syncwarp();  // every lane has read the buffer before lane 0 refills it
+    if (n_here < kChunk) {  // the sub-slice's last chunk: values past its end are stale
+#pragma unroll
+      for (int g = 0; g < kChunk / 128; ++g)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (128 * g + 4 * lane + u >= n_here) mask &= ~(1u << (4 * g + u));
+    }
+    __syncwarp();  // every lane holds the chunk in registers: lane 0 refills the buffer now
     if (lane == 0 && c + D < n_chunks) {
       fence_proxy_async_smem();
       issue(c + D);
+    }
+    if (__any_sync(0xffffffffu, mask != 0u)) {
+      // per-group kept counts (<= 4) one byte each, groups 0-3 in w0 and 4-7 in w1; an
+      // inclusive scan over the lanes stays below 256 per byte (no carries between bytes)
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        w0 |= static_cast<uint32_t>(__popc((mask >> (4 * g)) & 15u)) << (8 * g);
+        w1 |= static_cast<uint32_t>(__popc((mask >> (16 + 4 * g)) & 15u)) << (8 * g);
+      }
+      uint32_t i0 = w0, i1 = w1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y0 = __shfl_up_sync(0xffffffffu, i0, o), y1 = __shfl_up_sync(0xffffffffu, i1, o);
+        if (lane >= o) {
+          i0 += y0;
+          i1 += y1;
+        }
+      }
+      const uint32_t t0 = __shfl_sync(0xffffffffu, i0, 31), t1 = __shfl_sync(0xffffffffu, i1, 31);
+      const uint32_t e0 = i0 - w0, e1 = i1 - w1;  // exclusive, byte-wise (no borrows)
+      uint32_t goff = run;                        // first list slot of group g
+#pragma unroll
+      for (int g = 0; g < kChunk / 128; ++g) {
+        const int sh = 8 * (g & 3);
+        uint32_t o = goff + (((g < 4 ? e0 : e1) >> sh) & 0xffu);
+        goff += ((g < 4 ? t0 : t1) >> sh) & 0xffu;
+        const uint32_t bits = (mask >> (4 * g)) & 15u;
+        if (bits == 0u) continue;
+        const float v[4] = {q[g].x, q[g].y, q[g].z, q[g].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (!((bits >> u) & 1u)) continue;
+          const uint32_t key = order_key(v[u]);
+          if (digit1(key) == b1) atomicAdd(&S.h2[digit2(key)], 1u);
+          else ++sure;  // (kept keys have digit 1 >= b1)
+          const uint64_t e = (static_cast<uint64_t>(key) << 32) |
+                             static_cast<uint32_t>(base + 128 * g + 4 * lane + u);
+          if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
+          else glist[wlo + o] = e;  // (a warp keeps at most its sub-slice: the region holds them)
+          ++o;
+        }
+      }
+      run = goff;
     }
   }
   if (c_fail >= 0 && lane == 0) {
@@ -414,32 +446,35 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
   uint32_t r3 = 0, cnt_b2 = 0;
   if (have_b1) {
     const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
-    if (tid == 0) {
-      uint32_t cum = 0;
-      int qs = 0;
-      for (int q = static_cast<int>(C) - 1; q >= 0; --q) {
-        const uint32_t t = dsmem_ld(dsmem_map(&S.seg_total, static_cast<uint32_t>(q)));
-        if (cum + t >= r2) {
-          qs = q;
-          break;
-        }
-        cum += t;
+    if (warp == 0) {  // the segment (CTA) holding the r2-th key from the top; keys above it
+      const uint32_t t = static_cast<uint32_t>(lane) < C ? dsmem_ld(dsmem_map(&S.seg_total, static_cast<uint32_t>(lane))) : 0u;
+      uint32_t sfx = t;  // segments lane .. C - 1
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, sfx, o);
+        if (lane + o < 32) sfx += y;
       }
-      S.bc[1] = static_cast<uint32_t>(qs);
-      S.bc[2] = cum;
+      const uint32_t hit = __ballot_sync(0xffffffffu, static_cast<uint32_t>(lane) < C && sfx >= r2);
+      const int qs = hit ? 31 - __clz(static_cast<int>(hit)) : 0;
+      const uint32_t s_q = __shfl_sync(0xffffffffu, sfx, qs), t_q = __shfl_sync(0xffffffffu, t, qs);
+      const uint32_t s_0 = __shfl_sync(0xffffffffu, sfx, 0);
+      if (lane == 0) {
+        S.bc[1] = static_cast<uint32_t>(qs);
+        S.bc[2] = hit ? s_q - t_q : s_0;
+      }
     }
     __syncthreads();
     const uint32_t qs = S.bc[1], cum = S.bc[2];
     // the bins of segment qs (summed in CTA qs): thread t owns `per` of them from the top
     const int per = seg >= kThreads ? seg / kThreads : 1;
     const int top = static_cast<int>(qs) * seg + seg - per * tid;
-    uint32_t hv[16];
+    uint32_t hv[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 8; ++i)
       hv[i] = (i < per && per * tid + i < seg) ? dsmem_ld(dsmem_map(&S.h2[top - 1 - i], qs)) : 0u;
     int d;
     uint32_t above, cnt;
-    block_find_desc<16>(hv, per, seg, r2 - cum, &d, &above, &cnt, S.w, S.res);
+    block_find_desc<8>(hv, per, seg, r2 - cum, &d, &above, &cnt, S.w, S.res);
     b2 = static_cast<int>(qs) * seg + d;  // (the segment holds the crossing)
     r3 = r2 - cum - above;                // keys to take from the (b1, b2) bin
     cnt_b2 = cnt;
@@ -462,9 +497,9 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
     }
     __syncthreads();
     cluster_sync_all();  // (3) last-8-bit histograms visible
-    S.hsum[tid] = cluster_sum(&S.h8[tid], C);
+    if (tid < 256) S.hsum[tid] = cluster_sum(&S.h8[tid], C);
     __syncthreads();
-    uint32_t hv[1] = {S.hsum[255 - tid]};
+    uint32_t hv[1] = {tid < 256 ? S.hsum[255 - tid] : 0u};
     int d3;
     uint32_t above3, cnt3;
     block_find_desc<1>(hv, 1, 256, r3, &d3, &above3, &cnt3, S.w, S.res);
@@ -475,7 +510,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
       for (int pass = 0; pass < 4; ++pass) {  // 8-bit passes over the positions, from the top
         const int shift = 24 - 8 * pass;
         uint32_t* hp = S.hp[pass & 1];
-        hp[tid] = 0;
+        if (tid < 256) hp[tid] = 0;
         __syncthreads();
         for (uint32_t j = lane; j < wcnt; j += 32) {
           const uint64_t e = entry(j);
@@ -485,10 +520,10 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
         }
         __syncthreads();
         cluster_sync_all();  // (4 + pass) position-digit histograms visible
-        S.hsum[tid] = cluster_sum(&hp[tid], C);
+        if (tid < 256) S.hsum[tid] = cluster_sum(&hp[tid], C);
         __syncthreads();
         // lowest digit first: thread t holds bin t as the (255 - t)-th bin from the top
-        uint32_t hq[1] = {S.hsum[tid]};
+        uint32_t hq[1] = {tid < 256 ? S.hsum[tid] : 0u};
         int dv;
         uint32_t below, cntd;
         block_find_desc<1>(hq, 1, 256, rr, &dv, &below, &cntd, S.w, S.res);
@@ -511,14 +546,14 @@ __global__ void __launch_bounds__(kThreads) k_topk_select(const SelectArgs args)
 
   // ---- 5. count, place and write the selection ----
   // A Reindex pool whose valid blocks are strictly ascending in slot order keeps positions
-  // ascending in slot order: then no sort is needed. Thread t checks slots [16 t, 16 t + 16)
-  // and that its first valid block exceeds every valid block before it.
+  // ascending in slot order: then no sort is needed. Thread t checks slots [8 t, 8 t + 8)
+  // and that its first valid block exceeds every valid block before it (8 slots per thread).
   bool in_order = true;
   if (P.mode == 2) {
     const int32_t* pl = P.pool + int64_t(b) * P.npb;
     int32_t mx = -1, first = -1;
     bool ok = true;
-    for (int i = tid * 16; i < P.npb && i < tid * 16 + 16; ++i) {
+    for (int i = tid * 8; i < P.npb && i < tid * 8 + 8; ++i) {
       const int32_t j = pl[i];
       if (j < 0) continue;
       if (first < 0) first = j;
