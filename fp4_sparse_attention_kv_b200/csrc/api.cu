@@ -101,9 +101,9 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Workspace layouts
 // ---------------------------------------------------------------------------------------
 struct IndexerLayout {
-  size_t status = 0, scores = 0, bmax = 0, hist = 0, hist_end = 0, list = 0;
+  size_t status = 0, scores = 0, gmax = 0, bmax = 0, hist = 0, hist_end = 0, list = 0;
   size_t total = 0;
-  int64_t score_stride = 0, bmax_stride = 0;
+  int64_t score_stride = 0, gmax_stride = 0, bmax_stride = 0;
   int n_probs = 0;
   int64_t k[2] = {0, 0};
   int64_t vstride[2] = {0, 0};
@@ -116,6 +116,11 @@ IndexerLayout indexer_layout(int kind, int64_t B, int64_t cap, int64_t top_k, in
   L.score_stride = (kind == 1) ? npb * 8 : (cap + 7) / 8 * 8;
   L.scores = off;
   off += up(sizeof(float) * B * L.score_stride);
+  if (kind != 3) {  // the largest key of every 32 scores
+    L.gmax_stride = ((L.score_stride + 31) / 32 + 7) / 8 * 8;
+    L.gmax = off;
+    off += up(sizeof(uint32_t) * B * L.gmax_stride);
+  }
   if (kind == 2) {
     L.bmax_stride = ((cap + 7) / 8 + 7) / 8 * 8;
     L.bmax = off;
@@ -418,6 +423,8 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
   p.scores = reinterpret_cast<float*>(base + L.scores);
   p.score_stride = L.score_stride;
   p.hist = reinterpret_cast<uint32_t*>(base + L.hist);
+  p.gmax = reinterpret_cast<uint32_t*>(base + L.gmax);
+  p.gmax_stride = L.gmax_stride;
   if (kind == 1) {
     p.pool = pool;
     p.npb = n_pool_blocks;
@@ -446,6 +453,8 @@ static fp4kv_status run_indexer(int kind, const void* q, const float* w, int32_t
     P.pool = pool;
     P.npb = n_pool_blocks;
     P.k = static_cast<int>(L.k[i]);
+    P.gmax = (i == 0) ? p.gmax : nullptr;
+    P.gstride = L.gmax_stride;
     P.hist = p.hist + int64_t(i) * B * fp4kv::kHistBins;
     P.list = reinterpret_cast<uint64_t*>(base + list_off);
     list_off += up(sizeof(uint64_t) * B * L.vstride[i]);

@@ -39,6 +39,10 @@ struct IndexScoreParams {
   float* bmax;              // nullable [B][bmax_stride] (flat mode only)
   int64_t bmax_stride;
   uint32_t* bmax_hist;      // [B][4096] when bmax != nullptr
+  // nullable [B][gmax_stride]: per group of 32 consecutive values (value index / 32) the
+  // largest order key among its valid values (0 when none)
+  uint32_t* gmax;
+  int64_t gmax_stride;
   uint32_t* status;         // workspace status word
 };
 cudaError_t launch_index_score(const IndexScoreParams& p, int num_sms, cudaStream_t stream);
@@ -56,6 +60,8 @@ struct SelectProblem {
   const int32_t* pool;      // mode 2
   int npb;
   int k;
+  const uint32_t* gmax;     // nullable [B][gstride]: largest order key per 32-value group
+  int64_t gstride;          //   (groups below the K-th key's first digit are not read)
   uint32_t* hist;           // [B][4096] digit-1 histogram (from the scoring kernel); the
                             // select reads it and leaves it zeroed
   uint64_t* list;           // [B][vstride] overflow of the kept-entry lists

@@ -519,6 +519,10 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
 
       const int64_t seq_base = int64_t(ti.b) * p.cap;
       float* srow = p.scores + int64_t(ti.b) * p.score_stride;
+      // the largest key of the warp's 32 consecutive values (value index tile * 128 + row
+      // in both modes); 0 when none of them is valid
+      uint32_t* gmax_row = p.gmax != nullptr ? p.gmax + int64_t(ti.b) * p.gmax_stride + ti.tis * (kTileRows / 32) + quarter
+                                             : nullptr;
       if (!pool_mode) {
         const int64_t pos = ti.tis * kTileRows + row;
         const bool valid = pos < len;
@@ -526,6 +530,10 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
           if (p.key_scale != nullptr) s *= p.key_scale[seq_base + pos];
           srow[pos] = s;
           if (p.hist != nullptr) atomicAdd(&s_hist[order_key(s) >> (32 - kHistBits)], 1u);
+        }
+        if (gmax_row != nullptr) {
+          const uint32_t km = __reduce_max_sync(0xffffffffu, valid ? order_key(s) : 0u);
+          if (lane == 0) *gmax_row = km;
         }
         if (p.bmax != nullptr) {
           float m = valid ? s : -INFINITY;
@@ -548,6 +556,10 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
           srow[slot * kPoolBlock + (row % kPoolBlock)] = valid ? s : -INFINITY;
         }
         if (valid && p.hist != nullptr) atomicAdd(&s_hist[order_key(s) >> (32 - kHistBits)], 1u);
+        if (gmax_row != nullptr) {
+          const uint32_t km = __reduce_max_sync(0xffffffffu, valid ? order_key(s) : 0u);
+          if (lane == 0) *gmax_row = km;
+        }
       }
     }
     if (cur_b >= 0 && p.hist != nullptr) flush(cur_b);

@@ -7,15 +7,17 @@
 // 인덱서로 인덱싱 비용을 컨텍스트 길이에서 분리하기": the blocks with the highest block max).
 //
 // Values are mapped to order-preserving 32-bit keys. The scoring kernel has already built a
-// histogram of the top 12 key bits (digit 1) of every sequence. One kernel follows, with one
+// histogram of the top 12 key bits (digit 1) of every sequence and, for the scores, the
+// largest key of every group of 32 consecutive values. One kernel follows, with one
 // thread-block cluster of C CTAs per (problem, sequence); CTA r owns slice r of the values,
 // warp w of it sub-slice w (slices and sub-slices in position order):
-//  1. every CTA finds the digit-1 value b1 of the K-th largest key from the histogram, as two
-//     float thresholds: "digit 1 >= b1" is v >= f_lo, "digit 1 > b1" is v >= f_hi;
-//  2. each warp streams its sub-slice through a ring of shared-memory buffers filled by bulk
-//     asynchronous copies (the copy engine keeps every buffer's bytes in flight), keeps the
-//     values >= f_lo in position order (a warp prefix, no block barrier) in its own list, and
-//     the CTA histograms the next 12 key bits (digit 2) of the keys with digit 1 == b1;
+//  1. every CTA finds the digit-1 value b1 of the K-th largest key from the histogram, as a
+//     float threshold: "digit 1 >= b1" is v >= f_lo;
+//  2. each warp reads only the groups of its sub-slice whose largest key reaches b1 (a few
+//     percent of them for the top 2048 of a million), 16 groups in flight at a time, keeps
+//     the values >= f_lo in position order (a ballot prefix, no block barrier) in its own
+//     list, and the CTA histograms the next 12 key bits (digit 2) of the keys with
+//     digit 1 == b1;
 //  3. the CTAs add up the digit-2 histograms through distributed shared memory (CTA r sums
 //     segment r of the bins in place) and every CTA finds the digit-2 value b2 of the K-th key;
 //  4. only when the (b1, b2) bin is taken in part: the last 8 key bits, then the lowest
@@ -24,7 +26,7 @@
 //     positions at that offset: ascending without a sort. A Reindex pool whose blocks are not
 //     in ascending order gathers its at most 4096 selected pairs in CTA 0, which sorts them.
 // The CTAs also clear the scoring kernel's histogram for the next call. Cluster barriers are
-// the only synchronisation between CTAs; every mbarrier wait is bounded in time.
+// the only synchronisation between CTAs; nothing waits on a flag.
 // Kernels that live a few microseconds run mostly from a cold instruction cache, so the loop
 // bodies here are kept short.
 #include <cfloat>
@@ -38,38 +40,42 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kChunk = 1024;              // values per ring buffer (4 KiB)
-constexpr int kMaxDepth = 2;              // ring buffers per warp
+constexpr int kBatch = 16;                // 32-value groups a warp loads at once
+constexpr int kWords = 8;                 // 32-group words of group maxima loaded at once
+constexpr int kCandCap = 32 * kWords;     // candidate groups a warp lists per round
 constexpr int kWarpCap = 256;             // kept entries per warp held in shared memory
 constexpr int kMaxCluster = 16;
 constexpr int kMaxSel = 4096;
 constexpr int kMaxProblems = 2;
+constexpr int kTieCap = 64;               // a (b1, b2) bin of at most this many keys is ranked directly
 
 struct SelectArgs {
   SelectProblem p[kMaxProblems];
-  int depth;  // ring buffers per warp
 };
 
 struct SelSmem {
+  uint64_t pairs[kMaxSel];              // pool mode: (position, value index), CTA 0 sorts them
   uint32_t h2[kHistBins];               // digit-2 histogram; segment r is summed in place
   uint64_t list[kWarps][kWarpCap];      // kept entries: (order key << 32) | value index
-  uint64_t bar[kWarps][kMaxDepth];      // ring mbarriers
+  uint32_t cand[kWarps][kCandCap];      // candidate groups of a round, in position order
+  uint32_t h2c[64];                     // the same keys' digit 2 / 64 (coarse digit-2 bins)
   uint32_t h8[256];                     // last 8 key bits of the (b1, b2) bin
   uint32_t hp[2][256];                  // position digits among the keys equal to the K-th
   uint32_t hsum[256];                   // a 256-bin histogram summed over the cluster
+  uint64_t tie[kTieCap];                // this CTA's keys of a partly taken (b1, b2) bin: rank values
+  uint64_t tall[kTieCap];               // the whole cluster's, gathered
+  uint32_t tsrc[kTieCap];               // CTA of each gathered one
+  uint32_t tsel[kMaxCluster];           // how many of each CTA's are taken
+  uint32_t tie_n;
   uint32_t wcnt[kWarps];                // kept entries per warp
   uint32_t wsel[kWarps];                // selected entries per warp
   uint32_t w[kWarps];                   // block scans
   uint32_t res[4];
   uint32_t sure;                        // keys of this CTA with digit 1 > b1
-  uint32_t seg_total;                   // sum of this CTA's summed digit-2 segment
   uint32_t sel_total;                   // entries this CTA selects
   uint32_t bc[4];                       // block broadcasts
 };
-// the ring follows; after the filter phase CTA 0 reuses it for the pool mode's sorted pairs
-constexpr size_t kSmemFixed = (sizeof(SelSmem) + 127) / 128 * 128;
-size_t select_smem(int depth) { return kSmemFixed + size_t(kWarps) * depth * kChunk * sizeof(float); }
-static_assert(kWarps * kChunk * sizeof(float) >= kMaxSel * sizeof(uint64_t), "pairs fit a depth-1 ring");
+constexpr size_t kSelSmem = sizeof(SelSmem);
 
 FP4KV_DEV int64_t n_values(const SelectProblem& P, int b) {
   int64_t len = P.seq_lens[b];
@@ -105,6 +111,11 @@ FP4KV_DEV uint32_t dsmem_ld(uint32_t addr) {
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
+FP4KV_DEV uint64_t dsmem_ld64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
 FP4KV_DEV void dsmem_st64(uint32_t addr, uint64_t v) {
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
@@ -120,6 +131,24 @@ FP4KV_DEV uint32_t cluster_sum(const uint32_t* p, uint32_t C) {
   return s;
 }
 
+// the sums over the cluster's CTAs of the u32 at p0 and at p1 (all 2 C loads issued first)
+FP4KV_DEV void cluster_sum2(const uint32_t* p0, const uint32_t* p1, uint32_t C, uint32_t* s0, uint32_t* s1) {
+  uint32_t v0[kMaxCluster], v1[kMaxCluster];
+#pragma unroll
+  for (uint32_t q = 0; q < kMaxCluster; ++q) {
+    v0[q] = q < C ? dsmem_ld(dsmem_map(p0, q)) : 0u;
+    v1[q] = q < C ? dsmem_ld(dsmem_map(p1, q)) : 0u;
+  }
+  uint32_t a = 0, c = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxCluster; ++q) {
+    a += v0[q];
+    c += v1[q];
+  }
+  *s0 = a;
+  *s1 = c;
+}
+
 FP4KV_DEV uint32_t warp_incl_scan(uint32_t x) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -128,6 +157,30 @@ FP4KV_DEV uint32_t warp_incl_scan(uint32_t x) {
     if (lane >= o) x += y;
   }
   return x;
+}
+
+// Warp-wide: lane l holds the counts of bins 2 l and 2 l + 1 counted from the top. Finds the
+// bin (from the top) at which the count from the top reaches r (r >= 1), the count above it
+// and its own count, in every lane; if the total is below r, the lowest bin (63) with the
+// total above it and a count of 0.
+FP4KV_DEV void warp_find_desc2(uint32_t x0, uint32_t x1, uint32_t r, int* pos, uint32_t* above, uint32_t* cnt) {
+  const uint32_t sum = x0 + x1;
+  const uint32_t incl = warp_incl_scan(sum);
+  const uint32_t excl = incl - sum;
+  const uint32_t hit = __ballot_sync(0xffffffffu, excl < r && incl >= r);
+  if (hit == 0u) {
+    *pos = 63;
+    *above = __shfl_sync(0xffffffffu, incl, 31);
+    *cnt = 0;
+    return;
+  }
+  const int l = __ffs(static_cast<int>(hit)) - 1;
+  const uint32_t e = __shfl_sync(0xffffffffu, excl, l), a0 = __shfl_sync(0xffffffffu, x0, l);
+  const uint32_t a1 = __shfl_sync(0xffffffffu, x1, l);
+  const bool first = e + a0 >= r;
+  *pos = 2 * l + (first ? 0 : 1);
+  *above = first ? e : e + a0;
+  *cnt = first ? a0 : a1;
 }
 
 // Block-wide exclusive prefix sum; *total gets the block sum. Every thread calls it.
@@ -261,45 +314,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
   griddep_launch_dependents();
   extern __shared__ __align__(128) uint8_t sel_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(sel_raw);
-  float* ring = reinterpret_cast<float*>(sel_raw + kSmemFixed);           // [warp][depth][kChunk]
-  uint64_t* s_pairs = reinterpret_cast<uint64_t*>(sel_raw + kSmemFixed);  // pool pairs (after the filter)
   const SelectProblem& P = args.p[blockIdx.z];
-  const int D = args.depth;
   const int b = blockIdx.y;
   const uint32_t C = cluster_nctas(), r = cluster_ctarank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   for (int i = tid; i < kHistBins; i += kThreads) S.h2[i] = 0;
   if (tid < 256) S.h8[tid] = 0;
-  if (tid == 0) S.sure = 0;
-  if (lane < D) mbar_init(&S.bar[warp][lane], 1);
-  fence_mbar_init();
-  __syncwarp();
-  griddep_wait();  // the scores and the digit-1 histogram are complete past here
+  if (tid < 64) S.h2c[tid] = 0;
+  if (tid < kMaxCluster) S.tsel[tid] = 0;
+  if (tid == 0) {
+    S.sure = 0;
+    S.tie_n = 0;
+  }
+  griddep_wait();  // the scores, group maxima and digit-1 histogram are complete past here
 
   const int64_t n = n_values(P, b);
   const uint32_t k = static_cast<uint32_t>(P.k);
   const float* vals = P.values + int64_t(b) * P.vstride;
   uint64_t* glist = P.list + int64_t(b) * P.vstride;
   uint32_t* hist1 = P.hist + int64_t(b) * kHistBins;
-  // slices in position order, multiples of 128 values (whole 16-byte lane groups)
+  // slices in position order, multiples of 128 values
   const int64_t per_cta = ((n + C - 1) / C + 127) / 128 * 128;
   const int64_t lo = min(n, per_cta * r), hi = min(n, lo + per_cta);
   const int64_t per_w = ((hi - lo + kWarps - 1) / kWarps + 127) / 128 * 128;
   const int64_t wlo = min(hi, lo + per_w * warp), whi = min(hi, wlo + per_w);
-  const int n_chunks = static_cast<int>((whi - wlo + kChunk - 1) / kChunk);
-  float* wring = ring + size_t(warp) * D * kChunk;
-  // chunk c of the sub-slice into buffer c % D: [c0, c1) rounded up to whole 16-byte units
-  // (at most 3 values past c1, inside the row: vstride is a multiple of 8 and >= n)
-  auto issue = [&](int c) {
-    const int64_t c0 = wlo + int64_t(c) * kChunk, c1 = min(whi, c0 + kChunk);
-    const uint32_t bytes = static_cast<uint32_t>(((c1 - c0 + 3) / 4) * 16);
-    uint64_t* bar = &S.bar[warp][c % D];
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s(wring + (c % D) * kChunk, vals + c0, bytes, bar);
+  // the warp's 32-value groups (wlo is a multiple of 128, so they are the scan's groups)
+  const int64_t n_grp = (whi - wlo + 31) / 32;
+  const uint32_t* gk = P.gmax != nullptr ? P.gmax + int64_t(b) * P.gstride + wlo / 32 : nullptr;
+  // group maxima of groups g0 + 32 j + lane (0xffffffff without maxima: every group is read,
+  // 0 past the sub-slice); the first round's load while the first digit is found
+  uint32_t gkv[kWords];
+  auto load_gmax = [&](int64_t g0) {
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) {
+      const int64_t g = g0 + 32 * j + lane;
+      gkv[j] = g < n_grp ? (gk != nullptr ? __ldcg(gk + g) : 0xffffffffu) : 0u;
+    }
   };
-  if (lane == 0)
-    for (int c = 0; c < D && c < n_chunks; ++c) issue(c);
+  load_gmax(0);
 
   // ---- 1. digit 1 of the K-th largest key (b1 = -1: fewer than K values, all are kept) ----
   int b1;
@@ -313,97 +366,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
     block_find_desc<8>(h, 8, kHistBins, k, &b1, &above1, &cnt1, S.w, S.res);
   }
   const float f_lo = b1 < 0 ? -INFINITY : thresh(b1);
-  const float f_hi = b1 < 0 ? -INFINITY : thresh(b1 + 1);
 
   // ---- 2. keep digit 1 >= b1 per warp, in position order; digit-2 histogram of b1 ----
-  // v >= f_keep is v >= f_lo without -inf (an empty pool slot) and NaN
+  // v >= f_keep is v >= f_lo without -inf (an empty pool slot) and NaN. A group whose largest
+  // key is below f_keep's holds nothing to keep and is not read.
   const float f_keep = f_lo == -INFINITY ? -FLT_MAX : f_lo;
+  const uint32_t k_keep = order_key(f_keep);
+  const uint32_t below = (1u << lane) - 1u;
   uint32_t run = 0, sure = 0;
-  int c_fail = -1;
 #pragma unroll 1
-  for (int c = 0; c < n_chunks; ++c) {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_timed(&S.bar[warp][c % D], (c / D) & 1));
-    if (!ok) {
-      c_fail = c;
-      break;
+  for (int64_t g0 = 0; g0 < n_grp; g0 += kCandCap) {
+    // list the round's candidate groups (all of its maxima are already loading)
+    if (g0 > 0) load_gmax(g0);
+    uint32_t n_cand = 0;
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) {
+      const uint32_t cm = __ballot_sync(0xffffffffu, gkv[j] >= k_keep);  // (0 past the end)
+      if ((cm >> lane) & 1u) S.cand[warp][n_cand + __popc(cm & below)] = static_cast<uint32_t>(g0 + 32 * j + lane);
+      n_cand += __popc(cm);
     }
-    const float* buf = wring + (c % D) * kChunk;
-    const int64_t base = wlo + int64_t(c) * kChunk;
-    const int n_here = static_cast<int>(min(int64_t(kChunk), whi - base));
-    // the lane's 32 values of the chunk: group g (128 values), element u at 128 g + 4 lane + u
-    float4 q[kChunk / 128];
+    __syncwarp();
+    // read them kBatch at a time (lane l: value l of each group), keep in position order
+#pragma unroll 1
+    for (uint32_t c0 = 0; c0 < n_cand; c0 += kBatch) {
+      int64_t gq[kBatch];
+      float v[kBatch];
 #pragma unroll
-    for (int g = 0; g < kChunk / 128; ++g) q[g] = *reinterpret_cast<const float4*>(buf + 128 * g + 4 * lane);
-    uint32_t mask = 0;  // bit 4 g + u: value (g, u) is kept
-#pragma unroll
-    for (int g = 0; g < kChunk / 128; ++g) {
-      mask |= (q[g].x >= f_keep ? 1u : 0u) << (4 * g);
-      mask |= (q[g].y >= f_keep ? 2u : 0u) << (4 * g);
-      mask |= (q[g].z >= f_keep ? 4u : 0u) << (4 * g);
-      mask |= (q[g].w >= f_keep ? 8u : 0u) << (4 * g);
-    }
-    if (n_here < kChunk) {  // the sub-slice's last chunk: values past its end are stale
-#pragma unroll
-      for (int g = 0; g < kChunk / 128; ++g)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (128 * g + 4 * lane + u >= n_here) mask &= ~(1u << (4 * g + u));
-    }
-    __syncwarp();  // every lane holds the chunk in registers: lane 0 refills the buffer now
-    if (lane == 0 && c + D < n_chunks) {
-      fence_proxy_async_smem();
-      issue(c + D);
-    }
-    if (__any_sync(0xffffffffu, mask != 0u)) {
-      // per-group kept counts (<= 4) one byte each, groups 0-3 in w0 and 4-7 in w1; an
-      // inclusive scan over the lanes stays below 256 per byte (no carries between bytes)
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        w0 |= static_cast<uint32_t>(__popc((mask >> (4 * g)) & 15u)) << (8 * g);
-        w1 |= static_cast<uint32_t>(__popc((mask >> (16 + 4 * g)) & 15u)) << (8 * g);
+      for (int q = 0; q < kBatch; ++q) {
+        gq[q] = c0 + q < n_cand ? static_cast<int64_t>(S.cand[warp][c0 + q]) : -1;
+        const int64_t i = wlo + 32 * gq[q] + lane;
+        v[q] = (gq[q] >= 0 && i < whi) ? __ldcg(vals + i) : -INFINITY;
       }
-      uint32_t i0 = w0, i1 = w1;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y0 = __shfl_up_sync(0xffffffffu, i0, o), y1 = __shfl_up_sync(0xffffffffu, i1, o);
-        if (lane >= o) {
-          i0 += y0;
-          i1 += y1;
-        }
-      }
-      const uint32_t t0 = __shfl_sync(0xffffffffu, i0, 31), t1 = __shfl_sync(0xffffffffu, i1, 31);
-      const uint32_t e0 = i0 - w0, e1 = i1 - w1;  // exclusive, byte-wise (no borrows)
-      uint32_t goff = run;                        // first list slot of group g
-#pragma unroll
-      for (int g = 0; g < kChunk / 128; ++g) {
-        const int sh = 8 * (g & 3);
-        uint32_t o = goff + (((g < 4 ? e0 : e1) >> sh) & 0xffu);
-        goff += ((g < 4 ? t0 : t1) >> sh) & 0xffu;
-        const uint32_t bits = (mask >> (4 * g)) & 15u;
-        if (bits == 0u) continue;
-        const float v[4] = {q[g].x, q[g].y, q[g].z, q[g].w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (!((bits >> u) & 1u)) continue;
-          const uint32_t key = order_key(v[u]);
-          if (digit1(key) == b1) atomicAdd(&S.h2[digit2(key)], 1u);
-          else ++sure;  // (kept keys have digit 1 >= b1)
-          const uint64_t e = (static_cast<uint64_t>(key) << 32) |
-                             static_cast<uint32_t>(base + 128 * g + 4 * lane + u);
+      for (int q = 0; q < kBatch; ++q) {
+        if (gq[q] < 0) break;
+        const bool keep = v[q] >= f_keep;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+          const uint32_t key = order_key(v[q]);
+          if (digit1(key) == b1) {
+            atomicAdd(&S.h2[digit2(key)], 1u);
+            atomicAdd(&S.h2c[digit2(key) >> 6], 1u);
+          } else {
+            ++sure;  // (kept keys have digit 1 >= b1)
+          }
+          const uint32_t o = run + __popc(bal & below);
+          const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(wlo + 32 * gq[q] + lane);
           if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
           else glist[wlo + o] = e;  // (a warp keeps at most its sub-slice: the region holds them)
-          ++o;
         }
+        run += __popc(bal);
       }
-      run = goff;
     }
-  }
-  if (c_fail >= 0 && lane == 0) {
-    atomicOr(P.status, kFlagWaitTimeout);
-    // copies still in flight into this warp's ring land (bounded) before the CTA moves on
-    for (int c = c_fail; c < n_chunks && c < c_fail + D; ++c)
-      (void)mbar_wait_timed(&S.bar[warp][c % D], (c / D) & 1);
+    __syncwarp();  // the candidate list is read before the next round rewrites it
   }
   sure = __reduce_add_sync(0xffffffffu, sure);
   if (lane == 0) {
@@ -419,78 +434,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
     for (int i = static_cast<int>(r) * seg1 + tid; i < static_cast<int>(r + 1) * seg1; i += kThreads) hist1[i] = 0;
   }
   const bool have_b1 = b1 >= 0;
-  const int seg = kHistBins / static_cast<int>(C);
-  if (tid == 0) S.bc[0] = cluster_sum(&S.sure, C);
-  if (have_b1) {  // sum segment r of the digit-2 histograms in place
-    uint32_t tsum = 0;
-    for (int bin = static_cast<int>(r) * seg + tid; bin < static_cast<int>(r + 1) * seg; bin += kThreads) {
-      const uint32_t sv = cluster_sum(&S.h2[bin], C);
-      S.h2[bin] = sv;
-      tsum += sv;
-    }
-    tsum = __reduce_add_sync(0xffffffffu, tsum);
-    if (lane == 0) S.w[warp] = tsum;
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t t = 0;
-      for (int i = 0; i < kWarps; ++i) t += S.w[i];
-      S.seg_total = t;
-    }
-  }
-  __syncthreads();
-  cluster_sync_all();  // (2) summed segments and their totals are visible
-  const uint32_t n_sure = S.bc[0];
 
-  // ---- 3. digit 2 of the K-th key ----
+  // ---- 3. digit 2 of the K-th key, from the cluster's digit-2 histogram: its 64 coarse bins
+  // (digit 2 / 64) from the top, then the 64 bins of the coarse bin that holds the crossing.
+  // Warp 0 alone; the histograms are final since barrier (1).
   int b2 = -1;
   uint32_t r3 = 0, cnt_b2 = 0;
   if (have_b1) {
-    const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
-    if (warp == 0) {  // the segment (CTA) holding the r2-th key from the top; keys above it
-      const uint32_t t = static_cast<uint32_t>(lane) < C ? dsmem_ld(dsmem_map(&S.seg_total, static_cast<uint32_t>(lane))) : 0u;
-      uint32_t sfx = t;  // segments lane .. C - 1
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_down_sync(0xffffffffu, sfx, o);
-        if (lane + o < 32) sfx += y;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, static_cast<uint32_t>(lane) < C && sfx >= r2);
-      const int qs = hit ? 31 - __clz(static_cast<int>(hit)) : 0;
-      const uint32_t s_q = __shfl_sync(0xffffffffu, sfx, qs), t_q = __shfl_sync(0xffffffffu, t, qs);
-      const uint32_t s_0 = __shfl_sync(0xffffffffu, sfx, 0);
+    if (warp == 0) {
+      const uint32_t su = static_cast<uint32_t>(lane) < C ? dsmem_ld(dsmem_map(&S.sure, static_cast<uint32_t>(lane))) : 0u;
+      const uint32_t n_sure = __reduce_add_sync(0xffffffffu, su);
+      const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
+      uint32_t x0, x1;
+      cluster_sum2(&S.h2c[63 - 2 * lane], &S.h2c[62 - 2 * lane], C, &x0, &x1);
+      int pc;
+      uint32_t above_c, cnt_c;
+      warp_find_desc2(x0, x1, r2, &pc, &above_c, &cnt_c);
+      const int cb = 63 - pc;
+      cluster_sum2(&S.h2[64 * cb + 63 - 2 * lane], &S.h2[64 * cb + 62 - 2 * lane], C, &x0, &x1);
+      int pf;
+      uint32_t above_f, cnt_f;
+      warp_find_desc2(x0, x1, r2 - above_c, &pf, &above_f, &cnt_f);
       if (lane == 0) {
-        S.bc[1] = static_cast<uint32_t>(qs);
-        S.bc[2] = hit ? s_q - t_q : s_0;
+        S.bc[0] = static_cast<uint32_t>(64 * cb + 63 - pf);
+        S.bc[1] = r2 - above_c - above_f;  // keys to take from the (b1, b2) bin
+        S.bc[2] = cnt_f;
       }
     }
     __syncthreads();
-    const uint32_t qs = S.bc[1], cum = S.bc[2];
-    // the bins of segment qs (summed in CTA qs): thread t owns `per` of them from the top
-    const int per = seg >= kThreads ? seg / kThreads : 1;
-    const int top = static_cast<int>(qs) * seg + seg - per * tid;
-    uint32_t hv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      hv[i] = (i < per && per * tid + i < seg) ? dsmem_ld(dsmem_map(&S.h2[top - 1 - i], qs)) : 0u;
-    int d;
-    uint32_t above, cnt;
-    block_find_desc<8>(hv, per, seg, r2 - cum, &d, &above, &cnt, S.w, S.res);
-    b2 = static_cast<int>(qs) * seg + d;  // (the segment holds the crossing)
-    r3 = r2 - cum - above;                // keys to take from the (b1, b2) bin
-    cnt_b2 = cnt;
+    b2 = static_cast<int>(S.bc[0]);
+    r3 = S.bc[1];
+    cnt_b2 = S.bc[2];
+    __syncthreads();  // (S.bc is reused below)
   }
   const bool tie = have_b1 && r3 < cnt_b2;  // the (b1, b2) bin is taken in part
-  const uint32_t pre24 = tie ? (static_cast<uint32_t>(b1) << 12) | static_cast<uint32_t>(b2) : 0u;
+  // a small such bin is ranked directly, key first and then the lower position; a larger one
+  // (many equal or near-equal keys) by histograms of the last 8 key bits and the positions
+  const bool small_tie = tie && cnt_b2 <= static_cast<uint32_t>(kTieCap);
+  const uint32_t pre24 = have_b1 ? (static_cast<uint32_t>(b1) << 12) | static_cast<uint32_t>(b2) : 0u;
   const uint32_t wcnt = S.wcnt[warp];
   auto entry = [&](uint32_t j) -> uint64_t {
     return j < static_cast<uint32_t>(kWarpCap) ? S.list[warp][j]
                                                : __ldcg(reinterpret_cast<const unsigned long long*>(glist) + wlo + j);
   };
+  // rank value of an entry: larger = taken first (larger key, then lower position)
+  auto rank_value = [&](uint64_t e) -> uint64_t {
+    const uint32_t pos = static_cast<uint32_t>(position_of(P, b, ent_idx(e)));
+    return (static_cast<uint64_t>(ent_key(e)) << 32) | static_cast<uint64_t>(0xffffffffu - pos);
+  };
 
-  // ---- 4. the (b1, b2) bin: the last 8 key bits, then the lowest positions ----
+  // ---- 4. a large partly taken (b1, b2) bin: the last 8 key bits, then the lowest positions ----
   uint32_t ustar = 0;
   int64_t pos_star = INT64_MAX;
-  if (tie) {
+  if (tie && !small_tie) {
     for (uint32_t j = lane; j < wcnt; j += 32) {
       const uint32_t key = ent_key(entry(j));
       if ((key >> 8) == pre24) atomicAdd(&S.h8[key & 255u], 1u);
@@ -533,16 +529,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
       pos_star = static_cast<int64_t>(pprefix);
     }
   }
-  auto selected = [&](uint64_t e) -> bool {
+  // taken for certain (every entry when the bin is not ranked directly)
+  auto certain = [&](uint64_t e) -> bool {
     if (!have_b1) return true;
     const uint32_t key = ent_key(e);
-    const int d1 = digit1(key);
-    if (d1 != b1) return d1 > b1;
-    const int d2 = digit2(key);
-    if (d2 != b2) return d2 > b2;
+    const uint32_t k24 = key >> 8;
+    if (k24 != pre24) return k24 > pre24;
     if (!tie) return true;
+    if (small_tie) return false;
     return key > ustar || (key == ustar && position_of(P, b, ent_idx(e)) <= pos_star);
   };
+  auto in_small_tie = [&](uint64_t e) -> bool { return small_tie && (ent_key(e) >> 8) == pre24; };
 
   // ---- 5. count, place and write the selection ----
   // A Reindex pool whose valid blocks are strictly ascending in slot order keeps positions
@@ -574,9 +571,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
     ok = ok && (first < 0 || first > prev);
     in_order = __syncthreads_and(ok) != 0;
   }
-  {
+  {  // what this CTA takes for certain, and the keys of a small partly taken bin
     uint32_t m = 0;
-    for (uint32_t j = lane; j < wcnt; j += 32) m += selected(entry(j)) ? 1u : 0u;
+    for (uint32_t j = lane; j < wcnt; j += 32) {
+      const uint64_t e = entry(j);
+      m += certain(e) ? 1u : 0u;
+      if (in_small_tie(e)) {
+        const uint32_t slot = atomicAdd(&S.tie_n, 1u);
+        if (slot < static_cast<uint32_t>(kTieCap)) S.tie[slot] = rank_value(e);
+      }
+    }
     m = __reduce_add_sync(0xffffffffu, m);
     if (lane == 0) S.wsel[warp] = m;
   }
@@ -587,22 +591,66 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
     S.sel_total = t;
   }
   __syncthreads();
-  cluster_sync_all();  // (5) per-CTA selection counts visible
-  if (tid < 32) {
-    uint32_t before = 0, all = 0;
-    if (static_cast<uint32_t>(lane) < C) {
-      const uint32_t c = dsmem_ld(dsmem_map(&S.sel_total, static_cast<uint32_t>(lane)));
-      all = c;
-      before = static_cast<uint32_t>(lane) < r ? c : 0u;
+  cluster_sync_all();  // (5) per-CTA certain counts and small-bin keys visible
+  if (warp == 0) {
+    // gather the small bin's keys of every CTA, take its r3 best, and place this CTA after
+    // everything the CTAs before it take
+    const bool q_ok = static_cast<uint32_t>(lane) < C;
+    const uint32_t cq = q_ok ? dsmem_ld(dsmem_map(&S.sel_total, static_cast<uint32_t>(lane))) : 0u;
+    uint32_t nq = 0;
+    if (small_tie && q_ok) nq = min(dsmem_ld(dsmem_map(&S.tie_n, static_cast<uint32_t>(lane))), static_cast<uint32_t>(kTieCap));
+    const uint32_t incl = warp_incl_scan(nq);  // CTA q's keys go to [incl_q - n_q, incl_q)
+    const uint32_t n_all = min(__shfl_sync(0xffffffffu, incl, 31), static_cast<uint32_t>(kTieCap));
+    for (uint32_t i0 = 0; i0 < n_all; i0 += 32) {
+      const uint32_t i = i0 + lane;
+      uint32_t q = 0, qbase = 0;  // the CTA whose range holds i, and where that range starts
+      for (uint32_t qq = 0; qq < C; ++qq) {
+        const uint32_t end_q = __shfl_sync(0xffffffffu, incl, static_cast<int>(qq));
+        if (i >= end_q) {
+          q = qq + 1;
+          qbase = end_q;
+        }
+      }
+      if (i < n_all) {
+        S.tall[i] = dsmem_ld64(dsmem_map(&S.tie[i - qbase], q));
+        S.tsrc[i] = q;
+      }
     }
-    before = __reduce_add_sync(0xffffffffu, before);
-    all = __reduce_add_sync(0xffffffffu, all);
+    __syncwarp();
+    for (uint32_t i = lane; i < n_all; i += 32) {
+      const uint64_t v = S.tall[i];
+      uint32_t better = 0;
+      for (uint32_t j = 0; j < n_all; ++j) better += S.tall[j] > v ? 1u : 0u;
+      if (better < r3) atomicAdd(&S.tsel[S.tsrc[i]], 1u);
+    }
+    __syncwarp();
+    const uint32_t tq = q_ok ? cq + S.tsel[lane] : 0u;
+    const uint32_t before = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(lane) < r ? tq : 0u);
+    const uint32_t all = __reduce_add_sync(0xffffffffu, tq);
     if (lane == 0) {
       S.bc[1] = before;
       S.bc[2] = all;
+      S.bc[3] = n_all;
     }
   }
   __syncthreads();
+  const uint32_t n_tie_all = S.bc[3];
+  auto selected = [&](uint64_t e) -> bool {
+    if (certain(e)) return true;
+    if (!in_small_tie(e)) return false;
+    const uint64_t v = rank_value(e);
+    uint32_t better = 0;
+    for (uint32_t j = 0; j < n_tie_all; ++j) better += S.tall[j] > v ? 1u : 0u;
+    return better < r3;
+  };
+  if (small_tie) {  // per-warp counts with the small bin's keys that are taken
+    uint32_t m = 0;
+    for (uint32_t j = lane; j < wcnt; j += 32) m += selected(entry(j)) ? 1u : 0u;
+    m = __reduce_add_sync(0xffffffffu, m);
+    __syncthreads();
+    if (lane == 0) S.wsel[warp] = m;
+    __syncthreads();
+  }
   uint32_t off = S.bc[1];
   const uint32_t total_sel = S.bc[2];
   for (int w = 0; w < warp; ++w) off += S.wsel[w];
@@ -620,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
         oi[o] = static_cast<int32_t>(position_of(P, b, i));
         if (os) os[o] = key_to_float(ent_key(e));
       } else {  // (position, value index) into CTA 0's pair buffer
-        dsmem_st64(dsmem_map(s_pairs + o, 0),
+        dsmem_st64(dsmem_map(S.pairs + o, 0),
                    (static_cast<uint64_t>(position_of(P, b, i)) << 32) | static_cast<uint32_t>(i));
       }
     }
@@ -636,13 +684,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
   __syncthreads();
   cluster_sync_all();  // (6) remote reads done, pool pairs delivered: CTAs may leave
   if (!in_order && r == 0) {
-    for (uint32_t i = m + tid; i < static_cast<uint32_t>(kMaxSel); i += kThreads) s_pairs[i] = ~0ull;
+    for (uint32_t i = m + tid; i < static_cast<uint32_t>(kMaxSel); i += kThreads) S.pairs[i] = ~0ull;
     __syncthreads();
-    block_sort_pairs(s_pairs);
+    block_sort_pairs(S.pairs);
     for (uint32_t j = tid; j < k; j += kThreads) {
       if (j < m) {
-        oi[j] = static_cast<int32_t>(s_pairs[j] >> 32);
-        if (os) os[j] = vals[static_cast<uint32_t>(s_pairs[j] & 0xffffffffu)];
+        oi[j] = static_cast<int32_t>(S.pairs[j] >> 32);
+        if (os) os[j] = vals[static_cast<uint32_t>(S.pairs[j] & 0xffffffffu)];
       } else {
         oi[j] = -1;
         if (os) os[j] = -INFINITY;
@@ -651,16 +699,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
   }
 }
 
-// per device, cluster size 2^i and ring depth: clusters that can be resident at once
-// (0: not asked yet, -1: none)
-int g_sel_clusters[64][5][kMaxDepth + 1] = {};
+// per device and cluster size 2^i: clusters that can be resident at once (0: not asked
+// yet, -1: none)
+int g_sel_clusters[64][5] = {};
 
-int sel_max_clusters(int cluster, int depth) {
+int sel_max_clusters(int cluster) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   int li = 0;
   while ((1 << li) < cluster) ++li;
-  int& known = g_sel_clusters[dev & 63][li][depth];
+  int& known = g_sel_clusters[dev & 63][li];
   if (known == 0) {
     known = -1;
     if (cluster > 8 && cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
@@ -673,7 +721,7 @@ int sel_max_clusters(int cluster, int depth) {
     qa[0].val.clusterDim.z = 1;
     q.gridDim = dim3(cluster, 1, 1);
     q.blockDim = dim3(kThreads);
-    q.dynamicSmemBytes = select_smem(depth);
+    q.dynamicSmemBytes = kSelSmem;
     q.attrs = qa;
     q.numAttrs = 1;
     int nc = 0;
@@ -695,7 +743,7 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, i
     if (nv > n_max) n_max = nv;
   }
   cudaError_t e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(select_smem(kMaxDepth)));
+                                       static_cast<int>(kSelSmem));
   if (e != cudaSuccess) return e;
   // CTAs per sequence: a power of two up to 16, at least 4096 values each, the whole grid
   // within about one CTA per SM, and every cluster resident at once
@@ -703,17 +751,11 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, i
   while (cluster < kMaxCluster && n_max / (2 * cluster) >= 4096 &&
          int64_t(B) * n_probs * 2 * cluster <= num_sms)
     cluster *= 2;
-  auto depth_for = [&](int c) {
-    const int64_t per_warp = (n_max + int64_t(c) * kWarps - 1) / (int64_t(c) * kWarps);
-    const int64_t chunks = (per_warp + kChunk - 1) / kChunk;
-    return static_cast<int>(chunks < 1 ? 1 : (chunks > kMaxDepth ? kMaxDepth : chunks));
-  };
   while (cluster > 1) {
-    const int nc = sel_max_clusters(cluster, depth_for(cluster));
+    const int nc = sel_max_clusters(cluster);
     if (nc >= B * n_probs) break;
     cluster >>= 1;
   }
-  args.depth = depth_for(cluster);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
@@ -725,7 +767,7 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, i
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cluster, B, n_probs);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = select_smem(args.depth);
+  cfg.dynamicSmemBytes = kSelSmem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
