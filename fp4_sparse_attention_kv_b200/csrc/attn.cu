@@ -311,11 +311,12 @@ FP4KV_DEV bool load_dequant_win(uint8_t* smem, uint64_t* bars, const uint8_t* wi
 }
 
 // CTA `rank` of a cluster of C chunk CTAs: sums 16-byte units (head, 4 dims) of its dim slice
-// [rank * 512 / C, +512 / C) over the C chunk partials with the per-(chunk, head) weights sW
-// and writes them. Each thread keeps 16 loads in flight: 16 / C units over the C chunks.
+// [rank * 512 / C, +512 / C) over the C chunk partials with the log-sum-exp weights
+// 2^(m_c - M) / (2^6 L) (O holds p * 2^6) and writes them; CTA 0 also writes the lse. Each
+// thread loads its units' partials and their heads' (m, l) of every chunk at once (one L2
+// round trip) and forms the weights itself: 16 / C units per thread and batch.
 template <int C>
-FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint32_t rank, int64_t part0,
-                             const float* sW) {
+FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint32_t rank, int64_t part0) {
   constexpr int kSlice4 = kD / 4 / C;  // 16-byte units per head in the slice
   constexpr int kPer = 16 / C;         // units per thread and batch
   const int tid = threadIdx.x;
@@ -323,27 +324,43 @@ FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint
   const int d0 = static_cast<int>(rank) * kSlice4 * 4;
   const bool al16 = (reinterpret_cast<uintptr_t>(p.out) & 15u) == 0;
   const float4* part4 = reinterpret_cast<const float4*>(p.part_o + part0 * (kHeadsPerCta * kD));
+  const float2* ml2 = reinterpret_cast<const float2*>(p.part_ml + part0 * kHeadsPerCta * 2);
   for (int u0 = tid; u0 < n_units; u0 += kAttnThreads * kPer) {
     float4 v[kPer][C];
+    float2 ml[kPer][C];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int u = u0 + j * kAttnThreads;
       const int h = u / kSlice4, d = d0 + 4 * (u % kSlice4);
 #pragma unroll
-      for (int c = 0; c < C; ++c)
+      for (int c = 0; c < C; ++c) {
         v[j][c] = u < n_units ? __ldcg(part4 + (int64_t(c) * kHeadsPerCta * kD + h * kD + d) / 4)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        ml[j][c] = u < n_units ? __ldcg(ml2 + c * kHeadsPerCta + h) : make_float2(0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int u = u0 + j * kAttnThreads;
       if (u >= n_units) continue;
       const int h = u / kSlice4, d = d0 + 4 * (u % kSlice4);
+      float M = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < C; ++c)
+        if (ml[j][c].y > 0.0f) M = fmaxf(M, ml[j][c].x);
+      float Lt = 0.0f;
+      float w[C];
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        w[c] = ml[j][c].y > 0.0f ? exp2f(ml[j][c].x - M) : 0.0f;
+        Lt += w[c] * ml[j][c].y;
+      }
+      const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < C; ++c) {
-        const float w = sW[c * kHeadsPerCta + h];
-        acc.x += w * v[j][c].x; acc.y += w * v[j][c].y; acc.z += w * v[j][c].z; acc.w += w * v[j][c].w;
+        const float wc = w[c] * inv;
+        acc.x += wc * v[j][c].x; acc.y += wc * v[j][c].y; acc.z += wc * v[j][c].z; acc.w += wc * v[j][c].w;
       }
       float* dst = p.out + (int64_t(b) * p.H + hbase + h) * kD + d;
       if (al16) {
@@ -352,6 +369,8 @@ FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint
         reinterpret_cast<float2*>(dst)[0] = make_float2(acc.x, acc.y);
         reinterpret_cast<float2*>(dst)[1] = make_float2(acc.z, acc.w);
       }
+      if (rank == 0 && d == 0 && p.lse != nullptr)
+        p.lse[int64_t(b) * p.H + hbase + h] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
     }
   }
 }
@@ -788,42 +807,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     }
   }
   cluster_sync_all();  // every chunk CTA's partial is in the workspace and visible
-  float* sW = reinterpret_cast<float*>(smem + kOffV);  // [C][64] weights (V_hat is free now)
-  if (tid < kHeadsPerCta) {
-    const int h = tid;
-    float mc[kMaxCluster], lc[kMaxCluster];
-#pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c) {  // (all loads first, then their use)
-      mc[c] = -INFINITY;
-      lc[c] = 0.0f;
-      if (c < static_cast<int>(C)) {
-        const float* pml = p.part_ml + ((part0 + c) * kHeadsPerCta + h) * 2;
-        mc[c] = __ldcg(pml);
-        lc[c] = __ldcg(pml + 1);
-      }
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c)
-      if (lc[c] > 0.0f) M = fmaxf(M, mc[c]);
-    float Lt = 0.0f;
-#pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c)
-      if (lc[c] > 0.0f) Lt += exp2f(mc[c] - M) * lc[c];
-    const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
-#pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c)
-      if (c < static_cast<int>(C)) sW[c * kHeadsPerCta + h] = lc[c] > 0.0f ? exp2f(mc[c] - M) * inv : 0.0f;
-    if (rank == 0 && p.lse != nullptr && h < nh)
-      p.lse[int64_t(b) * p.H + hbase + h] = Lt > 0.0f ? M * kLn2 + logf(Lt) : -INFINITY;
-  }
-  __syncthreads();
   switch (C) {  // (only the instance that runs is ever fetched)
-    case 1: combine_slice<1>(p, b, hbase, nh, rank, part0, sW); break;
-    case 2: combine_slice<2>(p, b, hbase, nh, rank, part0, sW); break;
-    case 4: combine_slice<4>(p, b, hbase, nh, rank, part0, sW); break;
-    case 8: combine_slice<8>(p, b, hbase, nh, rank, part0, sW); break;
-    default: combine_slice<16>(p, b, hbase, nh, rank, part0, sW); break;
+    case 1: combine_slice<1>(p, b, hbase, nh, rank, part0); break;
+    case 2: combine_slice<2>(p, b, hbase, nh, rank, part0); break;
+    case 4: combine_slice<4>(p, b, hbase, nh, rank, part0); break;
+    case 8: combine_slice<8>(p, b, hbase, nh, rank, part0); break;
+    default: combine_slice<16>(p, b, hbase, nh, rank, part0); break;
   }
 
   tc_fence_before();
