@@ -49,8 +49,9 @@ FP4KV_DEV uint32_t f32_to_e4m3_satfinite(float x) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
   return r & 0xffu;
 }
-// Two non-negative fp32 -> one byte of E2M1 codes, round-to-nearest-even, saturating at
-// 6. `lo` lands in bits 0..3, `hi` in bits 4..7.
+// Two fp32 -> one byte of E2M1 codes, round-to-nearest-even, saturating at +-6 (the sign
+// in bits 3 and 7: -0 and negative values that round to zero give 0x8). `lo` lands in
+// bits 0..3, `hi` in bits 4..7.
 FP4KV_DEV uint32_t f32x2_to_e2m1x2_satfinite(float lo, float hi) {
   uint32_t r;
   asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}"

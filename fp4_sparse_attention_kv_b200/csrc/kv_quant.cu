@@ -12,14 +12,14 @@
 //    is either an E4M3 rounding midpoint itself (then the division is exact) or lies at a
 //    relative distance >= 2^-14.5 from every midpoint, far beyond the 2^-24 error of the
 //    division; the hardware cvt then rounds to nearest-even and saturates at 448.
-//  * |x| / S is formed as |x| * RN(1/S) (two roundings, relative error < 2^-23) and then
-//    snapped to a multiple of 2^-16 by adding and subtracting 128. For r < 8 an exact tie
-//    r = t (t a multiple of 1/4) is recovered exactly, while a non-tie bf16/E4M3 ratio is at
-//    least 2^-10 away from every E2M1 midpoint, so the snap cannot move it across one.
-//    Ratios >= 8 saturate either way.
-//  * cvt.rn.satfinite.e2m1x2.f32 rounds to nearest-even on the code and saturates at 6.
-//  * The sign bit of x is OR-ed in separately, so -0 and negative values rounding to zero
-//    keep the sign (code 0x8).
+//  * |x| / S is formed as |x| * RN(1/S) + 128 in one fused multiply-add (so the product is
+//    rounded once, to a multiple of 2^-16), minus 128. RN(1/S) is within 2^-24 relative of
+//    1/S, so for r < 8 an exact tie r = t (t a multiple of 1/4) is within 2^-21 of t and
+//    snaps to it exactly, while a non-tie bf16/E4M3 ratio is at least 2^-10 away from every
+//    E2M1 midpoint, so the snap cannot move it across one. Ratios >= 8 saturate either way.
+//  * cvt.rn.satfinite.e2m1x2.f32 rounds to nearest-even on the code and saturates at 6; it
+//    gets the ratio with x's sign bit put back, and rounding is symmetric, so the code is
+//    sign | RNE(|x| / S): -0 and negative values rounding to zero give 0x8.
 // Memory: at d = 512 (with 16-byte aligned codes) half a warp per row, two groups per lane,
 // four rows' loads in flight per warp; otherwise one warp per row, one 16-channel group per
 // lane (32 B read, 8 B + 1 B written per lane).
@@ -31,19 +31,19 @@ namespace fp4kv {
 
 namespace {
 
-FP4KV_DEV float snap_ratio(float r) {
-  return __fadd_rn(__fadd_rn(r, 128.0f), -128.0f);
+// RN(a * inv + 128) - 128: the ratio a * inv rounded once to a multiple of 2^-16 (for
+// a * inv < 128; larger ratios saturate the code either way)
+FP4KV_DEV float snap_ratio(float a, float inv) {
+  return __fadd_rn(__fmaf_rn(a, inv, 128.0f), -128.0f);
 }
 
 // Quantize one group of 16 bf16 values held as 8 words (2 values per word, low half first).
 // Returns the 8 packed bytes (low nibble = even channel) and the scale code.
 FP4KV_DEV void quant_group(const uint32_t (&w)[8], uint2& packed, uint32_t& scale_code) {
-  uint32_t m = 0;
+  uint32_t m2 = 0;  // per-half maxima of the 15-bit magnitudes
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    m = max(m, w[i] & 0x7fffu);
-    m = max(m, (w[i] >> 16) & 0x7fffu);
-  }
+  for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, w[i] & 0x7fff7fffu);
+  const uint32_t m = max(m2 & 0xffffu, m2 >> 16);
   const float amax = bf16_bits_to_f32(m);
   const uint32_t sc = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
   const float S = f16_lo_to_f32(e4m3x2_to_f16x2(static_cast<uint16_t>(sc)));
@@ -52,20 +52,17 @@ FP4KV_DEV void quant_group(const uint32_t (&w)[8], uint2& packed, uint32_t& scal
     const float inv = __frcp_rn(S);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float a0 = bf16_bits_to_f32(w[i] & 0x7fffu);
-      const float a1 = bf16_bits_to_f32((w[i] >> 16) & 0x7fffu);
-      const float r0 = snap_ratio(__fmul_rn(a0, inv));
-      const float r1 = snap_ratio(__fmul_rn(a1, inv));
-      bytes[i] = f32x2_to_e2m1x2_satfinite(r0, r1);
+      const uint32_t e = w[i] << 16, o = w[i] & 0xffff0000u;  // the two channels as f32 bits
+      const float r0 = snap_ratio(__uint_as_float(e & 0x7fffffffu), inv);
+      const float r1 = snap_ratio(__uint_as_float(o & 0x7fffffffu), inv);
+      // the sign goes back on before the rounding to E2M1, which is symmetric; a negative
+      // value that rounds to zero keeps its sign (code 0x8)
+      bytes[i] = f32x2_to_e2m1x2_satfinite(__uint_as_float(__float_as_uint(r0) | (e & 0x80000000u)),
+                                           __uint_as_float(__float_as_uint(r1) | (o & 0x80000000u)));
     }
-  } else {
+  } else {  // an all-zero group: sign-only codes
 #pragma unroll
-    for (int i = 0; i < 8; ++i) bytes[i] = 0;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    // sign of the even channel (bit 15) -> bit 3; odd channel (bit 31) -> bit 7
-    bytes[i] |= ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);
+    for (int i = 0; i < 8; ++i) bytes[i] = ((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u);
   }
   packed.x = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
   packed.y = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
