@@ -749,10 +749,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
                                                    : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, t + 1));
       }
     }
-    // ---- wait for the last P.V and reduce the row sums over the CTA ----
-    if (!fail && n_tiles > 0) {
-      const bool f = !softmax_wait(&bars[B_PFREE], (n_tiles - 1) & 1);
-      fail = softmax_any(f);
+    // ---- the partial O^T leaves for the workspace one dim tile at a time, as soon as the
+    // last tile's P.V has finished that dim tile (fp32, unscaled, [64 heads][512 dims]) ----
+    {
+      const int64_t part0 = (int64_t(b) * gridDim.y + hg) * cluster_nctas();
+      float* po = p.part_o + (part0 + cluster_ctarank()) * (kHeadsPerCta * kD);
+      bool f_part = false;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        bool have = !fail && !f_part && n_tiles > 0;
+        if (have && !softmax_wait(&bars[B_VFREE + 2 * c], (n_tiles - 1) & 1)) {
+          f_part = true;  // (this CTA's partial is dropped below)
+          have = false;
+        }
+        if (have) {
+          tc_fence_after();
+          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) r[k] = 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < 32; ++k) __stcg(po + (h0 + k) * kD + 128 * c + e, __uint_as_float(r[k]));
+      }
+      // ---- wait for the last P.V and reduce the row sums over the CTA ----
+      if (!fail && n_tiles > 0) {
+        const bool f = f_part || !softmax_wait(&bars[B_PFREE], (n_tiles - 1) & 1);
+        fail = softmax_any(f);
+      }
     }
     if (fail) {
       if (tid == 0) fail_wait(p, s_abort);
@@ -771,34 +797,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   }
 
   // ---- combine the chunk CTAs of this (sequence, head group): one cluster ----
-  // Each CTA writes its partial -- O^T as [64 heads][512 dims] fp32, unscaled, straight from
-  // TMEM, and (m, l) per head -- to the workspace (it stays in L2). One cluster barrier
-  // makes every chunk's partial visible to the others; then CTA `rank` sums dims
-  // [rank * 512 / C, +512 / C) of every head over the chunks with the log-sum-exp weights
-  // 2^(m_c - M) / (2^6 L) (O holds p * 2^6) and writes them.
+  // Each CTA has written its partial O^T to the workspace (it stays in L2); now (m, l) per
+  // head (l = 0: the partial is void). One cluster barrier makes every chunk's partial
+  // visible to the others; then CTA `rank` sums dims [rank * 512 / C, +512 / C) of every
+  // head over the chunks with the log-sum-exp weights 2^(m_c - M) / (2^6 L) (O holds
+  // p * 2^6) and writes them.
   __syncthreads();
   const uint32_t C = cluster_nctas(), rank = cluster_ctarank();
   const int64_t part0 = (int64_t(b) * gridDim.y + hg) * C;  // this (sequence, head group)'s first chunk
   {
-    float* po = p.part_o + (part0 + rank) * (kHeadsPerCta * kD);
-    if (warp < kSoftWarps) {
-      const int q4 = warp & 3, h0 = 32 * (warp >> 2), e = 32 * q4 + lane;
-      const uint32_t lane_addr = uint32_t(32 * q4) << 16;
-      const bool have = n_tiles > 0 && *s_fail == 0u;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        if (have) {
-          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = 0u;
-        }
-#pragma unroll
-        for (int k = 0; k < 32; ++k) __stcg(po + (h0 + k) * kD + 128 * c + e, __uint_as_float(r[k]));
-      }
-    }
     if (tid < kHeadsPerCta) {
       const float l = sL[tid];
       float* pml = p.part_ml + ((part0 + rank) * kHeadsPerCta + tid) * 2;
