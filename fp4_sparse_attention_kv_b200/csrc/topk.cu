@@ -633,6 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
       S.bc[3] = n_all;
     }
   }
+  // (6) this CTA has read everything it needs from the others: arrive now, wait only before
+  // leaving, so that the barrier's latency hides behind the writes below. When the pool
+  // mode's pairs go to CTA 0, arrive after they are delivered instead.
+  if (in_order) cluster_arrive();
   __syncthreads();
   const uint32_t n_tie_all = S.bc[3];
   auto selected = [&](uint64_t e) -> bool {
@@ -681,8 +685,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
       if (os) os[j] = -INFINITY;
     }
   }
-  __syncthreads();
-  cluster_sync_all();  // (6) remote reads done, pool pairs delivered: CTAs may leave
+  if (!in_order) {
+    __syncthreads();
+    cluster_arrive();
+  }
+  cluster_wait();  // (6) remote reads done, pool pairs delivered: CTAs may leave
   if (!in_order && r == 0) {
     for (uint32_t i = m + tid; i < static_cast<uint32_t>(kMaxSel); i += kThreads) S.pairs[i] = ~0ull;
     __syncthreads();
