@@ -40,7 +40,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 16;                // 32-value groups a warp loads at once
+constexpr int kBatch = 24;                // 32-value groups a warp loads at once
 constexpr int kWords = 8;                 // 32-group words of group maxima loaded at once
 constexpr int kCandCap = 32 * kWords;     // candidate groups a warp lists per round
 constexpr int kWarpCap = 256;             // kept entries per warp held in shared memory
@@ -389,12 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
     // read them kBatch at a time (lane l: value l of each group), keep in position order
 #pragma unroll 1
     for (uint32_t c0 = 0; c0 < n_cand; c0 += kBatch) {
-      int64_t gq[kBatch];
+      int32_t gq[kBatch];  // group within the sub-slice (-1: none)
       float v[kBatch];
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
-        gq[q] = c0 + q < n_cand ? static_cast<int64_t>(S.cand[warp][c0 + q]) : -1;
-        const int64_t i = wlo + 32 * gq[q] + lane;
+        gq[q] = c0 + q < n_cand ? static_cast<int32_t>(S.cand[warp][c0 + q]) : -1;
+        const int64_t i = wlo + 32 * int64_t(gq[q]) + lane;
         v[q] = (gq[q] >= 0 && i < whi) ? __ldcg(vals + i) : -INFINITY;
       }
 #pragma unroll
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
             ++sure;  // (kept keys have digit 1 >= b1)
           }
           const uint32_t o = run + __popc(bal & below);
-          const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(wlo + 32 * gq[q] + lane);
+          const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(wlo + 32 * int64_t(gq[q]) + lane);
           if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
           else glist[wlo + o] = e;  // (a warp keeps at most its sub-slice: the region holds them)
         }
@@ -442,11 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
   uint32_t r3 = 0, cnt_b2 = 0;
   if (have_b1) {
     if (warp == 0) {
+      // (the counts above b1 and the coarse bins load in one round trip)
       const uint32_t su = static_cast<uint32_t>(lane) < C ? dsmem_ld(dsmem_map(&S.sure, static_cast<uint32_t>(lane))) : 0u;
-      const uint32_t n_sure = __reduce_add_sync(0xffffffffu, su);
-      const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
       uint32_t x0, x1;
       cluster_sum2(&S.h2c[63 - 2 * lane], &S.h2c[62 - 2 * lane], C, &x0, &x1);
+      const uint32_t n_sure = __reduce_add_sync(0xffffffffu, su);
+      const uint32_t r2 = k > n_sure ? k - n_sure : 1u;  // keys to take from the b1 bin
       int pc;
       uint32_t above_c, cnt_c;
       warp_find_desc2(x0, x1, r2, &pc, &above_c, &cnt_c);

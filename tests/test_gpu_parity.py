@@ -215,6 +215,27 @@ def test_indexer_topk_all_equal_scores_beyond_the_staging_buffer(fk):
         assert idx[0].tolist() == list(range(k)), k
 
 
+@pytest.mark.parametrize("n_equal", [40, 64, 65, 200])
+def test_indexer_topk_equal_top_keys_spread_over_the_cluster(fk, n_equal):
+    # n_equal copies of the best-scoring key row at random positions of a 200,000-entry
+    # sequence (the select's cluster splits it over several CTAs): the K-th key lies inside
+    # a bin of n_equal equal keys, which is ranked directly up to 64 keys and by the last-8-bit
+    # and position histograms beyond; either way the lowest K positions of the copies win
+    cap, k = 200000, 30
+    q, w, keys = _indexer_inputs(21, 1, cap, 32, True)
+    lens = torch.tensor([cap], dtype=torch.int32, device=DEV)
+    ref = P.oracle_scores_seq(q[0], w[0], keys[0], cap)
+    top = int(np.argmax(ref))
+    rng = np.random.default_rng(21 + n_equal)
+    others = rng.choice(np.setdiff1d(np.arange(cap), [top]), size=n_equal - 1, replace=False)
+    pos = np.sort(np.concatenate([[top], others]))
+    keys[0, torch.from_numpy(others).to(DEV)] = keys[0, top].clone()
+    score = torch.empty((1, k), dtype=torch.float32, device=DEV)
+    idx = fk.indexer_topk(q, w, keys, lens, k, out_score=score).cpu().numpy()
+    assert idx[0].tolist() == pos[:k].tolist()
+    assert np.all(score.cpu().numpy()[0] == np.float32(score.cpu().numpy()[0, 0]))
+
+
 def test_reindex_with_a_pool_in_arbitrary_order(fk):
     # pool blocks listed out of position order: the output is still ascending positions
     B, cap, k, npb = 2, 20000, 300, 96
