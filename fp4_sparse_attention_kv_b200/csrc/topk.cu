@@ -14,7 +14,7 @@
 //  1. every CTA finds the digit-1 value b1 of the K-th largest key from the histogram, as a
 //     float threshold: "digit 1 >= b1" is v >= f_lo;
 //  2. each warp reads only the groups of its sub-slice whose largest key reaches b1 (a few
-//     percent of them for the top 2048 of a million), 16 groups in flight at a time, keeps
+//     percent of them for the top 2048 of a million), 24 groups in flight at a time, keeps
 //     the values >= f_lo in position order (a ballot prefix, no block barrier) in its own
 //     list, and the CTA histograms the next 12 key bits (digit 2) of the keys with
 //     digit 1 == b1;
