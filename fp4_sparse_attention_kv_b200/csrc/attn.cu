@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     if (threadIdx.x == 0) atomicOr(p.status, kFlagMisaligned);
     return;
   }
-  // The merge kernel that follows waits for this grid to complete; let it be scheduled now.
+  // The kernel that follows on the stream waits for this grid to complete; let it be
+  // scheduled now.
   griddep_launch_dependents();
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   float* sC = reinterpret_cast<float*>(smem + kOffC);

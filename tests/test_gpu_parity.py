@@ -202,9 +202,9 @@ def test_indexer_topk_ties_go_to_the_lowest_positions(fk):
 
 
 def test_indexer_topk_all_equal_scores_beyond_the_staging_buffer(fk):
-    # 20000 equal scores: every entry survives both radix digits, so the final selection
-    # runs over more entries than the finishing CTA stages in shared memory and is decided
-    # by position alone
+    # 20000 equal scores: every entry survives both radix digits and the last 8 key bits,
+    # so the selection is decided by the position histograms alone, over more kept entries
+    # than the warps hold in shared memory (the rest overflow to the workspace)
     cap = 20000
     q, w, _ = _indexer_inputs(9, 1, cap, 32, True)
     row = synth.indexer_keys(9, 0, torch.arange(1, dtype=torch.int64), 128, True)
