@@ -18,13 +18,17 @@
 //     the values >= f_lo in position order (a ballot prefix, no block barrier) in its own
 //     list, and the CTA histograms the next 12 key bits (digit 2) of the keys with
 //     digit 1 == b1;
-//  3. the CTAs add up the digit-2 histograms through distributed shared memory (CTA r sums
-//     segment r of the bins in place) and every CTA finds the digit-2 value b2 of the K-th key;
-//  4. only when the (b1, b2) bin is taken in part: the last 8 key bits, then the lowest
-//     positions among the keys equal to the K-th key, are resolved the same way;
-//  5. every CTA counts what it takes, reads the counts of the CTAs before it and writes its
-//     positions at that offset: ascending without a sort. A Reindex pool whose blocks are not
-//     in ascending order gathers its at most 4096 selected pairs in CTA 0, which sorts them.
+//  3. after one cluster barrier, warp 0 of every CTA adds up the CTAs' coarse digit-2 bins
+//     (digit 2 / 64) and then the 64 fine bins of the coarse bin that holds the K-th key,
+//     through distributed shared memory, and finds its digit-2 value b2 (no second barrier);
+//  4. when the (b1, b2) bin is taken in part and holds at most 64 keys, every CTA publishes
+//     those keys (rank value: key, then lower position) with its count of certain
+//     selections; a larger bin is resolved by histograms of the last 8 key bits and then of
+//     the positions among the keys equal to the K-th key, one cluster barrier each;
+//  5. after the next barrier every CTA ranks the published keys, reads the counts of the CTAs
+//     before it and writes its positions at that offset: ascending without a sort. A Reindex
+//     pool whose blocks are not in ascending order gathers its at most 4096 selected pairs in
+//     CTA 0, which sorts them.
 // The CTAs also clear the scoring kernel's histogram for the next call. Cluster barriers are
 // the only synchronisation between CTAs; nothing waits on a flag.
 // Kernels that live a few microseconds run mostly from a cold instruction cache, so the loop
@@ -55,7 +59,7 @@ struct SelectArgs {
 
 struct SelSmem {
   uint64_t pairs[kMaxSel];              // pool mode: (position, value index), CTA 0 sorts them
-  uint32_t h2[kHistBins];               // digit-2 histogram; segment r is summed in place
+  uint32_t h2[kHistBins];               // digit 2 of this CTA's kept keys with digit 1 = b1
   uint64_t list[kWarps][kWarpCap];      // kept entries: (order key << 32) | value index
   uint32_t cand[kWarps][kCandCap];      // candidate groups of a round, in position order
   uint32_t h2c[64];                     // the same keys' digit 2 / 64 (coarse digit-2 bins)
@@ -72,7 +76,7 @@ struct SelSmem {
   uint32_t w[kWarps];                   // block scans
   uint32_t res[4];
   uint32_t sure;                        // keys of this CTA with digit 1 > b1
-  uint32_t sel_total;                   // entries this CTA selects
+  uint32_t sel_total;                   // entries this CTA takes for certain (before the small-bin ranking)
   uint32_t bc[4];                       // block broadcasts
 };
 constexpr size_t kSelSmem = sizeof(SelSmem);
