@@ -757,10 +757,10 @@ cudaError_t launch_topk_select(const SelectProblem* probs, int n_probs, int B, i
   cudaError_t e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSelSmem));
   if (e != cudaSuccess) return e;
-  // CTAs per sequence: a power of two up to 16, at least 4096 values each, the whole grid
+  // CTAs per sequence: a power of two up to 16, at least 2048 values each, the whole grid
   // within about one CTA per SM, and every cluster resident at once
   int cluster = 1;
-  while (cluster < kMaxCluster && n_max / (2 * cluster) >= 4096 &&
+  while (cluster < kMaxCluster && n_max / (2 * cluster) >= 2048 &&
          int64_t(B) * n_probs * 2 * cluster <= num_sms)
     cluster *= 2;
   while (cluster > 1) {
