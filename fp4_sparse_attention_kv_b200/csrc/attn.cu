@@ -22,8 +22,12 @@
 //
 // Kernel (one CTA per (chunk of the index list, group of 64 heads, sequence); 13 warps):
 //  * the tile is 128 selected entries. S^T = V_hat Q^T (M = 128 entries, N = 64 heads,
-//    K = 512) and O^T += V_hat^T P^T (M = 128 dims x 4, N = 64 heads, K = 128 entries) run on
-//    tcgen05 with fp32 accumulators in TMEM (O^T: 256 columns; S^T: two 64-column slots).
+//    K = 512) and O^T += V_hat^T P^T (M = 128 dims x 4, K = 128 entries) run on tcgen05 with
+//    fp32 accumulators in TMEM. An MMA costs the same for N = 64 and N = 128, so for three of
+//    the four dim tiles P_hi and P_lo are one N = 128 operand (heads, then the same heads
+//    again) with separate accumulators that are added at the end; the fourth dim tile, for
+//    which the 512 TMEM columns have no room left beside S^T, takes two N = 64 MMAs per step
+//    into one accumulator.
 //  * warps 8-11 gather: each thread loads one selected row (256 B codes + 32 B scales) with
 //    16-byte loads, dequantizes it 64 dims at a time into a 128-byte-swizzled fp16 chunk
 //    buffer (8 chunks = the tile's 128 KiB V_hat) that serves as the K-major A operand of
@@ -91,8 +95,13 @@ static_assert(kSmemAttn <= 232448, "shared memory");
 // At the end the V_hat region holds the [64 heads][512 dims] fp32 output tile.
 static_assert(kChunks * kVChunkBytes == kHeadsPerCta * kD * 4, "output staging");
 
-// TMEM columns: O^T dim-tile c at [64c, 64c + 64); S^T slot u at [256 + 64u, +64)
-constexpr uint32_t kColS = 256;
+// TMEM columns: O^T of dim tile c < 3 at [128c, +64) (P_hi) and [128c + 64, +64) (P_lo);
+// dim tile 3 at [384, 448) (both halves); S^T at [448, 512). One S^T slot is enough: S^T of
+// tile t + 1 needs V_hat rows that only the end of P.V(t) frees, and P.V(t) starts after
+// every softmax warp has read S^T(t).
+constexpr uint32_t kColS = 448;
+constexpr int kPairTiles = 3;  // dim tiles with separate P_hi and P_lo accumulators
+FP4KV_DEV uint32_t o_col(int c) { return 128u * static_cast<uint32_t>(c); }
 static_assert(4096 / kTile <= 32, "the per-thread validity mask holds one bit per tile");
 
 enum { B_VREADY = 0, B_VFREE = 8, B_SFULL = 16, B_SFREE = 18, B_PREADY = 20, B_PFREE = 21,
@@ -429,10 +438,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       mbar_init(&bars[B_VREADY + j], kGatherWarps + kSoftWarps);
       mbar_init(&bars[B_VFREE + j], 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(&bars[B_SFULL + u], 1);
-      mbar_init(&bars[B_SFREE + u], kSoftWarps);
-    }
+    mbar_init(&bars[B_SFULL], 1);
+    mbar_init(&bars[B_SFREE], kSoftWarps);
     mbar_init(&bars[B_PREADY], kSoftWarps);
     mbar_init(&bars[B_PFREE], 1);
     mbar_init(&bars[B_QREADY], kSoftWarps);
@@ -488,6 +495,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     if (lane == 0) {
       constexpr uint32_t kIdescQK = umma_idesc(0u, 128, kHeadsPerCta, 0u, 0u);
       constexpr uint32_t kIdescPV = umma_idesc(0u, 128, kHeadsPerCta, 1u, 1u);
+      constexpr uint32_t kIdescPV2 = umma_idesc(0u, 128, 2 * kHeadsPerCta, 1u, 1u);
       // Descriptors are built once; each MMA adds its operand offset in 16-byte units to the
       // start-address field (shared-memory addresses stay below 2^18 bytes, so the 14-bit
       // field never carries). A single thread issues ~50 cycles apart at best for N = 64,
@@ -501,13 +509,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       if (!ok) fail_wait(p, s_abort);
       for (int t = 0; ok && t < n_tiles; ++t) {
         if (*s_abort) break;
-        const int u = t & 1;
-        if (!mbar_wait_timed(&bars[B_SFREE + u], ((t >> 1) & 1) ^ 1)) {
+        if (!mbar_wait_timed(&bars[B_SFREE], (t & 1) ^ 1)) {
           fail_wait(p, s_abort);
           break;
         }
         tc_fence_after();
-        const uint32_t ds = tmem + kColS + 64u * u;
+        const uint32_t ds = tmem + kColS;
         // (loops kept rolled: their first pass runs from a cold instruction cache)
 #pragma unroll 1
         for (int jc = 0; jc < kChunks && ok; ++jc) {
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
           fail_wait(p, s_abort);
           break;
         }
-        umma_commit(&bars[B_SFULL + u]);
+        umma_commit(&bars[B_SFULL]);
         if (!mbar_wait_timed(&bars[B_PREADY], t & 1)) {
           fail_wait(p, s_abort);
           break;
@@ -536,13 +543,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         const bool acc0 = t > 0;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          const uint32_t d = tmem + 64u * c;
+          const uint32_t d = tmem + o_col(c);
+          if (c < kPairTiles) {
+            // N = 128: P_hi's 64 heads, then P_lo's (the operand's second 64-element block
+            // along N lies kPBytes further, where P_lo is)
 #pragma unroll 2
-          for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
-            const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
-            const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
-            umma_f16(d, a, dph + ko, kIdescPV, acc0 || s > 0);
-            umma_f16(d, a, dpl + ko, kIdescPV, true);
+            for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
+              const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
+              const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
+              umma_f16(d, a, dph + ko, kIdescPV2, acc0 || s > 0);
+            }
+          } else {
+#pragma unroll 2
+            for (int s = 0; s < kTile / 16; ++s) {
+              const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
+              const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
+              umma_f16(d, a, dph + ko, kIdescPV, acc0 || s > 0);
+              umma_f16(d, a, dpl + ko, kIdescPV, true);
+            }
           }
           umma_commit(&bars[B_VFREE + 2 * c]);
           umma_commit(&bars[B_VFREE + 2 * c + 1]);
@@ -646,19 +664,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
                                               : load_dequant<1>(smem, bars, packed_b, scales_b, dp, drow, 0));
     }
     for (int t = 0; t < n_tiles; ++t) {
-      const int u = t & 1;
       const bool valid = (vmask >> t) & 1u;
-      bool f = !softmax_wait(&bars[B_SFULL + u], (t >> 1) & 1);
+      bool f = !softmax_wait(&bars[B_SFULL], t & 1);
       float z[32];
       bool over = false;
       if (!f) {
         tc_fence_after();
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kColS + 64u * u + h0, r);
+        tmem_ld32(tmem + lane_addr + kColS + h0, r);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_SFREE + u]);
+        if (lane == 0) mbar_arrive(&bars[B_SFREE]);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           z[j] = valid ? __uint_as_float(r[j]) * sC[h0 + j] : -INFINITY;
@@ -703,11 +720,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
           moved |= a != 1.0f;
         }
         if (t > 0 && moved) {  // rescale this thread's O^T elements of the moved heads
+          // (16 columns at a time: dim tiles 0-2 hold two accumulators, dim tile 3 one)
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 2 * (2 * kPairTiles + 1); ++c) {
             uint32_t r[16];
-            const int j0 = 16 * (c & 1);
-            const uint32_t addr = tmem + lane_addr + 64u * (c >> 1) + h0 + j0;
+            const int j0 = 16 * (c & 1), blk = c >> 1;
+            const uint32_t col = blk < 2 * kPairTiles ? o_col(blk >> 1) + 64u * (blk & 1) : o_col(kPairTiles);
+            const uint32_t addr = tmem + lane_addr + col + h0 + j0;
             tmem_ld16(addr, r);
             tmem_ld_wait();
 #pragma unroll
@@ -766,8 +785,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         }
         if (have) {
           tc_fence_after();
-          tmem_ld32(tmem + lane_addr + 64u * c + h0, r);
-          tmem_ld_wait();
+          tmem_ld32(tmem + lane_addr + o_col(c) + h0, r);
+          if (c < kPairTiles) {  // the P_lo accumulator of this dim tile
+            uint32_t r2[32];
+            tmem_ld32(tmem + lane_addr + o_col(c) + 64u + h0, r2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) + __uint_as_float(r2[k]));
+          } else {
+            tmem_ld_wait();
+          }
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) r[k] = 0u;
