@@ -37,7 +37,8 @@
 //    heads 32 (w / 4) .. + 32): per tile each thread reads its entry's 32 logits, keeps 32
 //    per-head running row sums in registers, and writes its half of the entry's row of P^T
 //    (MN-major B operand). Cross-lane reductions happen only when a reference moves and
-//    once at the end, when O^T is staged in shared memory and leaves in one bulk store.
+//    once at the end, for the per-head row sums; each thread writes its TMEM lane of O^T
+//    straight to the workspace.
 //  Per-chunk barriers let the next tile's dequantization overlap the current tile's P.V.
 //  * Chunks of the index list go to different CTAs, and the chunk CTAs of one (sequence,
 //    head group) form one thread-block cluster. At the end each writes its partial (O and
