@@ -209,7 +209,7 @@ FP4KV_DEV bool load_dequant(uint8_t* smem, uint64_t* bars, const uint8_t* packed
       const uint8_t* prow = packed_b + int64_t(pos[i]) * (kD / 2) + 16 * j;
 #pragma unroll
       for (int cp = 0; cp < 4; ++cp) pk[cp][i] = ld_nc_v4(prow + 64 * cp);
-      s8[i] = ld_nc_v2(scales_b + int64_t(pos[i]) * (kD / kGroup) + 8 * j);
+      s8[i] = ld_nc_v2_64b(scales_b + int64_t(pos[i]) * (kD / kGroup) + 8 * j);
     } else {
 #pragma unroll
       for (int cp = 0; cp < 4; ++cp) pk[cp][i] = make_uint4(0, 0, 0, 0);

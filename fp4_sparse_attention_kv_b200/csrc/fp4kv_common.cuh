@@ -168,9 +168,11 @@ FP4KV_DEV uint4 ld_nc_v4(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
-FP4KV_DEV uint2 ld_nc_v2(const void* p) {
+// 8 bytes of a randomly addressed 32-byte record: the 64-byte L2 fetch hint halves what a
+// miss brings from DRAM (a miss otherwise fills a whole 128-byte line)
+FP4KV_DEV uint2 ld_nc_v2_64b(const void* p) {
   uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  asm volatile("ld.global.nc.L1::no_allocate.L2::64B.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
   return r;
 }
 FP4KV_DEV uint4 ld_stream_v4(const void* p) {
