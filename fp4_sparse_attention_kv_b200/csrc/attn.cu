@@ -493,7 +493,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // The whole warp waits (every lane polls the mbarrier: one lane polling and then
+    // broadcasting resumed the warp measurably later); lane 0 issues the MMAs and commits.
+    {
       constexpr uint32_t kIdescQK = umma_idesc(0u, 128, kHeadsPerCta, 0u, 0u);
       constexpr uint32_t kIdescPV = umma_idesc(0u, 128, kHeadsPerCta, 1u, 1u);
       constexpr uint32_t kIdescPV2 = umma_idesc(0u, 128, 2 * kHeadsPerCta, 1u, 1u);
@@ -506,71 +508,77 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       const uint64_t dvm = sw128_mnmajor_desc(smem_u32(smem + kOffV), kVChunkBytes);
       const uint64_t dph = sw128_mnmajor_desc(smem_u32(smem + kOffPh), kPBytes);
       const uint64_t dpl = sw128_mnmajor_desc(smem_u32(smem + kOffPl), kPBytes);
-      bool ok = mbar_wait_timed(&bars[B_QREADY], 0);
-      if (!ok) fail_wait(p, s_abort);
+      const bool issuer = lane == 0;
+      bool ok = __all_sync(0xffffffffu, mbar_wait_timed(&bars[B_QREADY], 0));
+      if (!ok && issuer) fail_wait(p, s_abort);
       for (int t = 0; ok && t < n_tiles; ++t) {
-        if (*s_abort) break;
-        if (!mbar_wait_timed(&bars[B_SFREE], (t & 1) ^ 1)) {
-          fail_wait(p, s_abort);
+        if (__shfl_sync(0xffffffffu, *s_abort, 0)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_SFREE], (t & 1) ^ 1))) {
+          if (issuer) fail_wait(p, s_abort);
           break;
         }
-        tc_fence_after();
         const uint32_t ds = tmem + kColS;
         // (loops kept rolled: their first pass runs from a cold instruction cache)
 #pragma unroll 1
         for (int jc = 0; jc < kChunks && ok; ++jc) {
-          if (!mbar_wait_timed(&bars[B_VREADY + jc], t & 1)) {
+          if (!__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_VREADY + jc], t & 1))) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint64_t a = dvk + static_cast<uint64_t>((jc * kVChunkBytes) >> 4);
-          const uint64_t bq = dq + static_cast<uint64_t>((jc * kQChunkBytes) >> 4);
-          umma_f16(ds, a, bq, kIdescQK, jc != 0);  // K steps of 16 elements = 32 bytes
-          umma_f16(ds, a + 2, bq + 2, kIdescQK, true);
-          umma_f16(ds, a + 4, bq + 4, kIdescQK, true);
-          umma_f16(ds, a + 6, bq + 6, kIdescQK, true);
+          if (issuer) {
+            tc_fence_after();
+            const uint64_t a = dvk + static_cast<uint64_t>((jc * kVChunkBytes) >> 4);
+            const uint64_t bq = dq + static_cast<uint64_t>((jc * kQChunkBytes) >> 4);
+            umma_f16(ds, a, bq, kIdescQK, jc != 0);  // K steps of 16 elements = 32 bytes
+            umma_f16(ds, a + 2, bq + 2, kIdescQK, true);
+            umma_f16(ds, a + 4, bq + 4, kIdescQK, true);
+            umma_f16(ds, a + 6, bq + 6, kIdescQK, true);
+          }
+          __syncwarp();
         }
         if (!ok) {
-          fail_wait(p, s_abort);
+          if (issuer) fail_wait(p, s_abort);
           break;
         }
-        umma_commit(&bars[B_SFULL]);
-        if (!mbar_wait_timed(&bars[B_PREADY], t & 1)) {
-          fail_wait(p, s_abort);
+        if (issuer) umma_commit(&bars[B_SFULL]);
+        if (!__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_PREADY], t & 1))) {
+          if (issuer) fail_wait(p, s_abort);
           break;
         }
-        tc_fence_after();
-        const bool acc0 = t > 0;
+        if (issuer) {
+          tc_fence_after();
+          const bool acc0 = t > 0;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t d = tmem + o_col(c);
-          if (c < kPairTiles) {
-            // N = 128: P_hi's 64 heads, then P_lo's (the operand's second 64-element block
-            // along N lies kPBytes further, where P_lo is)
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t d = tmem + o_col(c);
+            if (c < kPairTiles) {
+              // N = 128: P_hi's 64 heads, then P_lo's (the operand's second 64-element block
+              // along N lies kPBytes further, where P_lo is)
 #pragma unroll 2
-            for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
-              const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
-              const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
-              umma_f16(d, a, dph + ko, kIdescPV2, acc0 || s > 0);
-            }
-          } else {
+              for (int s = 0; s < kTile / 16; ++s) {  // 16 entries = 2048 bytes of K per step
+                const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
+                const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
+                umma_f16(d, a, dph + ko, kIdescPV2, acc0 || s > 0);
+              }
+            } else {
 #pragma unroll 2
-            for (int s = 0; s < kTile / 16; ++s) {
-              const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
-              const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
-              umma_f16(d, a, dph + ko, kIdescPV, acc0 || s > 0);
-              umma_f16(d, a, dpl + ko, kIdescPV, true);
+              for (int s = 0; s < kTile / 16; ++s) {
+                const uint64_t a = dvm + static_cast<uint64_t>((2 * c * kVChunkBytes + 2048 * s) >> 4);
+                const uint64_t ko = static_cast<uint64_t>((2048 * s) >> 4);
+                umma_f16(d, a, dph + ko, kIdescPV, acc0 || s > 0);
+                umma_f16(d, a, dpl + ko, kIdescPV, true);
+              }
             }
+            umma_commit(&bars[B_VFREE + 2 * c]);
+            umma_commit(&bars[B_VFREE + 2 * c + 1]);
           }
-          umma_commit(&bars[B_VFREE + 2 * c]);
-          umma_commit(&bars[B_VFREE + 2 * c + 1]);
+          umma_commit(&bars[B_PFREE]);
         }
-        umma_commit(&bars[B_PFREE]);
+        __syncwarp();
       }
       // every MMA issued above completes before TMEM is released
-      umma_commit(&bars[B_DONE]);
-      if (!mbar_wait_timed(&bars[B_DONE], 0)) fail_wait(p, s_abort);
+      if (issuer) umma_commit(&bars[B_DONE]);
+      if (!__all_sync(0xffffffffu, mbar_wait_timed(&bars[B_DONE], 0)) && issuer) fail_wait(p, s_abort);
     }
     __syncwarp();
   } else {

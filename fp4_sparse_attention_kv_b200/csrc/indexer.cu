@@ -494,7 +494,9 @@ __global__ void __launch_bounds__(kThreads, ScanCfg<KT, N>::kCtasPerSm)
       // histogram flushes (named barriers) and none is left waiting at one alone.
       bool live = __shfl_sync(0xffffffffu, *s_abort, 0) == 0u;
       if (live) {
-        live = mbar_wait_warp(&tfull[acc], aph);
+        // (every lane polls: a wait polled by lane 0 alone and then broadcast resumed the warp
+        // measurably later, and the epilogue's wait is on the scan's per-tile path)
+        live = __all_sync(0xffffffffu, mbar_wait_timed(&tfull[acc], aph));
         if (!live && lane == 0) {
           atomicOr(p.status, kFlagWaitTimeout);
           *s_abort = 1;
