@@ -408,12 +408,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
         const uint32_t bal = __ballot_sync(0xffffffffu, keep);
         if (keep) {
           const uint32_t key = order_key(v[q]);
-          if (digit1(key) == b1) {
-            atomicAdd(&S.h2[digit2(key)], 1u);
-            atomicAdd(&S.h2c[digit2(key) >> 6], 1u);
-          } else {
-            ++sure;  // (kept keys have digit 1 >= b1)
-          }
           const uint32_t o = run + __popc(bal & below);
           const uint64_t e = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(wlo + 32 * int64_t(gq[q]) + lane);
           if (o < static_cast<uint32_t>(kWarpCap)) S.list[warp][o] = e;
@@ -423,6 +417,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
       }
     }
     __syncwarp();  // the candidate list is read before the next round rewrites it
+  }
+  // the digit-2 histograms of the kept keys with digit 1 == b1 and the count of those above
+  // it, one kept entry per lane (inside the loop above, the histogram atomics ran with one or
+  // two lanes active per group and cost ~2 us of the select on 1 M values)
+  for (uint32_t j = lane; j < run; j += 32) {
+    const uint32_t key = ent_key(j < static_cast<uint32_t>(kWarpCap) ? S.list[warp][j] : glist[wlo + j]);
+    if (digit1(key) == b1) {
+      atomicAdd(&S.h2[digit2(key)], 1u);
+      atomicAdd(&S.h2c[digit2(key) >> 6], 1u);
+    } else {
+      ++sure;  // (kept keys have digit 1 >= b1)
+    }
   }
   sure = __reduce_add_sync(0xffffffffu, sure);
   if (lane == 0) {
