@@ -119,6 +119,16 @@ FP4KV_DEV bool softmax_any(bool v) {
   return r != 0;
 }
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32: a few units
+// in the last place, results below 2^-126 flushed to zero). The probabilities are at most
+// 2^9 and feed a sum of at least 1, so neither the approximation nor the flush is visible
+// beside the fp16 hi / lo split of P.
+FP4KV_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Butterfly transpose-reduction of 32 values per lane across the warp: on return, lane l
 // holds the reduction over all 32 lanes of value l.
 template <bool kMax>
@@ -755,8 +765,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         for (int k = 0; k < 4; ++k) {
           const int j = 8 * unit + 2 * k;
           const float m0 = sM[h0 + j], m1 = sM[h0 + j + 1];
-          const float p0 = m0 == -INFINITY ? 0.0f : exp2f(z[j] - m0);
-          const float p1 = m1 == -INFINITY ? 0.0f : exp2f(z[j + 1] - m1);
+          const float p0 = m0 == -INFINITY ? 0.0f : ex2_approx(z[j] - m0);
+          const float p1 = m1 == -INFINITY ? 0.0f : ex2_approx(z[j + 1] - m1);
           lsum[j] += p0;
           lsum[j + 1] += p1;
           const float a = p0 * kPScale, c2 = p1 * kPScale;

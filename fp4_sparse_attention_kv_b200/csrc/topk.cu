@@ -14,7 +14,7 @@
 //  1. every CTA finds the digit-1 value b1 of the K-th largest key from the histogram, as a
 //     float threshold: "digit 1 >= b1" is v >= f_lo;
 //  2. each warp reads only the groups of its sub-slice whose largest key reaches b1 (a few
-//     percent of them for the top 2048 of a million), 24 groups in flight at a time, keeps
+//     percent of them for the top 2048 of a million), 16 groups in flight at a time, keeps
 //     the values >= f_lo in position order (a ballot prefix, no block barrier) in its own
 //     list, and the CTA histograms the next 12 key bits (digit 2) of the keys with
 //     digit 1 == b1;
@@ -44,7 +44,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 24;                // 32-value groups a warp loads at once
+constexpr int kBatch = 16;                // 32-value groups a warp loads at once
 constexpr int kWords = 8;                 // 32-group words of group maxima loaded at once
 constexpr int kCandCap = 32 * kWords;     // candidate groups a warp lists per round
 constexpr int kWarpCap = 256;             // kept entries per warp held in shared memory
@@ -151,6 +151,15 @@ FP4KV_DEV void cluster_sum2(const uint32_t* p0, const uint32_t* p1, uint32_t C, 
   }
   *s0 = a;
   *s1 = c;
+}
+
+// An L2 load the compiler keeps in program order (volatile, with a memory clobber): a batch's
+// loads are then all in flight before the first of them is consumed, which the compiler
+// otherwise does not guarantee under this kernel's register limit
+FP4KV_DEV float ld_cg_ordered(const float* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
 }
 
 FP4KV_DEV uint32_t warp_incl_scan(uint32_t x) {
@@ -399,7 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_select(const SelectArgs ar
       for (int q = 0; q < kBatch; ++q) {
         gq[q] = c0 + q < n_cand ? static_cast<int32_t>(S.cand[warp][c0 + q]) : -1;
         const int64_t i = wlo + 32 * int64_t(gq[q]) + lane;
-        v[q] = (gq[q] >= 0 && i < whi) ? __ldcg(vals + i) : -INFINITY;
+        v[q] = -INFINITY;
+        if (gq[q] >= 0 && i < whi) v[q] = ld_cg_ordered(vals + i);
       }
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
