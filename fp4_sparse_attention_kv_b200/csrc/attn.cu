@@ -121,8 +121,9 @@ FP4KV_DEV bool softmax_any(bool v) {
 
 // 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32: a few units
 // in the last place, results below 2^-126 flushed to zero). The probabilities are at most
-// 2^9 and feed a sum of at least 1, so neither the approximation nor the flush is visible
-// beside the fp16 hi / lo split of P.
+// 2^9 and feed a sum of at least 1, and the combine's chunk weights are at most 1 with the
+// largest exactly 1, so neither the approximation nor the flush is visible beside the fp16
+// hi / lo split of P.
 FP4KV_DEV float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -372,7 +373,7 @@ FP4KV_DEV void combine_slice(const AttnParams& p, int b, int hbase, int nh, uint
       float w[C];
 #pragma unroll
       for (int c = 0; c < C; ++c) {
-        w[c] = ml[j][c].y > 0.0f ? exp2f(ml[j][c].x - M) : 0.0f;
+        w[c] = ml[j][c].y > 0.0f ? ex2_approx(ml[j][c].x - M) : 0.0f;
         Lt += w[c] * ml[j][c].y;
       }
       const float inv = Lt > 0.0f ? 1.0f / (kPScale * Lt) : 0.0f;
