@@ -90,7 +90,9 @@ constexpr uint32_t kOffRed = kOffC + 256;       // [4][64] cross-warp exchange
 constexpr uint32_t kOffM = kOffRed + 1024;      // [64] per-head reference (log2 domain)
 constexpr uint32_t kOffA = kOffM + 256;         // [64] rescale factor of the last move
 constexpr uint32_t kOffL = kOffA + 256;         // [64] row sums at the end
-constexpr uint32_t kOffTmem = kOffL + 256;
+constexpr uint32_t kOffMT = kOffL + 256;        // [64] reference + 9: a logit above it moves it
+constexpr uint32_t kOffM6 = kOffMT + 256;       // [64] reference - 6: 2^(z - it) is p * 2^6
+constexpr uint32_t kOffTmem = kOffM6 + 256;
 constexpr uint32_t kSmemAttn = kOffTmem + 16;
 static_assert(kSmemAttn <= 232448, "shared memory");
 // At the end the V_hat region holds the [64 heads][512 dims] fp32 output tile.
@@ -414,6 +416,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
   float* sM = reinterpret_cast<float*>(smem + kOffM);
   float* sA = reinterpret_cast<float*>(smem + kOffA);
   float* sL = reinterpret_cast<float*>(smem + kOffL);
+  float* sMT = reinterpret_cast<float*>(smem + kOffMT);
+  float* sM6 = reinterpret_cast<float*>(smem + kOffM6);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
   volatile uint32_t* s_abort = s_tmem + 1;
   volatile uint32_t* s_fail = s_tmem + 2;  // a softmax wait gave up: this CTA's partial is void
@@ -642,6 +646,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
         if (lane == 0) {
           sC[hh] = c;
           sM[hh] = -INFINITY;
+          sMT[hh] = -INFINITY;
+          sM6[hh] = -INFINITY;
         }
       }
       fence_proxy_async_smem();
@@ -699,7 +705,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           z[j] = valid ? __uint_as_float(r[j]) * sC[h0 + j] : -INFINITY;
-          over |= z[j] > sM[h0 + j] + kMoveLog2;
+          over |= z[j] > sMT[h0 + j];
         }
         // the previous tile's P.V must be complete before P is rewritten or O rescaled
         // (it precedes this tile's S in the tensor pipe, so this wait is normally free)
@@ -729,6 +735,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
             a = mo == -INFINITY ? 0.0f : exp2f(mo - mn);
           }
           sM[h] = mn;
+          sMT[h] = mn + kMoveLog2;
+          sM6[h] = mn - 6.0f;  // (kPScale = 2^6)
           sA[h] = a;
         }
         softmax_sync();
@@ -765,12 +773,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int j = 8 * unit + 2 * k;
-          const float m0 = sM[h0 + j], m1 = sM[h0 + j + 1];
-          const float p0 = m0 == -INFINITY ? 0.0f : ex2_approx(z[j] - m0);
-          const float p1 = m1 == -INFINITY ? 0.0f : ex2_approx(z[j + 1] - m1);
-          lsum[j] += p0;
-          lsum[j + 1] += p1;
-          const float a = p0 * kPScale, c2 = p1 * kPScale;
+          // p * 2^6 straight from the exponent; the row sums add the same scaled values and
+          // are scaled back by the exact 2^-6 at the end
+          const float m0 = sM6[h0 + j], m1 = sM6[h0 + j + 1];
+          const float a = m0 == -INFINITY ? 0.0f : ex2_approx(z[j] - m0);
+          const float c2 = m1 == -INFINITY ? 0.0f : ex2_approx(z[j + 1] - m1);
+          lsum[j] += a;
+          lsum[j + 1] += c2;
           hi[k] = pack_f16x2(a, c2);
           lo[k] = pack_f16x2(a - f16_lo_to_f32(hi[k]), c2 - f16_hi_to_f32(hi[k]));
         }
@@ -838,7 +847,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn_tc(const AttnPa
       softmax_sync();
       if (q4 == 0) {
         const int h = h0 + lane;
-        sL[h] = sRed[h] + sRed[64 + h] + sRed[128 + h] + sRed[192 + h];
+        sL[h] = (sRed[h] + sRed[64 + h] + sRed[128 + h] + sRed[192 + h]) * (1.0f / kPScale);
       }
     }
     if (tid == 0) *s_fail = fail ? 1u : 0u;
