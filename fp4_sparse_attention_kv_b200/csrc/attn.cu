@@ -188,12 +188,9 @@ FP4KV_DEV bool gather_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait_timed(bar, parity));
 #endif
 }
+// (every lane polls: one lane polling and broadcasting resumed the warp measurably later)
 FP4KV_DEV bool softmax_wait(uint64_t* bar, uint32_t parity) {
-#ifdef ATTN_SOFTMAX_LANE0
-  return mbar_wait_warp(bar, parity);
-#else
   return __all_sync(0xffffffffu, mbar_wait_timed(bar, parity));
-#endif
 }
 
 FP4KV_DEV void fail_wait(const AttnParams& p, volatile uint32_t* abort_flag) {

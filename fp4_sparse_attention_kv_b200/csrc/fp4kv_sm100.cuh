@@ -42,17 +42,6 @@ FP4KV_DEV bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, uint32_t ns) {
   }
 }
 
-// Warp-collective bounded wait: lane 0 alone polls the mbarrier (the other lanes add no
-// shared-memory polling traffic), then the warp synchronizes, which orders every lane's
-// later accesses after lane 0's acquire. Returns the same result in every lane.
-FP4KV_DEV bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
-  uint32_t ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_timed(bar, parity) ? 1u : 0u;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
-}
-
 // ---------------------------------------------------------------------------------------
 // TMA (tiled tensor map) load into shared memory, completing on an mbarrier
 // ---------------------------------------------------------------------------------------
