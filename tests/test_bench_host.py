@@ -119,3 +119,29 @@ def test_layered_oracle_sample_runs_every_layer_on_a_small_case():
     finally:
         O.hier_pool_select, O.reindex_topk, O.sparse_attn_decode_rows = orig
     assert work == 1.0 and calls == {"hier": 1, "reindex": 3, "attn": 6}
+
+
+def test_traffic_records_are_current_or_ignored_and_near_the_algorithmic_bytes():
+    """profiles/traffic.txt: a record is used only while its kernel source digest matches; every
+    record that matches carries DRAM bytes between 1.0x and 1.5x of the launch's algorithmic
+    bytes (keys for the scan; gathered rows for the attention), so a record copied to the
+    wrong workload or a capture of the wrong kernel fails here."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cfgs = bench.CONFIGS
+    key_bytes = {"index_score": lambda c: c["B"] * c["cap"] * (128 if c.get("fp8") else 256),
+                 "sparse_attn": lambda c: c["B"] * c["K"] * bench.ROW_BYTES}
+    checked = 0
+    for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
+        if not line.startswith("kernel="):
+            continue
+        rec = dict(kv.split("=", 1) for kv in line.split())
+        got = bench.traffic_record(rec["kernel"], rec["workload"])
+        if got is None:  # the kernel has changed since the capture: the bench reports null
+            continue
+        assert got == float(rec["dram_bytes_per_launch"])
+        alg = key_bytes[rec["kernel"]](cfgs[rec["workload"]])
+        assert 1.0 <= got / alg <= 1.5, (rec, got / alg)
+        checked += 1
+    assert bench.traffic_record("sparse_attn", "no_such_workload") is None
+    assert checked >= 1
